@@ -1,0 +1,435 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix.
+
+Each test checks the oracle against something other than itself: a published
+test vector or table, an independent construction, a closed form, an
+invariant, brute force on tiny inputs, or a Monte-Carlo expectation.  They are
+chosen so that a plausible slip in the oracle (a dropped term, a wrong sign or
+index, a transposed operand, a wrong scale) fails at least one of them.
+"""
+import math
+
+import mpmath
+import numpy as np
+import pytest
+from scipy import stats
+
+import oracle as O
+import synth
+from conftest import golden_path
+
+
+# ------------------------------------------------------------------ random draws
+def test_splitmix64_reference_outputs():
+    want = [int(l, 16) for l in open(golden_path("splitmix64_state0.txt")) if l.startswith("0x")]
+    assert O.splitmix64(0, 3) == want
+
+
+def test_rademacher_signs_follow_top_bit():
+    outs = O.splitmix64(7, 256)
+    D = O.rademacher_signs(7, 256)
+    assert set(np.unique(D)) == {-1.0, 1.0}
+    # top bit set <=> the integer is at least 2^63
+    assert all((D[i] < 0) == (outs[i] >= 2 ** 63) for i in range(256))
+    assert abs(np.mean(D)) < 0.2
+
+
+def test_gaussian_sketch_is_standard_normal():
+    S = O.gaussian_sketch(3, 64, 512).astype(np.float64).ravel()
+    assert S.dtype == np.float64 and S.size == 64 * 512
+    ks = stats.kstest(S, "norm")
+    assert ks.pvalue > 1e-3, ks
+    assert abs(S.mean()) < 0.02 and abs(S.var() - 1) < 0.02
+    # the D stream and the S stream are different streams of the same seed
+    assert not np.allclose(O.gaussian_sketch(3, 1, 8), O.gaussian_sketch(4, 1, 8))
+
+
+def test_sketch_is_row_major_m_by_d():
+    # entry (j, i) comes from the output pair 2*(j*d + i), 2*(j*d + i) + 1
+    m, d = 3, 8
+    S = O.gaussian_sketch(5, m, d)
+    outs = O.splitmix64(5 ^ O.S_SEED_XOR, 2 * m * d)
+    j, i = 2, 5
+    k = j * d + i
+    u1 = ((outs[2 * k] >> 11) + 1) / 2.0 ** 53
+    u2 = (outs[2 * k + 1] >> 11) / 2.0 ** 53
+    # a Box-Muller normal from (u1, u2) has |g| <= sqrt(-2 ln u1)
+    assert abs(S[j, i]) <= math.sqrt(-2 * math.log(u1)) * (1 + 1e-6)
+    assert np.sign(S[j, i]) == np.sign(math.cos(2 * math.pi * u2))
+
+
+# --------------------------------------------------------------------- rotation
+def _kron_hadamard(n):
+    H = np.array([[1.0]])
+    while H.shape[0] < n:
+        H = np.block([[H, H], [H, -H]])
+    return H
+
+
+@pytest.mark.parametrize("n", [2, 8, 64, 128, 512])
+def test_hadamard_matches_sylvester_recursion(n):
+    assert np.array_equal(O.sylvester_hadamard(n), _kron_hadamard(n))
+
+
+def test_hadamard_8_literal():
+    H8 = O.sylvester_hadamard(8)
+    # rows of H_8 in Sylvester order, written out
+    lit = ["++++++++", "+-+-+-+-", "++--++--", "+--++--+",
+           "++++----", "+-+--+-+", "++----++", "+--+-++-"]
+    want = np.array([[1.0 if c == "+" else -1.0 for c in r] for r in lit])
+    assert np.array_equal(H8, want)
+    assert np.array_equal(H8 @ H8, 8 * np.eye(8))
+
+
+@pytest.mark.parametrize("d", [8, 64, 128, 1536])
+def test_rotation_is_orthogonal(d):
+    D = O.rademacher_signs(11, d)
+    Pi = O.rotation_matrix(D)
+    assert np.abs(Pi @ Pi.T - np.eye(d)).max() < 1e-12
+    rng = np.random.default_rng(0)
+    x, y = rng.standard_normal((2, d)) * 3
+    assert abs(np.linalg.norm(Pi @ x) - np.linalg.norm(x)) < 1e-12 * np.linalg.norm(x)
+    assert abs((Pi @ x) @ (Pi @ y) - x @ y) < 1e-12 * np.linalg.norm(x) * np.linalg.norm(y)
+
+
+def test_rotation_spreads_an_outlier():
+    # a single-channel spike is spread evenly over all rotated coordinates
+    d = 128
+    Pi = O.rotation_matrix(O.rademacher_signs(0, d))
+    e = np.zeros(d)
+    e[17] = 100.0
+    y = Pi @ e
+    assert np.allclose(np.abs(y), 100.0 / math.sqrt(d), atol=1e-12)
+
+
+def test_rope_before_rotation_keeps_scores():
+    # TurboESM, "Resumo tecnico" section 2: RoPE first, then Pi; Pi^T Pi = I
+    d = 64
+    rng = np.random.default_rng(3)
+    q, k = rng.standard_normal((2, 5, d))
+    pos = np.array([0, 1, 17, 400, 4095])
+    qr = synth.rope_rotate_half(q, pos, 10000.0)
+    kr = synth.rope_rotate_half(k, pos, 10000.0)
+    Pi = O.rotation_matrix(O.rademacher_signs(1, d))
+    lhs = np.einsum("td,td->t", qr @ Pi.T, kr @ Pi.T)
+    rhs = np.einsum("td,td->t", qr, kr)
+    assert np.abs(lhs - rhs).max() < 1e-11
+
+
+# --------------------------------------------------------------------- codebook
+def _golden_max():
+    rows = {}
+    for line in open(golden_path("max1960_gaussian_lloyd_max.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        b, lv, mse = line.split()
+        # tolerance: one unit in the last printed digit of each entry (the 1960
+        # table's last digit is not always correctly rounded)
+        rows[int(b)] = ([(float(v), 10.0 ** -len(v.split(".")[1])) for v in lv.split(",")],
+                        float(mse))
+    return rows
+
+
+def _mse(cen, bnd, f, edge):
+    from scipy import integrate
+    e = np.concatenate([[-edge], bnd, [edge]])
+    return sum(integrate.quad(lambda z: (z - cen[k]) ** 2 * f(z), e[k], e[k + 1], epsrel=1e-12)[0]
+               for k in range(len(cen)))
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+def test_lloyd_max_gaussian_limit_matches_max_1960(bits):
+    levels, mse = _golden_max()[bits]
+    cen, bnd, _ = O.lloyd_max(bits, O.gaussian_density())
+    pos = cen[len(cen) // 2:]
+    for got, (want, tol) in zip(pos, levels):
+        assert abs(got - want) <= tol * 1.0001, (pos, levels)
+    f, edge = O.gaussian_density()
+    assert abs(_mse(cen, bnd, f, edge) - mse) < 1e-3 * mse
+
+
+@pytest.mark.parametrize("d", [8, 64, 128, 1536])
+def test_lloyd_max_one_bit_closed_form(d):
+    # c_1 = E[z | z > 0] = sqrt(d) Gamma(d/2) / (sqrt(pi) Gamma((d+1)/2))
+    want = math.sqrt(d) * math.exp(math.lgamma(d / 2) - math.lgamma((d + 1) / 2)) / math.sqrt(math.pi)
+    cen, bnd, _ = O.lloyd_max(1, O.fd_density(d))
+    assert abs(cen[1] - want) < 1e-11 and cen[0] == -cen[1] and bnd[0] == 0.0
+    pub_c, pub_b = O.published_codebook(1, d)
+    assert pub_c[1] == np.float32(want)
+
+
+@pytest.mark.parametrize("d", [8, 64, 1536])
+def test_fd_density_is_the_sphere_marginal(d):
+    # sqrt(d) * (first coordinate of a uniform unit vector) has density f_d
+    f, edge = O.fd_density(d)
+    total = mpmath.quad(lambda z: f(float(z)), [-edge, 0, edge])
+    assert abs(total - 1) < 1e-10
+    rng = np.random.default_rng(d)
+    g = rng.standard_normal((40000, d))
+    z = math.sqrt(d) * g[:, 0] / np.linalg.norm(g, axis=1)
+    from scipy import integrate
+    cdf = np.vectorize(lambda t: integrate.quad(f, -edge, t)[0])
+    ks = stats.kstest(z[:4000], cdf)
+    assert ks.pvalue > 1e-3, ks
+    # the variance of the marginal is exactly 1
+    var = mpmath.quad(lambda z: float(z) ** 2 * f(float(z)), [-edge, 0, edge])
+    assert abs(var - 1) < 1e-9
+
+
+@pytest.mark.parametrize("bits,d", [(2, 128), (3, 128), (4, 128), (2, 64), (3, 1536), (3, 8)])
+def test_lloyd_max_centroid_and_midpoint_conditions(bits, d):
+    cen, bnd, _ = O.lloyd_max(bits, O.fd_density(d))
+    f, edge = O.fd_density(d)
+    mpmath.mp.dps = 30
+    e = [-edge] + list(bnd) + [edge]
+    for k in range(len(cen)):
+        lo, hi = mpmath.mpf(e[k]), mpmath.mpf(e[k + 1])
+        p = mpmath.quad(lambda z: f(float(z)), [lo, hi])
+        m1 = mpmath.quad(lambda z: z * f(float(z)), [lo, hi])
+        assert abs(cen[k] - float(m1 / p)) < 1e-10, (k, cen[k], float(m1 / p))
+    assert np.allclose(bnd, 0.5 * (cen[:-1] + cen[1:]), rtol=0, atol=0)
+    assert np.array_equal(cen, -cen[::-1])
+    pub_c, pub_b = O.published_codebook(bits, d)
+    assert np.array_equal(pub_c, cen.astype(np.float32))
+    assert np.array_equal(pub_b, bnd.astype(np.float32))
+
+
+def test_lloyd_max_is_a_local_minimum():
+    bits, d = 3, 64
+    cen, bnd, _ = O.lloyd_max(bits, O.fd_density(d))
+    f, edge = O.fd_density(d)
+    base = _mse(cen, bnd, f, edge)
+    for k in range(len(cen)):
+        for eps in (1e-3, -1e-3):
+            c2 = cen.copy()
+            c2[k] += eps
+            assert _mse(c2, bnd, f, edge) > base
+    for k in range(len(bnd)):
+        for eps in (1e-3, -1e-3):
+            b2 = bnd.copy()
+            b2[k] += eps
+            assert _mse(cen, b2, f, edge) > base
+    # distortion falls by roughly 4x per bit (6 dB per bit rule) at these rates
+    m2 = _mse(*O.lloyd_max(2, O.fd_density(d))[:2], f, edge)
+    assert 3.0 < m2 / base < 4.5
+
+
+# -------------------------------------------------------------------- quantiser
+def _codec(d, bits, m, seed=0):
+    return O.make_codec(d, bits, m, seed)
+
+
+@pytest.mark.parametrize("bits", [1, 2])
+def test_quantizer_is_nearest_product_codeword_d8(bits):
+    d = 8
+    c = _codec(d, (bits,), 32)
+    rng = np.random.default_rng(bits)
+    x = rng.standard_t(3, size=(40, d))
+    comp = O.quantize(x, c)
+    cen = c.cen[0].astype(np.float64)
+    L = len(cen)
+    grid = np.array(np.meshgrid(*[np.arange(L)] * d, indexing="ij")).reshape(d, -1).T  # L^d codewords
+    words = cen[grid]
+    for n in range(x.shape[0]):
+        dist = np.sum((words - comp.z[n][None, :]) ** 2, axis=1)
+        best = grid[np.argmin(dist)]
+        if np.min(comp.code_margin[n]) > 1e-9:
+            assert np.array_equal(best, comp.code_idx[n])
+
+
+def test_quantizer_three_bits_nearest_centroid_per_coordinate():
+    d = 8
+    c = _codec(d, (3,), 32)
+    x = np.random.default_rng(9).standard_normal((200, d))
+    comp = O.quantize(x, c)
+    cen = c.cen[0].astype(np.float64)
+    near = np.argmin(np.abs(comp.z[:, :, None] - cen[None, None, :]), axis=2)
+    ok = comp.code_margin > 1e-9
+    assert np.array_equal(near[ok], comp.code_idx[ok])
+
+
+def test_code_rule_boundary_goes_to_upper_cell():
+    d = 8
+    c = _codec(d, (2,), 32)
+    bnd = c.bnd[0].astype(np.float64)
+    z = np.array([[bnd[0], bnd[1], bnd[2], np.nextafter(bnd[2], -np.inf), -10.0, 10.0, 0.0, bnd[0] - 1e-300]])
+    comp = O.quantize_with(z, z / math.sqrt(d), np.ones(1), c)
+    assert list(comp.code_idx[0]) == [1, 2, 3, 2, 0, 3, 2, 0 if bnd[0] - 1e-300 < bnd[0] else 1]
+
+
+def test_planar_packing_positions():
+    # segment s, plane p, word w, bit t  <->  bit p of the code of coordinate s*L + 32w + t
+    c = O.make_codec(128, (2, 3), 64, 0)   # W = 2*2 + 3*2 = 10 words
+    assert c.words == 10
+    codes = np.zeros((1, 128), dtype=np.int64)
+    codes[0, 64 + 32 + 5] = 0b100     # segment 1, word 1, bit 5, plane 2
+    codes[0, 3] = 0b10                # segment 0, word 0, bit 3, plane 1
+    w = O.pack_codes(codes, c)[0]
+    want = np.zeros(10, dtype=np.uint32)
+    want[1 * 2 + 0] = 1 << 3                  # seg 0: planes 0,1 x words 0,1 -> plane 1 word 0 = index 2
+    want[4 + 2 * 2 + 1] = 1 << 5              # seg 1 starts at 4; plane 2 word 1 -> 4 + 4 + 1
+    assert np.array_equal(w, want)
+    rnd = np.random.default_rng(0).integers(0, 4, size=(7, 128))
+    rnd[:, 64:] = np.random.default_rng(1).integers(0, 8, size=(7, 64))
+    assert np.array_equal(O.unpack_codes(O.pack_codes(rnd, c), c), rnd)
+    bits = np.random.default_rng(2).integers(0, 2, size=(5, 64))
+    assert np.array_equal(O.unpack_bits(O.pack_bits(bits), 64), bits)
+    one = np.zeros((1, 64), dtype=np.int64)
+    one[0, 37] = 1
+    assert list(O.pack_bits(one)[0]) == [0, 1 << 5]
+
+
+def test_sketch_index_convention():
+    # t_j = sum_i S[j, i] r_i : an S with one non-zero picks one residual coordinate
+    d, m = 8, 32
+    S = np.zeros((m, d), dtype=np.float32)
+    S[4, 6] = 1.0
+    S[9, 2] = -1.0
+    c = O.make_codec(d, (1,), m, 0, S=S)
+    x = np.random.default_rng(4).standard_normal((3, d))
+    comp = O.quantize(x, c)
+    r = comp.z / math.sqrt(d) - c.coord_cen(comp.code_idx) / math.sqrt(d)
+    assert np.allclose(comp.t[:, 4], r[:, 6], atol=1e-15)
+    assert np.allclose(comp.t[:, 9], -r[:, 2], atol=1e-15)
+    assert np.allclose(comp.t[:, 0], 0)
+
+
+def test_zero_vector_and_zero_residual():
+    d, m = 64, 64
+    c = _codec(d, (3,), m, seed=2)
+    # a rotated point exactly on the reconstruction grid has zero residual, so
+    # the estimate is nu <Pi q, y_hat> = <q, nu Pi^T y_hat> exactly
+    rng = np.random.default_rng(5)
+    codes = rng.integers(0, 8, size=(4, d))
+    z = c.coord_cen(codes)
+    nu = np.array([2.5, 1.0, 0.125, 3.0])
+    comp = O.quantize_with(z, z / math.sqrt(d), nu, c)
+    assert np.array_equal(comp.code_idx, codes)
+    assert comp.gamma64.max() == 0.0 and np.all(comp.t == 0)
+    assert np.all(O.unpack_bits(comp.signs, m) == 1)          # sign(0) = +1
+    x = nu[:, None] * (z / math.sqrt(d)) @ c.Pi
+    q = rng.standard_normal((1, 4, d))
+    l = O.estimate_scores(q, comp, c, 1, 4, 4, 1)
+    exact = np.einsum("hd,hd->h", q[0], x)
+    assert np.allclose(l[0, :, 0], exact, rtol=1e-12, atol=1e-12)
+    # nu = 0: all logits are zero, codes are those of z = 0
+    zc = O.quantize(np.zeros((1, d)), c)
+    assert zc.norms[0] == 0 and np.all(zc.code_idx == np.sum(c.bnd[0] <= 0))
+    assert np.all(O.estimate_scores(q[:, :1], zc, c, 1, 1, 1, 1) == 0)
+
+
+def test_decoder_error_matches_codebook_distortion():
+    # E ||x - x_hat||^2 / ||x||^2 equals the per-coordinate Lloyd-Max MSE
+    d, bits = 128, 3
+    c = _codec(d, (bits,), 0)
+    x = np.random.default_rng(8).standard_t(3, size=(3000, d))
+    comp = O.quantize(x, c)
+    xh = O.dequantize(comp, c)
+    rel = np.sum((x - xh) ** 2, axis=1) / np.sum(x * x, axis=1)
+    f, edge = O.fd_density(d)
+    cen, bnd, _ = O.lloyd_max(bits, O.fd_density(d))
+    want = _mse(cen, bnd, f, edge)
+    assert abs(rel.mean() - want) < 0.05 * want, (rel.mean(), want)
+
+
+# -------------------------------------------------------------------- estimator
+def test_qjl_estimator_is_unbiased_monte_carlo():
+    # QJL (TurboQuant news page; explainer page section "Por dentro"): over the
+    # Gaussian sketch, E[l] = <q, x> given the codes
+    d, m, N = 16, 32, 20000
+    rng = np.random.default_rng(21)
+    x = rng.standard_t(3, size=(1, d))
+    q = rng.standard_normal((1, 1, d))
+    c0 = O.make_codec(d, (2,), m, 0, S=np.zeros((m, d)))
+    comp0 = O.quantize(x, c0)
+    exact = float(q[0, 0] @ x[0])
+    est = np.empty(N)
+    qr = (q[0, 0] @ c0.Pi.T)
+    r = comp0.z[0] / math.sqrt(d) - c0.coord_cen(comp0.code_idx)[0] / math.sqrt(d)
+    mse_part = qr @ c0.coord_cen(comp0.code_idx)[0] / math.sqrt(d)
+    for k in range(N):
+        S = rng.standard_normal((m, d))
+        c = O.make_codec(d, (2,), m, 0, D=c0.D, S=S)
+        comp = O.quantize(x, c)
+        est[k] = O.estimate_scores(q, comp, c, 1, 1, 1, 1)[0, 0, 0]
+    se = est.std() / math.sqrt(N)
+    assert abs(est.mean() - exact) < 4 * se + 1e-6 * abs(exact), (est.mean(), exact, se)
+    # the single-draw spread is bounded by nu * ||r|| * ||q|| * sqrt(pi / (2 m))
+    nu = np.linalg.norm(x)
+    assert est.std() <= nu * np.linalg.norm(r) * np.linalg.norm(q) * math.sqrt(math.pi / (2 * m)) * 1.05
+    # the MSE-only part alone misses the residual term
+    assert abs(nu * mse_part - exact) > 10 * se
+
+
+def test_mse_only_estimator_is_biased_and_qjl_is_not():
+    # one-bit codes, averaged over rotations: E<q', y_hat> / <q, u> -> c_1 sqrt(2/pi) ~ 2/pi
+    d, N = 64, 3000
+    rng = np.random.default_rng(33)
+    x = rng.standard_normal((1, d))
+    q = (x + 0.5 * rng.standard_normal((1, d)))[None]
+    exact = float(q[0, 0] @ x[0])
+    mse_only, full = np.empty(N), np.empty(N)
+    for k in range(N):
+        D = rng.choice([-1.0, 1.0], size=d)
+        c = O.make_codec(d, (1,), 64, 0, D=D, S=rng.standard_normal((64, d)))
+        comp = O.quantize(x, c)
+        full[k] = O.estimate_scores(q, comp, c, 1, 1, 1, 1)[0, 0, 0]
+        cm = O.make_codec(d, (1,), 0, 0, D=D)
+        mse_only[k] = O.estimate_scores(q, O.quantize(x, cm), cm, 1, 1, 1, 1)[0, 0, 0]
+    ratio = mse_only.mean() / exact
+    c1 = O.published_codebook(1, d)[0][1]
+    assert abs(ratio - c1 * math.sqrt(2 / math.pi)) < 0.03, ratio
+    assert abs(full.mean() - exact) < 4 * full.std() / math.sqrt(N)
+
+
+def test_gqa_rows_and_accuracy_at_four_bits():
+    # with 4-bit codes and m = 128 each logit is close to its own key's inner product
+    B, Hq, Hkv, T, d = 2, 4, 2, 16, 128
+    c = _codec(d, (4,), 128, seed=3)
+    x = synth.heavy_rows(5, B * Hkv * T, d).to(dtype=__import__("torch").float64).numpy()
+    q = np.random.default_rng(6).standard_normal((B, Hq, d))
+    comp = O.quantize(x, c)
+    l = O.estimate_scores(q, comp, c, B, Hq, Hkv, T)
+    for b in range(B):
+        for h in range(Hq):
+            rows = (b * Hkv + h // (Hq // Hkv)) * T + np.arange(T)
+            exact = x[rows] @ q[b, h]
+            scale = np.linalg.norm(x[rows], axis=1) * np.linalg.norm(q[b, h])
+            assert np.all(np.abs(l[b, h] - exact) < 0.08 * scale)
+
+
+# -------------------------------------------------------------------- attention
+def test_attend_special_cases():
+    d = 64
+    kc = _codec(d, (2,), 64, seed=1)
+    vc = _codec(d, (4,), 0, seed=1)
+    rng = np.random.default_rng(2)
+    # T = 1: the output is the single dequantised value
+    k1, v1 = rng.standard_normal((2, 1, d))
+    q = rng.standard_normal((1, 2, d))
+    K, V = O.quantize(k1, kc), O.quantize(v1, vc)
+    out = O.attend(q, K, V, kc, vc, 1, 2, 1, 1)
+    vhat = O.dequantize(V, vc)[0]
+    assert np.allclose(out[0, 0], vhat, atol=1e-12) and np.allclose(out[0, 1], vhat, atol=1e-12)
+    # all logits equal (q = 0): the output is the mean of the dequantised values
+    T = 9
+    k, v = rng.standard_normal((2, T, d))
+    K, V = O.quantize(k, kc), O.quantize(v, vc)
+    out = O.attend(np.zeros((1, 1, d)), K, V, kc, vc, 1, 1, 1, T)
+    assert np.allclose(out[0, 0], O.dequantize(V, vc).mean(axis=0), atol=1e-12)
+    # a dominant logit selects its value
+    q = 50 * k[3:4][None] / np.linalg.norm(k[3])
+    out = O.attend(q, K, V, kc, vc, 1, 1, 1, T, scale=1.0)
+    assert np.allclose(out[0, 0], O.dequantize(V, vc)[3], atol=1e-6)
+
+
+# ----------------------------------------------------------------------- top-k
+def test_topk_order_and_ties():
+    sc = np.array([[0.5, 2.0, 2.0, -1.0, 2.0, 0.7]])
+    idx, val = O.topk_rows(sc, 4, 100)
+    assert list(idx[0]) == [101, 102, 104, 105] and list(val[0]) == [2.0, 2.0, 2.0, 0.7]
+    rng = np.random.default_rng(1)
+    sc = rng.integers(0, 20, size=(3, 200)).astype(float)
+    idx, _ = O.topk_rows(sc, 10, 0)
+    for i in range(3):
+        want = sorted(range(200), key=lambda j: (-sc[i, j], j))[:10]
+        assert list(idx[i]) == want
