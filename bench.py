@@ -1,0 +1,424 @@
+#!/usr/bin/env python
+"""Throughput benchmark of the TurboQuant-style KV-cache path on B200.
+
+One step = the whole hot path over one decode layer shaped like
+Llama-3.1-8B at 32k context (batch 8, 32 query heads, 8 KV heads, head_dim
+128, bf16 K/V with Student-t(3) entries and 1% outlier channels x100):
+  tq_quantize(K: 3-bit Lloyd-Max + QJL m=128), tq_quantize(V: 4-bit),
+  tq_scores (logits of the 8x32 decode queries), tq_attend (decode attention).
+The headline value is compressed keys processed per second (keys of the
+layer / step time); per-stage figures, the roofline of the dominant kernel
+and of the scoring kernel, an end-to-end figure through host buffers and the
+CPU oracle's throughput on a bounded sample are reported alongside.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl tq|reference]
+
+Under torchrun (N > 1) every rank processes its own layer (independent data),
+no collective touches the data path, and the step time is the maximum over
+ranks (weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "compressed keys scored/s and % of B200 HBM peak (32k ctx); tokens quantised/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ------------------------------------------------------------------ helpers
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """Polls NVML for SM clock and clock-event reasons in a background thread."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples = []
+        self.period = period_s
+        self._stop = threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = None
+            try:
+                uuid = torch.cuda.get_device_properties(device_index).uuid
+            except Exception:
+                pass
+            h = None
+            if uuid is not None:
+                try:
+                    h = pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + str(uuid)).encode())
+                except Exception:
+                    h = None
+            if h is None:
+                vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+                idx = int(vis.split(",")[device_index]) if vis and vis.split(",")[0].isdigit() else device_index
+                h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.nvml, self.h = pynvml, h
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report it
+            self.err = str(e)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                t = time.perf_counter()
+                mhz = self.nvml.nvmlDeviceGetClockInfo(self.h, self.nvml.NVML_CLOCK_SM)
+                rs = self.nvml.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((t, mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self.th = threading.Thread(target=self._run, daemon=True)
+            self.th.start()
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self.th.join()
+
+    def summary(self, t0: float, t1: float):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        if not inside and self.samples:
+            inside = [min(self.samples, key=lambda s: abs(s[0] - 0.5 * (t0 + t1)))]
+        mhz = [s[1] for s in inside]
+        bits = 0
+        for s in inside:
+            bits |= s[2]
+        reasons = sorted(v for k, v in self.REASONS.items() if bits & k and v != "gpu_idle")
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(inside)}
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+# ---------------------------------------------------------------- workload
+class Layer:
+    """Device-resident inputs, codecs and outputs of one decode layer."""
+
+    def __init__(self, tq, w: synth.Workload, dev: torch.device, rank: int):
+        import dataclasses
+        self.w = w = dataclasses.replace(w, data_seed=w.data_seed + rank)
+        self.tq = tq
+        d = w.d
+        self.k_host = synth.kv_full(w, "K").reshape(-1, d)
+        self.v_host = synth.kv_full(w, "V").reshape(-1, d)
+        self.q_host = synth.queries(w)
+        self.k = self.k_host.to(dev)
+        self.v = self.v_host.to(dev)
+        self.q = self.q_host.to(dev).contiguous()
+        self.kc = tq.Codec(d, w.k_bits, w.k_m, w.codec_seed, device=dev.index)
+        self.vc = tq.Codec(d, w.v_bits, w.v_m, w.codec_seed + 1, device=dev.index)
+        n = w.n_keys
+        self.K = tq.Compressed.empty(self.kc, n, dev)
+        self.V = tq.Compressed.empty(self.vc, n, dev)
+        self.logits = torch.empty((w.B, w.Hq, w.T), device=dev)
+        self.out = torch.empty((w.B, w.Hq, d), device=dev)
+        self.ws_s = tq.workspace(tq.tq_scores_workspace_size(self.kc, w.B, w.Hq), dev)
+        self.ws_a = tq.workspace(tq.tq_attend_workspace_size(self.kc, self.vc, w.B, w.Hq, w.Hkv, w.T), dev)
+
+    def stages(self, k=None, v=None, q=None):
+        tq, w = self.tq, self.w
+        k = self.k if k is None else k
+        v = self.v if v is None else v
+        q = self.q if q is None else q
+        return [
+            ("tq_quantize_K", lambda: tq.tq_quantize(self.kc, k, self.K)),
+            ("tq_quantize_V", lambda: tq.tq_quantize(self.vc, v, self.V)),
+            ("tq_scores", lambda: tq.tq_scores(self.kc, q, w.B, w.Hq, w.Hkv, w.T, self.K, self.logits, self.ws_s)),
+            ("tq_attend", lambda: tq.tq_attend(self.kc, self.vc, q, w.B, w.Hq, w.Hkv, w.T, self.K, self.V, self.out,
+                                               self.ws_a)),
+        ]
+
+    # launches of libtq kernels per stage (quantize: 1; scores: query prep +
+    # scoring; attend: query prep + split-context attention + combine)
+    LAUNCHES = {"tq_quantize_K": 1, "tq_quantize_V": 1, "tq_scores": 2, "tq_attend": 3}
+
+    def algorithmic_bytes(self):
+        w, d = self.w, self.w.d
+        n = w.n_keys
+        esz = 2 if w.dtype == "bf16" else 4
+        kc, vc = self.kc, self.vc
+        krow = 4 * kc.code_words + 4 * kc.sign_words + 4 + (4 if kc.m else 0)
+        vrow = 4 * vc.code_words + 4 * vc.sign_words + 4 + (4 if vc.m else 0)
+        return {
+            "tq_quantize_K": n * (d * esz + krow),
+            "tq_quantize_V": n * (d * esz + vrow),
+            "tq_scores": n * (krow + 4 * w.G),
+            "tq_attend": n * (krow + vrow),
+        }, {"key_row": krow, "value_row": vrow, "input_row": d * esz}
+
+
+def time_steps(layer, steps: int, stream, stages=None, pre=None, post=None):
+    """Times `steps` steps with CUDA events on `stream`; returns total ms and
+    per-stage ms lists."""
+    stages = stages or layer.stages()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)] for _ in range(steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for s in range(steps):
+        if pre:
+            pre()
+        evs[s][0].record(stream)
+        for i, (_, fn) in enumerate(stages):
+            fn()
+            evs[s][i + 1].record(stream)
+        if post:
+            post()
+    end.record(stream)
+    end.synchronize()
+    total = start.elapsed_time(end)
+    per = {name: [evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(steps)] for i, (name, _) in enumerate(stages)}
+    return total, per
+
+
+# ------------------------------------------------------------ CPU baseline
+def cpu_oracle_sample(w: synth.Workload, budget_s: float, rank_seed: int = 0):
+    """The oracle, as it stands, on bounded samples of the workload: whole
+    (b, KV head) slabs cut to their first `tn` tokens, each quantised (K and V),
+    scored for the G query heads and attended.  Returns (keys/s, seconds,
+    keys, threads, description)."""
+    import oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        threads = 1
+    d = w.d
+    okc = O.make_codec(d, w.k_bits, w.k_m, w.codec_seed)
+    ovc = O.make_codec(d, w.v_bits, w.v_m, w.codec_seed + 1) if w.v_bits else None
+    qall = synth.queries(w).to(torch.float64).numpy()
+    tn = 1024
+    keys, secs, slabs = 0, 0.0, 0
+    t_start = time.perf_counter()
+    while secs < budget_s:
+        b = slabs % w.B
+        h = (slabs // w.B) % w.Hkv
+        k = synth.kv_slab(w, "K", b, h, 0, tn).to(torch.float64).numpy()
+        v = synth.kv_slab(w, "V", b, h, 0, tn).to(torch.float64).numpy() if ovc else None
+        q = qall[b, h * w.G:(h + 1) * w.G][None]
+        t0 = time.perf_counter()
+        Ko = O.quantize(k, okc)
+        if ovc is not None:
+            Vo = O.quantize(v, ovc)
+        O.estimate_scores(q, Ko, okc, 1, w.G, 1, tn)
+        if ovc is not None:
+            O.attend(q, Ko, Vo, okc, ovc, 1, w.G, 1, tn)
+        secs += time.perf_counter() - t0
+        keys += tn
+        slabs += 1
+        if time.perf_counter() - t_start > 4 * budget_s:
+            break
+    desc = (f"{slabs} (batch, KV head) slabs of the {w.name} layer cut to {tn} tokens: quantise K and V, "
+            f"score {w.G} query heads, attend; keys/s = keys / oracle seconds")
+    return keys / secs, secs, keys, threads, desc
+
+
+# ------------------------------------------------------------------- main
+def run_reference(args, rank, world):
+    """The oracle as the reference arm: rank 0 only, bounded samples per step."""
+    if rank != 0:
+        return 0
+    w = synth.WORKLOADS[args.workload]
+    times, keys_total = [], 0
+    for s in range(args.warmup + args.steps):
+        kps, secs, keys, threads, desc = cpu_oracle_sample(w, args.ref_step_seconds)
+        if s >= args.warmup:
+            times.append(secs)
+            keys_total += keys
+    total = sum(times)
+    value = keys_total / total
+    line = {
+        "metric": METRIC, "value": value, "unit": "keys/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "T": w.T, "d": w.d,
+                   "k_bits": list(w.k_bits), "k_m": w.k_m, "v_bits": list(w.v_bits), "input_dtype": w.dtype,
+                   "step": "quantise K and V, score, attend (bounded sample per step)"},
+        "cpu_baseline": {"value": value, "unit": "keys/s", "cores": threads, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "keys/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["tq", "reference"], default="tq")
+    ap.add_argument("--workload", default="llama8b_decode")
+    ap.add_argument("--e2e-steps", type=int, default=0, help="0: same as --steps")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-step-seconds", type=float, default=3.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import kv_cache_vector_09_b200 as tq  # fails loudly without libtq.so
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+    w = synth.WORKLOADS[args.workload]
+    layer = Layer(tq, w, dev, rank)
+    stream = torch.cuda.current_stream()
+
+    for _ in range(args.warmup):
+        for _, fn in layer.stages():
+            fn()
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.perf_counter()
+    total_ms, per = time_steps(layer, args.steps, stream)
+    torch.cuda.synchronize()
+    t_wall1 = time.perf_counter()
+    if pg:
+        pg.barrier()
+    clocks.stop()
+    ms_step = total_ms / args.steps
+    if pg:
+        t = torch.tensor([ms_step], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms_step = float(t.item())
+    keys_step = w.n_keys
+    value = keys_step * world / (ms_step * 1e-3)
+
+    # end to end through host buffers: pinned K, V, Q copied in, logits and the
+    # attention output copied out, every step, on the same stream
+    e2e_steps = args.e2e_steps or args.steps
+    kh = layer.k_host.pin_memory()
+    vh = layer.v_host.pin_memory()
+    qh = layer.q_host.pin_memory()
+    lh = torch.empty(layer.logits.shape, dtype=torch.float32).pin_memory()
+    oh = torch.empty(layer.out.shape, dtype=torch.float32).pin_memory()
+    kd, vd, qd = torch.empty_like(layer.k), torch.empty_like(layer.v), torch.empty_like(layer.q)
+
+    def pre():
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        qd.copy_(qh, non_blocking=True)
+
+    def post():
+        lh.copy_(layer.logits, non_blocking=True)
+        oh.copy_(layer.out, non_blocking=True)
+
+    e2e_stages = layer.stages(kd, vd, qd)
+    time_steps(layer, 1, stream, e2e_stages, pre, post)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    e2e_ms, _ = time_steps(layer, e2e_steps, stream, e2e_stages, pre, post)
+    e2e_ms /= e2e_steps
+    if pg:
+        t = torch.tensor([e2e_ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = kh.numel() * kh.element_size() + vh.numel() * vh.element_size() + qh.numel() * qh.element_size()
+    d2h = lh.numel() * 4 + oh.numel() * 4
+    del kd, vd
+
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    hbm, peak_src = load_peaks()
+    alg, rows = layer.algorithmic_bytes()
+    stages = {}
+    for name, lst in per.items():
+        ms = statistics.mean(lst)
+        gbs = alg[name] / (ms * 1e-3) / 1e9
+        stages[name] = {"ms": round(ms, 5), "algorithmic_bytes": alg[name], "GB_s": round(gbs, 1),
+                        "frac_hbm": round(gbs / hbm, 4), "launches": Layer.LAUNCHES[name]}
+    dom = max(stages, key=lambda k: stages[k]["ms"])
+
+    def roof(name):
+        s = stages[name]
+        return {"kernel": name, "bound": "hbm", "achieved": s["GB_s"], "peak": hbm, "unit": "GB/s",
+                "frac": s["frac_hbm"], "traffic": None, "peak_source": f"{peak_src} hbm_gbs",
+                "bytes_per_launch": s["algorithmic_bytes"]}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "keys/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "T": w.T, "d": w.d,
+                   "k_bits": list(w.k_bits), "k_m": w.k_m, "v_bits": list(w.v_bits), "v_m": w.v_m,
+                   "input_dtype": w.dtype, "parallelism": f"dp{world} (independent layers per rank)",
+                   "step": "tq_quantize K, tq_quantize V, tq_scores, tq_attend",
+                   "l2": "inputs larger than L2: 1.07 GB of bf16 K/V read per step",
+                   "key_row_bytes": rows["key_row"], "value_row_bytes": rows["value_row"]},
+        "tokens_quantised_per_s": w.B * w.T * world / ((stages["tq_quantize_K"]["ms"] + stages["tq_quantize_V"]["ms"])
+                                                       * 1e-3),
+        "stages": stages,
+        "roofline": roof(dom),
+        "roofline_scores": roof("tq_scores"),
+        "gpu_launches": args.steps * sum(Layer.LAUNCHES.values()),
+        "e2e": {"value": keys_step * world / (e2e_ms * 1e-3), "unit": "keys/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "clocks": clocks.summary(t_wall0, t_wall1),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        kps, secs, keys, threads, desc = cpu_oracle_sample(w, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": kps, "unit": "keys/s", "cores": threads, "kind": "oracle",
+                                "sample": desc, "seconds": round(secs, 2)}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

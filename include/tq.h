@@ -1,0 +1,209 @@
+/*
+ * tq.h -- C ABI of libtq: TurboQuant-style KV-cache compression and scoring
+ * over the compressed keys and values, for NVIDIA B200 (sm_100a).
+ *
+ * The method (as the source pages describe it):
+ *   "FibQuant: Quantizacao Vetorial Universal para Compressao de KV-Cache de
+ *   Acesso Aleatorio", section 1: a random-access codec stores the vector norm,
+ *   applies a shared random orthogonal rotation and quantises every rotated
+ *   coordinate with a scalar Lloyd-Max table; section 2.3: the decoder reads
+ *   the codes, undoes the rotation and scales by the norm; every token's record
+ *   has a fixed size and a fixed address.
+ *   "TurboQuant: Compressao Avancada da Google para Cache KV ...", section
+ *   "TurboQuant: Uma Nova Abordagem": the rotation is a randomized Hadamard
+ *   transform and a 1-bit quantized Johnson-Lindenstrauss (QJL) stage on the
+ *   residual makes inner-product estimates unbiased.
+ *   "Compressao KV eficaz com TurboQuant", section "Por dentro do processo":
+ *   the JL transform of the residual is reduced to one sign bit per projected
+ *   coordinate.
+ *   "TurboESM ...", "Resumo tecnico" section 2: one fused decode kernel
+ *   dequantises and runs an online softmax with no dequantised copy.
+ *
+ * Definitions used by every call (d = head dimension, m = QJL rows):
+ *   nu = ||x||_2,  u = x / nu (u = 0 if nu = 0)
+ *   y  = Pi u,  Pi = blockdiag(H_p, ..., H_p) diag(D) / sqrt(p),
+ *        H_p the Sylvester-Hadamard matrix H[i][j] = (-1)^popcount(i & j),
+ *        p = d if d is a power of two, else p = 512 (d a multiple of 512);
+ *        D = +-1 signs drawn from the codec seed
+ *   z  = sqrt(d) y                         (unit-variance rotated coordinate)
+ *   code_i = #{k : bnd_k <= z_i}           (Lloyd-Max cells, ties go up)
+ *   r  = y - cen[code] / sqrt(d),  gamma = ||r||_2
+ *   bit_j = ((S r)_j >= 0),  S an m x d matrix of iid N(0,1) fp32 entries
+ *   estimate of <q, x>:
+ *        nu * ( <Pi q, cen[code]> / sqrt(d)
+ *               + gamma * sqrt(pi/2) / m * <S Pi q, 2 bit - 1> )
+ *
+ * Conventions.
+ *   - Every pointer passed to a compute call is a device pointer on the codec's
+ *     device, 16-byte aligned, owned by the caller.  The library owns only the
+ *     tq_codec.  Compute calls allocate no memory: tq_scores and tq_attend take
+ *     a caller workspace sized by their *_workspace_size call.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Calls are asynchronous on that stream.  The calling thread's current
+ *     device must be the codec's device.
+ *   - Arguments are validated on the host before anything is launched; on any
+ *     error nothing is written and the status says why
+ *     (tq_last_error_string() has the detail, per thread).  Errors of earlier
+ *     asynchronous work surface as TQ_ERR_CUDA on a later call or at sync.
+ *   - A codec is immutable after creation; concurrent calls on distinct
+ *     streams are safe.
+ */
+#ifndef TQ_H_
+#define TQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TQ_API __attribute__((visibility("default")))
+#else
+#define TQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TQ_OK = 0,
+  TQ_ERR_INVALID_ARG = 1,   /* bad size, pointer, alignment, device or enum */
+  TQ_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. d = 96)       */
+  TQ_ERR_NO_MEMORY = 3,     /* codec creation could not allocate             */
+  TQ_ERR_CUDA = 4,          /* a CUDA runtime call failed                    */
+  TQ_ERR_DEVICE_ASSERT = 5, /* a kernel reported a failed internal check     */
+  TQ_ERR_NOT_CONVERGED = 6  /* Lloyd-Max iteration limit reached             */
+} tq_status;
+
+typedef enum { TQ_F32 = 0, TQ_BF16 = 1, TQ_F16 = 2 } tq_dtype;
+
+/* Codec parameters.
+ *   d        : 64, 128, 256, 512, 1024 or 1536 (1024 and 1536 rotate in
+ *              512-coordinate Hadamard blocks)
+ *   nseg     : 1, or 2 = the two coordinate halves [0, d/2) and [d/2, d) use
+ *              seg_bits[0] and seg_bits[1] bits (e.g. 2 + 3 = 2.5 bits/coord)
+ *   seg_bits : 1..4 bits per coordinate for each segment
+ *   m        : QJL rows, 0 (MSE-only codes, no signs, no residual norm) or a
+ *              multiple of 32, at most 1024
+ *   seed     : draws D (splitmix64 from `seed`, top bit 1 -> -1) and S
+ *              (splitmix64 from seed ^ 0x5851F42D4C957F2D, Box-Muller cosine
+ *              branch on output pairs, double, rounded to fp32, row-major m x d) */
+typedef struct {
+  int32_t d;
+  int32_t nseg;
+  int32_t seg_bits[2];
+  int32_t m;
+  uint64_t seed;
+} tq_spec;
+
+/* One compressed row per vector, structure-of-arrays, all caller-owned device
+ * memory with n rows:
+ *   codes  [n][W] uint32, W = sum_s seg_bits[s] * (d / nseg) / 32.
+ *          Planar layout: segments in order; inside segment s, bit planes
+ *          p = 0..seg_bits[s]-1; inside a plane, word w holds bit p of the codes
+ *          of the segment's coordinates 32w..32w+31, coordinate 32w+t at bit t.
+ *   signs  [n][m/32] uint32, bit j%32 of word j/32 = bit_j; NULL iff m == 0
+ *   norms  [n] fp32, nu
+ *   rnorms [n] fp32, gamma; NULL iff m == 0                                   */
+typedef struct {
+  uint32_t *codes;
+  uint32_t *signs;
+  float *norms;
+  float *rnorms;
+} tq_compressed;
+
+typedef struct tq_codec tq_codec; /* opaque: codebooks, D, S, device tables */
+
+/* Lloyd-Max codebook for the rotated-coordinate law (host only, pure).
+ * Solves the 2^bits-level MSE-optimal scalar quantiser of
+ *   f_d(z) = C_d (1 - z^2/d)^((d-3)/2),  |z| < sqrt(d),
+ * the exact marginal of sqrt(d) * u_1 for u uniform on the unit sphere (the
+ * "Beta" coordinate law the explainer page attributes to the random rotation;
+ * the FibQuant page's k = 1 spherical-Beta source), alternating the midpoint
+ * and centroid conditions until the centroids move by less than `tol`.
+ *   bits in 1..4; d >= 4; tol <= 0 selects 1e-12; max_iter <= 0 selects 20000.
+ *   centroids  [2^bits]     out, ascending, symmetric, fp32 of the double solution
+ *   boundaries [2^bits - 1] out, fp32 of the double midpoints
+ * Returns TQ_ERR_NOT_CONVERGED (outputs untouched) if max_iter is reached.   */
+TQ_API tq_status tq_make_codebook(int bits, int d, double tol, int max_iter,
+                           float *centroids, float *boundaries);
+
+/* Create a codec for `spec` on CUDA device `device` (uploads D, S, codebooks
+ * and derived tables; this call allocates device memory).  device = -1 makes a
+ * host-only codec usable with tq_codec_export and tq_codec_layout only.
+ * *out is set only on TQ_OK.                                                 */
+TQ_API tq_status tq_codec_create(const tq_spec *spec, int device, tq_codec **out);
+
+/* Free a codec (NULL is a no-op).  The caller must ensure no work using it is
+ * still in flight.                                                           */
+TQ_API tq_status tq_codec_destroy(tq_codec *codec);
+
+/* Host copies of the codec's random draws and codebooks, for checking.
+ * Any pointer may be NULL to skip it.
+ *   S      [m][d] fp32
+ *   dsigns [ceil(d/32)] words, bit t of word w set  <=>  D_{32w+t} = -1
+ *   cen    [sum_s 2^seg_bits[s]]      per-segment centroids, concatenated
+ *   bnd    [sum_s 2^seg_bits[s] - 1]  per-segment boundaries, concatenated    */
+TQ_API tq_status tq_codec_export(const tq_codec *codec, float *S, uint32_t *dsigns,
+                          float *cen, float *bnd);
+
+/* Row sizes of the compressed format in 32-bit words (either pointer may be
+ * NULL): code_words = W, sign_words = m / 32.                               */
+TQ_API tq_status tq_codec_layout(const tq_codec *codec, int *code_words,
+                          int *sign_words);
+
+/* Compress n rows (encoder of the FibQuant page, section 2.3, plus the QJL
+ * residual sketch of the TurboQuant pages).
+ *   x     [n][ld] elements of `dtype` (TQ_F32, TQ_BF16 or TQ_F16); row i
+ *         starts at element i*ld; ld >= d and ld * sizeof(dtype) % 16 == 0
+ *   out   device arrays with n rows (see tq_compressed)
+ * Codes and sign bits equal those of an exact (real-arithmetic) evaluation of
+ * the definitions above: a fast fp32 evaluation decides every code and sign
+ * whose margin exceeds a proven fp32 error bound, and the few rows with a
+ * closer decision are recomputed in fp64.  n = 0 is a no-op.                */
+TQ_API tq_status tq_quantize(const tq_codec *codec, const void *x, tq_dtype dtype,
+                      int64_t n, int64_t ld, const tq_compressed *out,
+                      void *stream);
+
+/* Workspace bytes for tq_scores with B batches of Hq query heads.           */
+TQ_API tq_status tq_scores_workspace_size(const tq_codec *kc, int B, int Hq,
+                                   size_t *bytes);
+
+/* Attention logits over compressed keys (unscaled estimator above).
+ *   q       [B][Hq][d] of `dtype`, contiguous
+ *   K       compressed keys, B*Hkv*T rows; key (b, h_kv, t) is row
+ *           (b*Hkv + h_kv)*T + t
+ *   logits  [B][Hq][T] fp32 out; query head h uses KV head h / (Hq / Hkv)
+ *   workspace, ws_bytes  >= tq_scores_workspace_size(kc, B, Hq)
+ * Hq must be a multiple of Hkv, Hq / Hkv <= 32.  T = 0 is a no-op.          */
+TQ_API tq_status tq_scores(const tq_codec *kc, const void *q, tq_dtype dtype, int B,
+                    int Hq, int Hkv, int64_t T, const tq_compressed *K,
+                    float *logits, void *workspace, size_t ws_bytes,
+                    void *stream);
+
+/* Workspace bytes for tq_attend (depends on the current device's SM count). */
+TQ_API tq_status tq_attend_workspace_size(const tq_codec *kc, const tq_codec *vc,
+                                   int B, int Hq, int Hkv, int64_t T,
+                                   size_t *bytes);
+
+/* Decode attention over compressed keys and values (fused decode of the
+ * TurboESM page, "Resumo tecnico" section 2): for each (b, h):
+ *   p   = softmax over t of scale * logit(b, h, t)   (scale 0 -> 1/sqrt(d))
+ *   out = Pi_v^T  sum_t p_t nu_v,t cen_v[code_v,t] / sqrt(d)
+ * i.e. the values are dequantised with their own codec `vc` (vc->m is not
+ * used) and never written out.  Shapes as tq_scores; out [B][Hq][d] fp32.
+ * kc and vc must have the same d.  T >= 1.                                 */
+TQ_API tq_status tq_attend(const tq_codec *kc, const tq_codec *vc, const void *q,
+                    tq_dtype dtype, int B, int Hq, int Hkv, int64_t T,
+                    float scale, const tq_compressed *K,
+                    const tq_compressed *V, void *workspace, size_t ws_bytes,
+                    float *out, void *stream);
+
+/* Human-readable status and the calling thread's last error detail.        */
+TQ_API const char *tq_status_string(tq_status status);
+TQ_API const char *tq_last_error_string(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H_ */

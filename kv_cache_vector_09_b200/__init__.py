@@ -1,0 +1,234 @@
+"""B200-native TurboQuant-style KV-cache compression: Python binding of libtq.
+
+This module only marshals arguments for the C ABI declared in ``include/tq.h``
+(same function names); every step of the codec runs in the CUDA kernels of
+``libtq.so``.  PyTorch supplies device memory and streams.  There is no CPU
+fallback: importing this package fails loudly if ``libtq.so`` is missing
+(build it with ``python -m kv_cache_vector_09_b200.build``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence, Tuple
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtq.so")
+
+TQ_OK = 0
+STATUS_NAMES = {0: "TQ_OK", 1: "TQ_ERR_INVALID_ARG", 2: "TQ_ERR_UNSUPPORTED", 3: "TQ_ERR_NO_MEMORY",
+                4: "TQ_ERR_CUDA", 5: "TQ_ERR_DEVICE_ASSERT", 6: "TQ_ERR_NOT_CONVERGED"}
+TQ_F32, TQ_BF16, TQ_F16 = 0, 1, 2
+_DTYPES = {torch.float32: TQ_F32, torch.bfloat16: TQ_BF16, torch.float16: TQ_F16}
+
+
+class TQError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}: {detail}")
+
+
+class tq_spec(ctypes.Structure):
+    _fields_ = [("d", ctypes.c_int32), ("nseg", ctypes.c_int32), ("seg_bits", ctypes.c_int32 * 2),
+                ("m", ctypes.c_int32), ("seed", ctypes.c_uint64)]
+
+
+class tq_compressed(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("signs", ctypes.c_void_p), ("norms", ctypes.c_void_p),
+                ("rnorms", ctypes.c_void_p)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m kv_cache_vector_09_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, I64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+    sig = {
+        "tq_make_codebook": [I, I, ctypes.c_double, I, P, P],
+        "tq_codec_create": [P, I, ctypes.POINTER(P)],
+        "tq_codec_destroy": [P],
+        "tq_codec_export": [P, P, P, P, P],
+        "tq_codec_layout": [P, ctypes.POINTER(I), ctypes.POINTER(I)],
+        "tq_quantize": [P, P, I, I64, I64, P, P],
+        "tq_scores_workspace_size": [P, I, I, ctypes.POINTER(SZ)],
+        "tq_scores": [P, P, I, I, I, I, I64, P, P, P, SZ, P],
+        "tq_attend_workspace_size": [P, P, I, I, I, I64, ctypes.POINTER(SZ)],
+        "tq_attend": [P, P, P, I, I, I, I, I64, ctypes.c_float, P, P, P, SZ, P, P],
+    }
+    for name, args in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = ctypes.c_int
+    lib.tq_status_string.argtypes = [ctypes.c_int]
+    lib.tq_status_string.restype = ctypes.c_char_p
+    lib.tq_last_error_string.argtypes = []
+    lib.tq_last_error_string.restype = ctypes.c_char_p
+    return lib
+
+
+_lib = _load()
+
+
+def _check(status: int, where: str) -> None:
+    if status != TQ_OK:
+        raise TQError(status, where, _lib.tq_last_error_string().decode())
+
+
+def tq_status_string(status: int) -> str:
+    return _lib.tq_status_string(status).decode()
+
+
+def tq_last_error_string() -> str:
+    return _lib.tq_last_error_string().decode()
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+# ---------------------------------------------------------------------- calls
+def tq_make_codebook(bits: int, d: int, tol: float = 0.0, max_iter: int = 0) -> Tuple[np.ndarray, np.ndarray]:
+    """Host Lloyd-Max codebook: (centroids [2^bits], boundaries [2^bits - 1]) fp32."""
+    cen = np.zeros(1 << bits, dtype=np.float32)
+    bnd = np.zeros((1 << bits) - 1, dtype=np.float32)
+    _check(_lib.tq_make_codebook(bits, d, tol, max_iter, cen.ctypes.data, bnd.ctypes.data), "tq_make_codebook")
+    return cen, bnd
+
+
+class Codec:
+    """A tq_codec handle (freed with the object)."""
+
+    def __init__(self, d: int, seg_bits: Sequence[int], m: int, seed: int = 0, device: int = 0):
+        seg_bits = tuple(int(b) for b in seg_bits)
+        self.d, self.seg_bits, self.m, self.seed, self.device = d, seg_bits, m, seed, device
+        spec = tq_spec(d, len(seg_bits), (ctypes.c_int32 * 2)(*(seg_bits + (0,) * (2 - len(seg_bits)))), m, seed)
+        h = ctypes.c_void_p()
+        _check(_lib.tq_codec_create(ctypes.byref(spec), device, ctypes.byref(h)), "tq_codec_create")
+        self._h = h
+        cw, sw = ctypes.c_int(), ctypes.c_int()
+        _check(_lib.tq_codec_layout(h, ctypes.byref(cw), ctypes.byref(sw)), "tq_codec_layout")
+        self.code_words, self.sign_words = cw.value, sw.value
+
+    @property
+    def handle(self) -> ctypes.c_void_p:
+        return self._h
+
+    def export(self):
+        """(S [m, d] fp32, dsigns [ceil(d/32)] uint32, cen list, bnd list) host copies."""
+        S = np.zeros((self.m, self.d), dtype=np.float32)
+        ds = np.zeros((self.d + 31) // 32, dtype=np.uint32)
+        nc = sum(1 << b for b in self.seg_bits)
+        cen = np.zeros(nc, dtype=np.float32)
+        bnd = np.zeros(nc - len(self.seg_bits), dtype=np.float32)
+        _check(_lib.tq_codec_export(self._h, S.ctypes.data if self.m else None, ds.ctypes.data, cen.ctypes.data,
+                                    bnd.ctypes.data), "tq_codec_export")
+        cl, bl, oc, ob = [], [], 0, 0
+        for b in self.seg_bits:
+            cl.append(cen[oc:oc + (1 << b)])
+            bl.append(bnd[ob:ob + (1 << b) - 1])
+            oc += 1 << b
+            ob += (1 << b) - 1
+        return S, ds, cl, bl
+
+    def close(self) -> None:
+        if getattr(self, "_h", None) is not None and self._h.value:
+            _check(_lib.tq_codec_destroy(self._h), "tq_codec_destroy")
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def tq_codec_create(d: int, seg_bits: Sequence[int], m: int, seed: int = 0, device: int = 0) -> Codec:
+    return Codec(d, seg_bits, m, seed, device)
+
+
+class Compressed:
+    """Caller-owned compressed rows (device tensors): codes [n, W] uint32 (held
+    as int32), signs [n, m/32], norms [n] fp32, rnorms [n] fp32."""
+
+    def __init__(self, codes: torch.Tensor, signs: Optional[torch.Tensor], norms: torch.Tensor,
+                 rnorms: Optional[torch.Tensor]):
+        self.codes, self.signs, self.norms, self.rnorms = codes, signs, norms, rnorms
+
+    @classmethod
+    def empty(cls, codec: Codec, n: int, device=None) -> "Compressed":
+        device = device if device is not None else torch.device("cuda", codec.device)
+        codes = torch.empty((n, codec.code_words), dtype=torch.int32, device=device)
+        signs = torch.empty((n, codec.sign_words), dtype=torch.int32, device=device) if codec.m else None
+        norms = torch.empty((n,), dtype=torch.float32, device=device)
+        rnorms = torch.empty((n,), dtype=torch.float32, device=device) if codec.m else None
+        return cls(codes, signs, norms, rnorms)
+
+    def struct(self) -> tq_compressed:
+        return tq_compressed(_ptr(self.codes), _ptr(self.signs), _ptr(self.norms), _ptr(self.rnorms))
+
+    def rows(self, r0: int, r1: int) -> "Compressed":
+        sl = lambda t: None if t is None else t[r0:r1]
+        return Compressed(sl(self.codes), sl(self.signs), sl(self.norms), sl(self.rnorms))
+
+
+def tq_quantize(codec: Codec, x: torch.Tensor, out: Compressed, stream=None) -> Compressed:
+    """Compress the rows of x ([n, ld >= d] with unit column stride)."""
+    assert x.dim() == 2 and x.stride(1) == 1, "x must be [n, ld] with contiguous rows"
+    st = out.struct()
+    _check(_lib.tq_quantize(codec.handle, x.data_ptr(), _DTYPES[x.dtype], x.shape[0], x.stride(0),
+                            ctypes.byref(st), _stream(stream)), "tq_quantize")
+    return out
+
+
+def tq_scores_workspace_size(kc: Codec, B: int, Hq: int) -> int:
+    v = ctypes.c_size_t()
+    _check(_lib.tq_scores_workspace_size(kc.handle, B, Hq, ctypes.byref(v)), "tq_scores_workspace_size")
+    return v.value
+
+
+def tq_scores(kc: Codec, q: torch.Tensor, B: int, Hq: int, Hkv: int, T: int, K: Compressed,
+              logits: torch.Tensor, workspace: torch.Tensor, stream=None) -> torch.Tensor:
+    assert q.is_contiguous() and logits.is_contiguous() and logits.dtype == torch.float32
+    st = K.struct()
+    _check(_lib.tq_scores(kc.handle, q.data_ptr(), _DTYPES[q.dtype], B, Hq, Hkv, T, ctypes.byref(st),
+                          logits.data_ptr(), workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                          _stream(stream)), "tq_scores")
+    return logits
+
+
+def tq_attend_workspace_size(kc: Codec, vc: Codec, B: int, Hq: int, Hkv: int, T: int) -> int:
+    v = ctypes.c_size_t()
+    _check(_lib.tq_attend_workspace_size(kc.handle, vc.handle, B, Hq, Hkv, T, ctypes.byref(v)),
+           "tq_attend_workspace_size")
+    return v.value
+
+
+def tq_attend(kc: Codec, vc: Codec, q: torch.Tensor, B: int, Hq: int, Hkv: int, T: int, K: Compressed,
+              V: Compressed, out: torch.Tensor, workspace: torch.Tensor, scale: float = 0.0,
+              stream=None) -> torch.Tensor:
+    assert q.is_contiguous() and out.is_contiguous() and out.dtype == torch.float32
+    ks, vs = K.struct(), V.struct()
+    _check(_lib.tq_attend(kc.handle, vc.handle, q.data_ptr(), _DTYPES[q.dtype], B, Hq, Hkv, T, scale,
+                          ctypes.byref(ks), ctypes.byref(vs), workspace.data_ptr(),
+                          workspace.numel() * workspace.element_size(), out.data_ptr(), _stream(stream)),
+           "tq_attend")
+    return out
+
+
+def workspace(nbytes: int, device) -> torch.Tensor:
+    """A device byte buffer for the *_workspace_size calls."""
+    return torch.empty((max(nbytes, 16),), dtype=torch.uint8, device=device)
+
+
+def c_api():
+    """The loaded ctypes library (for tests of the raw C ABI)."""
+    return _lib

@@ -1,0 +1,63 @@
+// Device helpers shared by the libtq kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "tq_internal.h"
+
+#define TQ_FULL_MASK 0xffffffffu
+
+__device__ __forceinline__ float tq_to_f32(float v) { return v; }
+__device__ __forceinline__ float tq_to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+__device__ __forceinline__ float tq_to_f32(__half v) { return __half2float(v); }
+
+template <typename F>
+__device__ __forceinline__ F tq_warp_sum(F v) {
+#pragma unroll
+  for (int s = 16; s > 0; s >>= 1) v += __shfl_xor_sync(TQ_FULL_MASK, v, s);
+  return v;
+}
+
+template <typename F>
+__device__ __forceinline__ F tq_warp_max(F v) {
+#pragma unroll
+  for (int s = 16; s > 0; s >>= 1) v = max(v, __shfl_xor_sync(TQ_FULL_MASK, v, s));
+  return v;
+}
+
+// Unnormalised Walsh-Hadamard transform (Sylvester order) of a vector spread
+// over a warp: lane `lane` holds coordinates j = lane + 32 k, k < VPL.  Bits 0-4
+// of j are the lane (shuffle butterflies), higher bits are k (in-register
+// butterflies).  With VPL > 16 the in-register stages stop at 16, i.e. the
+// transform is block-diagonal with blocks of 512 coordinates.
+template <int VPL, typename F>
+__device__ __forceinline__ void tq_fwht_warp(F (&v)[VPL], int lane) {
+  constexpr int KB = VPL < 16 ? VPL : 16;
+#pragma unroll
+  for (int h = 1; h < KB; h <<= 1) {
+#pragma unroll
+    for (int k = 0; k < VPL; ++k) {
+      if ((k & h) == 0) {
+        const F a = v[k], b = v[k + h];
+        v[k] = a + b;
+        v[k + h] = a - b;
+      }
+    }
+  }
+#pragma unroll
+  for (int s = 1; s < 32; s <<= 1) {
+#pragma unroll
+    for (int k = 0; k < VPL; ++k) {
+      const F o = __shfl_xor_sync(TQ_FULL_MASK, v[k], s);
+      v[k] = (lane & s) ? (o - v[k]) : (v[k] + o);
+    }
+  }
+}
+
+// D_j = -1 for coordinate j = lane + 32 k  <=>  bit `lane` of dbits[k]
+__device__ __forceinline__ bool tq_dneg(const uint32_t* dbits, int k, int lane) {
+  return (__ldg(dbits + k) >> lane) & 1u;
+}

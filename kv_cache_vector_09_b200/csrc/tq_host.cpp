@@ -1,0 +1,525 @@
+// Host side of libtq: random draws, Lloyd-Max codebooks, codec lifecycle, and
+// the argument checking in front of every kernel launch.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "tq_internal.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+// ------------------------------------------------------------------ random draws
+// splitmix64 (S. Vigna, public domain): the state advances by the golden-ratio
+// increment and every output is the state passed through two xor-shift-multiply
+// rounds and a final xor-shift.
+struct SplitMix64 {
+  uint64_t s;
+  explicit SplitMix64(uint64_t seed) : s(seed) {}
+  uint64_t next() {
+    s += 0x9E3779B97F4A7C15ull;
+    uint64_t z = s;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    return z ^ (z >> 31);
+  }
+};
+
+constexpr uint64_t kSketchSeedXor = 0x5851F42D4C957F2Dull;
+
+// D: sign i is -1 when the top bit of the i-th output is set.
+void draw_signs(uint64_t seed, int d, std::vector<uint32_t>& bits) {
+  bits.assign((d + 31) / 32, 0u);
+  SplitMix64 g(seed);
+  for (int i = 0; i < d; ++i)
+    if (g.next() >> 63) bits[i / 32] |= 1u << (i % 32);
+}
+
+// S: m x d row-major, one normal per pair of outputs by the Box-Muller cosine
+// branch, u1 in (0, 1] and u2 in [0, 1) from the top 53 bits, rounded to fp32.
+void draw_sketch(uint64_t seed, int m, int d, std::vector<float>& S) {
+  S.resize((size_t)m * d);
+  SplitMix64 g(seed ^ kSketchSeedXor);
+  const double two_pi = 6.283185307179586476925286766559;
+  for (size_t k = 0; k < S.size(); ++k) {
+    const double u1 = (double)((g.next() >> 11) + 1) * 0x1.0p-53;
+    const double u2 = (double)(g.next() >> 11) * 0x1.0p-53;
+    S[k] = (float)(std::sqrt(-2.0 * std::log(u1)) * std::cos(two_pi * u2));
+  }
+}
+
+// ----------------------------------------------------------------- Lloyd-Max
+// Gauss-Legendre rule on [-1, 1] by Newton's method on the Legendre recurrence.
+struct GaussLegendre {
+  std::vector<double> x, w;
+  explicit GaussLegendre(int n) : x(n), w(n) {
+    const double pi = 3.14159265358979323846;
+    for (int i = 0; i < n; ++i) {
+      double t = std::cos(pi * (i + 0.75) / (n + 0.5));
+      double dp = 1.0;
+      for (int it = 0; it < 100; ++it) {
+        double p0 = 1.0, p1 = t;
+        for (int k = 2; k <= n; ++k) {
+          const double p2 = ((2.0 * k - 1.0) * t * p1 - (k - 1.0) * p0) / k;
+          p0 = p1;
+          p1 = p2;
+        }
+        dp = n * (t * p1 - p0) / (t * t - 1.0);
+        const double dt = p1 / dp;
+        t -= dt;
+        if (std::fabs(dt) < 1e-16) break;
+      }
+      x[i] = t;
+      w[i] = 2.0 / ((1.0 - t * t) * dp * dp);
+    }
+  }
+};
+
+// The law of z = sqrt(d) u_1 for u uniform on the unit sphere:
+//   f_d(z) = C_d (1 - z^2/d)^((d-3)/2),  |z| < sqrt(d).
+// With z = sqrt(d) sin(theta) the density becomes C_d sqrt(d) cos^(d-2)(theta),
+// a smooth integrand on [-pi/2, pi/2], so Gauss-Legendre converges fast.
+struct SphereMarginal {
+  int d;
+  double sd, cd;
+  GaussLegendre gl{32};
+  explicit SphereMarginal(int d_) : d(d_), sd(std::sqrt((double)d_)) {
+    cd = std::exp(std::lgamma(0.5 * d) - std::lgamma(0.5 * (d - 1))) / std::sqrt(3.14159265358979323846 * d);
+  }
+  double theta(double z) const {
+    const double s = z / sd;
+    return std::asin(s > 1 ? 1.0 : (s < -1 ? -1.0 : s));
+  }
+  // P(a <= z <= b)
+  double prob(double a, double b) const {
+    const double ta = theta(a), tb = theta(b);
+    const int panels = 16;
+    const double h = (tb - ta) / panels;
+    double acc = 0.0;
+    for (int p = 0; p < panels; ++p) {
+      const double c = ta + (p + 0.5) * h;
+      for (size_t k = 0; k < gl.x.size(); ++k) {
+        const double t = c + 0.5 * h * gl.x[k];
+        acc += gl.w[k] * std::pow(std::cos(t), d - 2);
+      }
+    }
+    return cd * sd * 0.5 * h * acc;
+  }
+  // E[z ; a <= z <= b] in closed form: the antiderivative of z f_d(z) is
+  //   -C_d d/(d-1) (1 - z^2/d)^((d-1)/2).
+  double first_moment(double a, double b) const {
+    auto g = [&](double z) {
+      const double t = 1.0 - z * z / d;
+      return t > 0 ? std::exp(0.5 * (d - 1) * std::log1p(-z * z / d)) : 0.0;
+    };
+    return cd * d / (d - 1.0) * (g(a) - g(b));
+  }
+};
+
+}  // namespace
+
+// --------------------------------------------------------------------- errors
+void tq_set_error(const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+}
+
+tq_status tq_fail(tq_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+static tq_status cuda_fail(cudaError_t e, const char* what) {
+  return tq_fail(TQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+extern "C" const char* tq_status_string(tq_status s) {
+  switch (s) {
+    case TQ_OK: return "ok";
+    case TQ_ERR_INVALID_ARG: return "invalid argument";
+    case TQ_ERR_UNSUPPORTED: return "unsupported configuration";
+    case TQ_ERR_NO_MEMORY: return "out of memory";
+    case TQ_ERR_CUDA: return "CUDA error";
+    case TQ_ERR_DEVICE_ASSERT: return "device-side check failed";
+    case TQ_ERR_NOT_CONVERGED: return "Lloyd-Max did not converge";
+  }
+  return "unknown status";
+}
+
+extern "C" const char* tq_last_error_string(void) { return g_last_error.c_str(); }
+
+// ------------------------------------------------------------------- codebook
+static tq_status lloyd_max(int bits, int d, double tol, int max_iter, std::vector<double>& cen) {
+  const SphereMarginal f(d);
+  const int L = 1 << bits, h = L / 2;
+  std::vector<double> c(h), nc(h), b(h + 1);
+  for (int j = 0; j < h; ++j) c[j] = std::min((j + 0.5) * 2.5 / h, 0.9 * f.sd);
+  bool done = false;
+  for (int it = 0; it < max_iter && !done; ++it) {
+    b[0] = 0.0;
+    for (int j = 1; j < h; ++j) b[j] = 0.5 * (c[j - 1] + c[j]);
+    b[h] = f.sd;
+    double delta = 0.0;
+    for (int j = 0; j < h; ++j) {
+      nc[j] = f.first_moment(b[j], b[j + 1]) / f.prob(b[j], b[j + 1]);
+      delta = std::max(delta, std::fabs(nc[j] - c[j]));
+    }
+    c.swap(nc);
+    done = delta < tol;
+  }
+  if (!done) return tq_fail(TQ_ERR_NOT_CONVERGED, "Lloyd-Max: no convergence in %d iterations", max_iter);
+  cen.resize(L);
+  for (int j = 0; j < h; ++j) {
+    cen[h + j] = c[j];
+    cen[h - 1 - j] = -c[j];
+  }
+  return TQ_OK;
+}
+
+extern "C" tq_status tq_make_codebook(int bits, int d, double tol, int max_iter, float* centroids,
+                                      float* boundaries) {
+  if (bits < 1 || bits > 4) return tq_fail(TQ_ERR_INVALID_ARG, "bits must be 1..4 (got %d)", bits);
+  if (d < 4) return tq_fail(TQ_ERR_INVALID_ARG, "d must be >= 4 (got %d)", d);
+  if (!centroids || !boundaries) return tq_fail(TQ_ERR_INVALID_ARG, "null output pointer");
+  if (tol <= 0) tol = 1e-12;
+  if (max_iter <= 0) max_iter = 20000;
+  std::vector<double> cen;
+  const tq_status st = lloyd_max(bits, d, tol, max_iter, cen);
+  if (st != TQ_OK) return st;
+  const int L = 1 << bits;
+  for (int k = 0; k < L; ++k) centroids[k] = (float)cen[k];
+  for (int k = 0; k + 1 < L; ++k) boundaries[k] = (float)(0.5 * (cen[k] + cen[k + 1]));
+  return TQ_OK;
+}
+
+// ---------------------------------------------------------------------- codec
+static bool is_pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
+
+static tq_status check_spec(const tq_spec* s) {
+  if (!s) return tq_fail(TQ_ERR_INVALID_ARG, "null spec");
+  const int d = s->d;
+  if (!(d == 64 || d == 128 || d == 256 || d == 512 || d == 1024 || d == 1536))
+    return tq_fail(TQ_ERR_UNSUPPORTED, "d = %d: need 64, 128, 256, 512, 1024 or 1536", d);
+  if (s->nseg != 1 && s->nseg != 2) return tq_fail(TQ_ERR_INVALID_ARG, "nseg must be 1 or 2");
+  for (int i = 0; i < s->nseg; ++i)
+    if (s->seg_bits[i] < 1 || s->seg_bits[i] > 4)
+      return tq_fail(TQ_ERR_INVALID_ARG, "seg_bits[%d] = %d not in 1..4", i, s->seg_bits[i]);
+  if (s->m < 0 || s->m % 32 != 0 || s->m > TQ_MAX_M)
+    return tq_fail(TQ_ERR_INVALID_ARG, "m = %d: need 0 or a multiple of 32 up to %d", s->m, TQ_MAX_M);
+  return TQ_OK;
+}
+
+static size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+extern "C" tq_status tq_codec_create(const tq_spec* spec, int device, tq_codec** out) {
+  tq_status st = check_spec(spec);
+  if (st != TQ_OK) return st;
+  if (!out) return tq_fail(TQ_ERR_INVALID_ARG, "null output pointer");
+  if (device < -1) return tq_fail(TQ_ERR_INVALID_ARG, "device %d", device);
+  tq_codec* c = new (std::nothrow) tq_codec();
+  if (!c) return tq_fail(TQ_ERR_NO_MEMORY, "host allocation");
+  c->spec = *spec;
+  if (spec->nseg == 1) c->spec.seg_bits[1] = 0;
+  c->device = device;
+  const int d = spec->d, m = spec->m;
+  tq_params& p = c->p;
+  std::memset(&p, 0, sizeof p);
+  p.d = d;
+  p.nseg = spec->nseg;
+  p.seg_len = d / spec->nseg;
+  p.pw = p.seg_len / 32;
+  p.m = m;
+  p.MS = m / 32;
+  p.hblock = is_pow2(d) ? d : TQ_HBLOCK_MAX;
+  p.log2_hblock = 0;
+  while ((1 << p.log2_hblock) < p.hblock) ++p.log2_hblock;
+  p.zscale = (float)std::sqrt((double)d / p.hblock);
+  p.inv_sqrt_d = (float)(1.0 / std::sqrt((double)d));
+  p.inv_sqrt_p = (float)(1.0 / std::sqrt((double)p.hblock));
+  p.qjl_coef = m > 0 ? (float)(std::sqrt(3.14159265358979323846 / 2.0) / m) : 0.0f;
+  int W = 0;
+  for (int s = 0; s < spec->nseg; ++s) {
+    const int bits = spec->seg_bits[s];
+    p.bits[s] = bits;
+    p.segbase[s] = W;
+    W += bits * p.pw;
+    std::vector<double> cen;
+    st = lloyd_max(bits, d, 1e-12, 20000, cen);
+    if (st != TQ_OK) {
+      delete c;
+      return st;
+    }
+    const int L = 1 << bits;
+    c->cen_host[s].resize(L);
+    c->bnd_host[s].resize(L - 1);
+    for (int k = 0; k < TQ_MAX_LEVELS; ++k) p.bnd[s][k] = INFINITY;
+    for (int k = 0; k < L; ++k) {
+      c->cen_host[s][k] = (float)cen[k];
+      p.cen[s][k] = c->cen_host[s][k];
+      p.cmax = std::max(p.cmax, std::fabs(p.cen[s][k]));
+    }
+    for (int k = 0; k + 1 < L; ++k) {
+      c->bnd_host[s][k] = (float)(0.5 * (cen[k] + cen[k + 1]));
+      p.bnd[s][k] = c->bnd_host[s][k];
+    }
+  }
+  p.W = W;
+  draw_signs(spec->seed, d, c->dbits_host);
+  if (m > 0) draw_sketch(spec->seed, m, d, c->S_host);
+
+  if (device >= 0) {
+    int cur = -1;
+    cudaError_t e = cudaGetDevice(&cur);
+    if (e != cudaSuccess) {
+      delete c;
+      return cuda_fail(e, "cudaGetDevice");
+    }
+    if (cur != device) {
+      delete c;
+      return tq_fail(TQ_ERR_INVALID_ARG, "device %d is not the current device (%d)", device, cur);
+    }
+    // one block: S [m][d] | St [d][m] | s_l1 [m] | s_l2 [m] | dbits
+    const int Q = m / 32;
+    std::vector<float> St((size_t)d * m), l1(m), l2(m);
+    for (int lane = 0; lane < 32; ++lane)
+      for (int q = 0; q < Q; ++q) {
+        const int j = lane + 32 * q, col = lane * Q + q;
+        double a1 = 0, a2 = 0;
+        for (int i = 0; i < d; ++i) {
+          const float v = c->S_host[(size_t)j * d + i];
+          St[(size_t)i * m + col] = v;
+          a1 += std::fabs((double)v);
+          a2 += (double)v * v;
+        }
+        l1[col] = (float)(a1 * (1 + 1e-6));
+        l2[col] = (float)(std::sqrt(a2) * (1 + 1e-6));
+      }
+    const size_t oS = 0, oSt = align256(oS + sizeof(float) * (size_t)m * d);
+    const size_t o1 = align256(oSt + sizeof(float) * (size_t)m * d);
+    const size_t o2 = align256(o1 + sizeof(float) * m);
+    const size_t oD = align256(o2 + sizeof(float) * m);
+    const size_t total = align256(oD + sizeof(uint32_t) * c->dbits_host.size());
+    e = cudaMalloc(&c->dev_block, total);
+    if (e != cudaSuccess) {
+      delete c;
+      cudaGetLastError();
+      return tq_fail(TQ_ERR_NO_MEMORY, "cudaMalloc(%zu): %s", total, cudaGetErrorString(e));
+    }
+    char* base = (char*)c->dev_block;
+    e = cudaMemcpy(base + oD, c->dbits_host.data(), sizeof(uint32_t) * c->dbits_host.size(), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess && m > 0) {
+      e = cudaMemcpy(base + oS, c->S_host.data(), sizeof(float) * (size_t)m * d, cudaMemcpyHostToDevice);
+      if (e == cudaSuccess) e = cudaMemcpy(base + oSt, St.data(), sizeof(float) * St.size(), cudaMemcpyHostToDevice);
+      if (e == cudaSuccess) e = cudaMemcpy(base + o1, l1.data(), sizeof(float) * m, cudaMemcpyHostToDevice);
+      if (e == cudaSuccess) e = cudaMemcpy(base + o2, l2.data(), sizeof(float) * m, cudaMemcpyHostToDevice);
+    }
+    if (e != cudaSuccess) {
+      cudaFree(c->dev_block);
+      delete c;
+      return cuda_fail(e, "codec upload");
+    }
+    p.S = (const float*)(base + oS);
+    p.St = (const float*)(base + oSt);
+    p.s_l1 = (const float*)(base + o1);
+    p.s_l2 = (const float*)(base + o2);
+    p.dbits = (const uint32_t*)(base + oD);
+  }
+  *out = c;
+  return TQ_OK;
+}
+
+extern "C" tq_status tq_codec_destroy(tq_codec* c) {
+  if (!c) return TQ_OK;
+  tq_status st = TQ_OK;
+  if (c->dev_block) {
+    int cur = -1;
+    cudaGetDevice(&cur);
+    if (cur != c->device) cudaSetDevice(c->device);
+    const cudaError_t e = cudaFree(c->dev_block);
+    if (cur != c->device && cur >= 0) cudaSetDevice(cur);
+    if (e != cudaSuccess) st = cuda_fail(e, "cudaFree");
+  }
+  delete c;
+  return st;
+}
+
+extern "C" tq_status tq_codec_export(const tq_codec* c, float* S, uint32_t* dsigns, float* cen, float* bnd) {
+  if (!c) return tq_fail(TQ_ERR_INVALID_ARG, "null codec");
+  if (S && c->spec.m > 0) std::copy(c->S_host.begin(), c->S_host.end(), S);
+  if (dsigns) std::copy(c->dbits_host.begin(), c->dbits_host.end(), dsigns);
+  for (int s = 0; s < c->spec.nseg; ++s) {
+    if (cen) cen = std::copy(c->cen_host[s].begin(), c->cen_host[s].end(), cen);
+    if (bnd) bnd = std::copy(c->bnd_host[s].begin(), c->bnd_host[s].end(), bnd);
+  }
+  return TQ_OK;
+}
+
+extern "C" tq_status tq_codec_layout(const tq_codec* c, int* code_words, int* sign_words) {
+  if (!c) return tq_fail(TQ_ERR_INVALID_ARG, "null codec");
+  if (code_words) *code_words = c->p.W;
+  if (sign_words) *sign_words = c->p.MS;
+  return TQ_OK;
+}
+
+// ------------------------------------------------------------ compute checks
+static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+static size_t dtype_size(tq_dtype dt) { return dt == TQ_F32 ? 4 : 2; }
+
+static tq_status check_device_codec(const tq_codec* c, const char* name) {
+  if (!c) return tq_fail(TQ_ERR_INVALID_ARG, "%s: null codec", name);
+  if (c->device < 0) return tq_fail(TQ_ERR_INVALID_ARG, "%s: host-only codec", name);
+  int cur = -1;
+  const cudaError_t e = cudaGetDevice(&cur);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (cur != c->device)
+    return tq_fail(TQ_ERR_INVALID_ARG, "%s: current device %d is not the codec's device %d", name, cur, c->device);
+  return TQ_OK;
+}
+
+static tq_status check_dtype(tq_dtype dt) {
+  if (dt != TQ_F32 && dt != TQ_BF16 && dt != TQ_F16) return tq_fail(TQ_ERR_INVALID_ARG, "dtype %d", (int)dt);
+  return TQ_OK;
+}
+
+static tq_status check_compressed(const tq_codec* c, const tq_compressed* t, const char* name) {
+  if (!t) return tq_fail(TQ_ERR_INVALID_ARG, "%s: null tq_compressed", name);
+  if (!t->codes || !aligned16(t->codes)) return tq_fail(TQ_ERR_INVALID_ARG, "%s.codes null or not 16-byte aligned", name);
+  if (!t->norms || !aligned16(t->norms)) return tq_fail(TQ_ERR_INVALID_ARG, "%s.norms null or not 16-byte aligned", name);
+  if (c->p.m > 0) {
+    if (!t->signs || !aligned16(t->signs))
+      return tq_fail(TQ_ERR_INVALID_ARG, "%s.signs null or not 16-byte aligned (m = %d)", name, c->p.m);
+    if (!t->rnorms || !aligned16(t->rnorms))
+      return tq_fail(TQ_ERR_INVALID_ARG, "%s.rnorms null or not 16-byte aligned (m = %d)", name, c->p.m);
+  }
+  return TQ_OK;
+}
+
+static tq_status launch_status(cudaError_t e, const char* what) {
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  return TQ_OK;
+}
+
+extern "C" tq_status tq_quantize(const tq_codec* c, const void* x, tq_dtype dt, int64_t n, int64_t ld,
+                                 const tq_compressed* out, void* stream) {
+  tq_status st = check_device_codec(c, "tq_quantize");
+  if (st != TQ_OK) return st;
+  if ((st = check_dtype(dt)) != TQ_OK) return st;
+  if (n < 0) return tq_fail(TQ_ERR_INVALID_ARG, "tq_quantize: n = %lld", (long long)n);
+  if (ld < c->p.d) return tq_fail(TQ_ERR_INVALID_ARG, "tq_quantize: ld %lld < d %d", (long long)ld, c->p.d);
+  if ((ld * (int64_t)dtype_size(dt)) % 16 != 0)
+    return tq_fail(TQ_ERR_INVALID_ARG, "tq_quantize: row pitch %lld bytes is not a multiple of 16",
+                   (long long)(ld * (int64_t)dtype_size(dt)));
+  if (n == 0) return TQ_OK;
+  if (!x || !aligned16(x)) return tq_fail(TQ_ERR_INVALID_ARG, "tq_quantize: x null or not 16-byte aligned");
+  if ((st = check_compressed(c, out, "out")) != TQ_OK) return st;
+  return launch_status(tq_launch_quantize(c->p, x, dt, n, ld, *out, (cudaStream_t)stream), "tq_quantize launch");
+}
+
+static size_t qprep_bytes(const tq_params& p, int nq) { return align256(sizeof(float) * (size_t)nq * (p.d + p.m)); }
+
+extern "C" tq_status tq_scores_workspace_size(const tq_codec* kc, int B, int Hq, size_t* bytes) {
+  if (!kc || !bytes) return tq_fail(TQ_ERR_INVALID_ARG, "tq_scores_workspace_size: null argument");
+  if (B < 0 || Hq < 0) return tq_fail(TQ_ERR_INVALID_ARG, "tq_scores_workspace_size: negative size");
+  *bytes = qprep_bytes(kc->p, B * Hq);
+  return TQ_OK;
+}
+
+static tq_status check_heads(int B, int Hq, int Hkv, int64_t T, const char* name) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || T < 0)
+    return tq_fail(TQ_ERR_INVALID_ARG, "%s: bad shape B=%d Hq=%d Hkv=%d T=%lld", name, B, Hq, Hkv, (long long)T);
+  if (Hq % Hkv != 0) return tq_fail(TQ_ERR_INVALID_ARG, "%s: Hq %d not a multiple of Hkv %d", name, Hq, Hkv);
+  if (Hq / Hkv > 32) return tq_fail(TQ_ERR_UNSUPPORTED, "%s: Hq/Hkv = %d above 32", name, Hq / Hkv);
+  if (T > (int64_t)1 << 31) return tq_fail(TQ_ERR_UNSUPPORTED, "%s: T above 2^31", name);
+  return TQ_OK;
+}
+
+extern "C" tq_status tq_scores(const tq_codec* kc, const void* q, tq_dtype dt, int B, int Hq, int Hkv, int64_t T,
+                               const tq_compressed* K, float* logits, void* workspace, size_t ws_bytes,
+                               void* stream) {
+  tq_status st = check_device_codec(kc, "tq_scores");
+  if (st != TQ_OK) return st;
+  if ((st = check_dtype(dt)) != TQ_OK) return st;
+  if ((st = check_heads(B, Hq, Hkv, T, "tq_scores")) != TQ_OK) return st;
+  if (B == 0 || T == 0) return TQ_OK;
+  if (!q || !aligned16(q)) return tq_fail(TQ_ERR_INVALID_ARG, "tq_scores: q null or not 16-byte aligned");
+  if (!logits || !aligned16(logits)) return tq_fail(TQ_ERR_INVALID_ARG, "tq_scores: logits null or not 16-byte aligned");
+  if ((st = check_compressed(kc, K, "K")) != TQ_OK) return st;
+  const size_t need = qprep_bytes(kc->p, B * Hq);
+  if (!workspace || !aligned16(workspace) || ws_bytes < need)
+    return tq_fail(TQ_ERR_INVALID_ARG, "tq_scores: workspace null, misaligned or smaller than %zu bytes", need);
+  const cudaStream_t s = (cudaStream_t)stream;
+  float* qprep = (float*)workspace;
+  cudaError_t e = tq_launch_qprep(kc->p, q, dt, B * Hq, qprep, s);
+  if (e == cudaSuccess) e = tq_launch_scores(kc->p, qprep, B, Hq, Hkv, T, *K, logits, s);
+  return launch_status(e, "tq_scores launch");
+}
+
+static int device_sms(int device) {
+  int v = 0;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || v <= 0) v = 148;
+  return v;
+}
+
+static size_t attend_bytes(const tq_params& kp, int B, int Hq, int nchunk) {
+  return qprep_bytes(kp, B * Hq) + align256(sizeof(float) * (size_t)B * Hq * nchunk * (kp.d + 2));
+}
+
+extern "C" tq_status tq_attend_workspace_size(const tq_codec* kc, const tq_codec* vc, int B, int Hq, int Hkv,
+                                              int64_t T, size_t* bytes) {
+  if (!kc || !vc || !bytes) return tq_fail(TQ_ERR_INVALID_ARG, "tq_attend_workspace_size: null argument");
+  tq_status st = check_heads(B, Hq, Hkv, T, "tq_attend_workspace_size");
+  if (st != TQ_OK) return st;
+  const int nchunk = tq_attend_chunks(B, Hq, Hkv, T, device_sms(kc->device < 0 ? 0 : kc->device));
+  *bytes = attend_bytes(kc->p, B, Hq, nchunk);
+  return TQ_OK;
+}
+
+extern "C" tq_status tq_attend(const tq_codec* kc, const tq_codec* vc, const void* q, tq_dtype dt, int B, int Hq,
+                               int Hkv, int64_t T, float scale, const tq_compressed* K, const tq_compressed* V,
+                               void* workspace, size_t ws_bytes, float* out, void* stream) {
+  tq_status st = check_device_codec(kc, "tq_attend");
+  if (st != TQ_OK) return st;
+  if ((st = check_device_codec(vc, "tq_attend")) != TQ_OK) return st;
+  if (kc->p.d != vc->p.d) return tq_fail(TQ_ERR_INVALID_ARG, "tq_attend: key d %d != value d %d", kc->p.d, vc->p.d);
+  if (kc->p.d > 256) return tq_fail(TQ_ERR_UNSUPPORTED, "tq_attend: d = %d above 256", kc->p.d);
+  if ((st = check_dtype(dt)) != TQ_OK) return st;
+  if ((st = check_heads(B, Hq, Hkv, T, "tq_attend")) != TQ_OK) return st;
+  if (B == 0) return TQ_OK;
+  if (T < 1) return tq_fail(TQ_ERR_INVALID_ARG, "tq_attend: T must be >= 1");
+  if (!std::isfinite(scale) || scale < 0) return tq_fail(TQ_ERR_INVALID_ARG, "tq_attend: scale must be finite and >= 0");
+  if (!q || !aligned16(q)) return tq_fail(TQ_ERR_INVALID_ARG, "tq_attend: q null or not 16-byte aligned");
+  if (!out || !aligned16(out)) return tq_fail(TQ_ERR_INVALID_ARG, "tq_attend: out null or not 16-byte aligned");
+  if ((st = check_compressed(kc, K, "K")) != TQ_OK) return st;
+  if (!V || !V->codes || !aligned16(V->codes) || !V->norms || !aligned16(V->norms))
+    return tq_fail(TQ_ERR_INVALID_ARG, "tq_attend: V.codes / V.norms null or not 16-byte aligned");
+  const int nchunk = tq_attend_chunks(B, Hq, Hkv, T, device_sms(kc->device));
+  const size_t need = attend_bytes(kc->p, B, Hq, nchunk);
+  if (!workspace || !aligned16(workspace) || ws_bytes < need)
+    return tq_fail(TQ_ERR_INVALID_ARG, "tq_attend: workspace null, misaligned or smaller than %zu bytes", need);
+  if (scale == 0.0f) scale = kc->p.inv_sqrt_d;
+  const cudaStream_t s = (cudaStream_t)stream;
+  float* qprep = (float*)workspace;
+  float* partials = (float*)((char*)workspace + qprep_bytes(kc->p, B * Hq));
+  cudaError_t e = tq_launch_qprep(kc->p, q, dt, B * Hq, qprep, s);
+  if (e == cudaSuccess)
+    e = tq_launch_attend(kc->p, vc->p, qprep, B, Hq, Hkv, T, scale, *K, *V, partials, nchunk, out, s);
+  return launch_status(e, "tq_attend launch");
+}

@@ -1,0 +1,69 @@
+// Internal definitions shared by the host code and the kernel launchers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+#include <vector>
+
+#include "../../include/tq.h"
+
+#define TQ_MAX_LEVELS 16
+#define TQ_MAX_M 1024
+#define TQ_HBLOCK_MAX 512  // longest Hadamard block; longer vectors use blocks
+
+// Everything a kernel needs about a codec, passed by value as a kernel argument.
+struct tq_params {
+  int d;          // head dimension
+  int nseg;       // 1 or 2 segments (coordinate halves)
+  int seg_len;    // d / nseg
+  int pw;         // words per bit plane = seg_len / 32
+  int m;          // QJL rows (0: none)
+  int W;          // code words per row
+  int MS;         // sign words per row = m / 32
+  int hblock;     // Hadamard block length p
+  int log2_hblock;
+  int bits[2];    // bits per segment
+  int segbase[2]; // first code word of each segment in a row
+  float zscale;   // sqrt(d / p): z = H(D u) * zscale
+  float inv_sqrt_d;
+  float inv_sqrt_p;
+  float qjl_coef; // sqrt(pi/2) / m
+  float cmax;     // max |centroid| over segments
+  float cen[2][TQ_MAX_LEVELS];
+  float bnd[2][TQ_MAX_LEVELS];  // 2^bits - 1 used, rest +inf
+  const float* S;       // [m][d] row-major
+  const float* St;      // [d][m] transposed, columns permuted: column lane*Q + q = row lane + 32q
+  const float* s_l1;    // [m] sum_i |S_ji| (permuted like St's columns)
+  const float* s_l2;    // [m] ||S_j||_2    (permuted like St's columns)
+  const uint32_t* dbits;  // [ceil(d/32)] bit t of word w set <=> D_{32w+t} = -1
+};
+
+struct tq_codec {
+  tq_spec spec;
+  int device;  // -1: host-only
+  tq_params p;
+  std::vector<float> S_host;        // [m][d]
+  std::vector<uint32_t> dbits_host; // [ceil(d/32)]
+  std::vector<float> cen_host[2];
+  std::vector<float> bnd_host[2];
+  // device allocations (one block)
+  void* dev_block = nullptr;
+};
+
+// thread-local error detail
+void tq_set_error(const char* fmt, ...);
+tq_status tq_fail(tq_status st, const char* fmt, ...);
+
+// launchers implemented in the .cu files; arguments already validated
+cudaError_t tq_launch_quantize(const tq_params& p, const void* x, tq_dtype dt, int64_t n, int64_t ld,
+                               const tq_compressed& out, cudaStream_t st);
+cudaError_t tq_launch_qprep(const tq_params& p, const void* q, tq_dtype dt, int nq, float* qprep,
+                            cudaStream_t st);
+cudaError_t tq_launch_scores(const tq_params& p, const float* qprep, int B, int Hq, int Hkv, int64_t T,
+                             const tq_compressed& K, float* logits, cudaStream_t st);
+int tq_attend_chunks(int B, int Hq, int Hkv, int64_t T, int num_sms);
+cudaError_t tq_launch_attend(const tq_params& kp, const tq_params& vp, const float* qprep, int B, int Hq,
+                             int Hkv, int64_t T, float scale, const tq_compressed& K, const tq_compressed& V,
+                             float* partials, int nchunk, float* out, cudaStream_t st);

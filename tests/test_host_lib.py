@@ -1,0 +1,99 @@
+"""libtq on the host (no GPU): exported symbols, the host Lloyd-Max solver and
+the codec's random draws against the oracle, and argument checking.
+
+The library and the oracle share no code; these tests compare two independent
+implementations of the same definitions (splitmix64 + Box-Muller draws, and a
+Lloyd-Max solver in theta-space with Gauss-Legendre quadrature and a
+closed-form first moment against the oracle's adaptive quadrature in z).
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import kv_cache_vector_09_b200 as tq
+import oracle as O
+from conftest import ROOT
+
+
+def _header_symbols():
+    src = open(os.path.join(ROOT, "include", "tq.h")).read()
+    return sorted(set(re.findall(r"TQ_API\s+[\w\s\*]*?\b(tq_\w+)\s*\(", src)))
+
+
+def test_library_exports_every_header_symbol():
+    syms = _header_symbols()
+    assert len(syms) >= 12, syms
+    lib = ctypes.CDLL(tq.LIB_PATH)
+    for s in syms:
+        assert hasattr(lib, s), s
+
+
+@pytest.mark.parametrize("bits,d", [(1, 64), (2, 64), (2, 128), (3, 128), (4, 128), (3, 1536), (2, 256), (4, 64)])
+def test_host_codebook_matches_oracle(bits, d):
+    cen, bnd = tq.tq_make_codebook(bits, d)
+    oc, ob = O.published_codebook(bits, d)
+    assert np.array_equal(cen, oc), (cen, oc)
+    assert np.array_equal(bnd, ob), (bnd, ob)
+
+
+@pytest.mark.parametrize("d,bits,m,seed", [(128, (2,), 128, 0), (128, (3,), 128, 0), (128, (2, 3), 64, 0),
+                                           (64, (2,), 64, 0), (128, (4,), 0, 0), (1536, (3,), 256, 0),
+                                           (256, (1,), 32, 12345)])
+def test_host_codec_draws_match_oracle(d, bits, m, seed):
+    c = tq.Codec(d, bits, m, seed, device=-1)
+    S, ds, cen, bnd = c.export()
+    oc = O.make_codec(d, bits, m, seed)
+    neg = np.array([(ds[i // 32] >> (i % 32)) & 1 for i in range(d)], dtype=bool)
+    assert np.array_equal(np.where(neg, -1.0, 1.0), oc.D)
+    if m:
+        assert np.array_equal(S, oc.S), np.abs(S - oc.S).max()
+    for s in range(len(bits)):
+        assert np.array_equal(cen[s], oc.cen[s]) and np.array_equal(bnd[s], oc.bnd[s])
+    W = sum(b * (d // len(bits)) // 32 for b in bits)
+    assert c.code_words == W and c.sign_words == m // 32
+    assert c.code_words == oc.words
+
+
+def test_invalid_arguments_are_rejected_on_the_host():
+    lib = tq.c_api()
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_make_codebook(5, 128)
+    assert e.value.status == 1
+    with pytest.raises(tq.TQError) as e:
+        tq.Codec(96, (2,), 64, 0, device=-1)
+    assert e.value.status == 2
+    for bad in [dict(d=128, seg_bits=(0,), m=32), dict(d=128, seg_bits=(2,), m=40),
+                dict(d=128, seg_bits=(2, 2, 2), m=32), dict(d=128, seg_bits=(2,), m=2048)]:
+        with pytest.raises(tq.TQError) as e:
+            tq.Codec(bad["d"], bad["seg_bits"][:3], bad["m"], 0, device=-1) if len(bad["seg_bits"]) <= 2 else \
+                _raw_spec(lib, bad)
+        assert e.value.status == 1
+    # compute calls on a host-only codec fail before touching a GPU
+    c = tq.Codec(128, (2,), 64, 0, device=-1)
+    comp = tq.tq_compressed()
+    st = lib.tq_quantize(c.handle, None, 1, 1, 128, ctypes.byref(comp), None)
+    assert st == 1 and "host-only" in tq.tq_last_error_string()
+    v = ctypes.c_size_t()
+    assert lib.tq_scores_workspace_size(c.handle, 8, 32, ctypes.byref(v)) == 0 and v.value >= 8 * 32 * (128 + 64) * 4
+    assert lib.tq_codec_destroy(None) == 0
+    c.close()
+    c.close()
+    assert tq.tq_status_string(6) == "Lloyd-Max did not converge"
+
+
+def _raw_spec(lib, bad):
+    spec = tq.tq_spec(bad["d"], 3, (ctypes.c_int32 * 2)(2, 2), bad["m"], 0)
+    h = ctypes.c_void_p()
+    st = lib.tq_codec_create(ctypes.byref(spec), -1, ctypes.byref(h))
+    raise tq.TQError(st, "tq_codec_create", tq.tq_last_error_string())
+
+
+def test_not_converged_is_reported():
+    cen = np.zeros(8, np.float32)
+    bnd = np.zeros(7, np.float32)
+    lib = tq.c_api()
+    st = lib.tq_make_codebook(3, 128, 1e-15, 3, cen.ctypes.data, bnd.ctypes.data)
+    assert st == 6 and np.all(cen == 0)
