@@ -124,6 +124,26 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(inside)}
 
 
+def max_over_ranks(dist, value: float, device) -> float:
+    """Maximum of a per-rank scalar over all ranks (identity without a group)."""
+    if dist is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_workload(w: synth.Workload, rank: int) -> synth.Workload:
+    """Each rank processes its own layer: same shapes, its own data seed."""
+    import dataclasses
+    return dataclasses.replace(w, data_seed=w.data_seed + rank)
+
+
+def whole_job_value(units_per_rank: int, world: int, ms_max: float) -> float:
+    """Units processed by all ranks divided by the slowest rank's time."""
+    return units_per_rank * world / (ms_max * 1e-3)
+
+
 def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -136,8 +156,7 @@ class Layer:
     """Device-resident inputs, codecs and outputs of one decode layer."""
 
     def __init__(self, tq, w: synth.Workload, dev: torch.device, rank: int):
-        import dataclasses
-        self.w = w = dataclasses.replace(w, data_seed=w.data_seed + rank)
+        self.w = w = rank_workload(w, rank)
         self.tq = tq
         d = w.d
         self.k_host = synth.kv_full(w, "K").reshape(-1, d)
@@ -328,13 +347,9 @@ def main():
     if pg:
         pg.barrier()
     clocks.stop()
-    ms_step = total_ms / args.steps
-    if pg:
-        t = torch.tensor([ms_step], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms_step = float(t.item())
+    ms_step = max_over_ranks(pg, total_ms / args.steps, dev)
     keys_step = w.n_keys
-    value = keys_step * world / (ms_step * 1e-3)
+    value = whole_job_value(keys_step, world, ms_step)
 
     # end to end through host buffers: pinned K, V, Q copied in, logits and the
     # attention output copied out, every step, on the same stream
@@ -361,11 +376,7 @@ def main():
         pg.barrier()
     torch.cuda.synchronize()
     e2e_ms, _ = time_steps(layer, e2e_steps, stream, e2e_stages, pre, post)
-    e2e_ms /= e2e_steps
-    if pg:
-        t = torch.tensor([e2e_ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(pg, e2e_ms / e2e_steps, dev)
     h2d = kh.numel() * kh.element_size() + vh.numel() * vh.element_size() + qh.numel() * qh.element_size()
     d2h = lh.numel() * 4 + oh.numel() * 4
     del kd, vd
@@ -408,7 +419,7 @@ def main():
         "roofline": roof(dom),
         "roofline_scores": roof("tq_scores"),
         "gpu_launches": args.steps * sum(Layer.LAUNCHES.values()),
-        "e2e": {"value": keys_step * world / (e2e_ms * 1e-3), "unit": "keys/s", "ms_per_step": e2e_ms,
+        "e2e": {"value": whole_job_value(keys_step, world, e2e_ms), "unit": "keys/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "clocks": clocks.summary(t_wall0, t_wall1),
     }
