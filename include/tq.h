@@ -180,6 +180,25 @@ TQ_API tq_status tq_scores(const tq_codec *kc, const void *q, tq_dtype dtype, in
                     float *logits, void *workspace, size_t ws_bytes,
                     void *stream);
 
+/* tq_scores for callers that cannot allocate device memory (no counterpart on
+ * the source pages; it exists for callers such as code under a fixed,
+ * pre-allocated memory budget, plug-ins whose host framework owns every
+ * allocation, or bindings without access to CUDA's allocator).  Same
+ * arguments and result as tq_scores, minus the workspace: the scratch is a
+ * 2 MiB array inside libtq (held on every GPU that loads the library until
+ * the process exits).
+ *   - Calls needing more scratch than that (tq_scores_workspace_size(kc, B, Hq)
+ *     above 2 MiB) return TQ_ERR_UNSUPPORTED and write nothing.
+ *   - The first call on a device looks up the array's device address; make it
+ *     before any stream capture.
+ *   - Every call shares the one array: calls whose kernels may overlap on the
+ *     GPU (other streams, other host threads) race and must be serialised.
+ *   - It calls no allocator (no cudaMalloc, cudaFree or allocating library). */
+TQ_API tq_status tq_scores_noalloc(const tq_codec *kc, const void *q,
+                                   tq_dtype dtype, int B, int Hq, int Hkv,
+                                   int64_t T, const tq_compressed *K,
+                                   float *logits, void *stream);
+
 /* Workspace bytes for tq_attend (depends on the current device's SM count). */
 TQ_API tq_status tq_attend_workspace_size(const tq_codec *kc, const tq_codec *vc,
                                    int B, int Hq, int Hkv, int64_t T,

@@ -4,7 +4,7 @@ This module only marshals arguments for the C ABI declared in ``include/tq.h``
 (same function names); every step of the codec runs in the CUDA kernels of
 ``libtq.so``.  PyTorch supplies device memory and streams.  There is no CPU
 fallback: importing this package fails loudly if ``libtq.so`` is missing
-(build it with ``python -m kv_cache_vector_09_b200.build``).
+(build it with ``python kv_cache_vector_09_b200/build.py``).
 """
 from __future__ import annotations
 
@@ -43,7 +43,7 @@ class tq_compressed(ctypes.Structure):
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m kv_cache_vector_09_b200.build`")
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python kv_cache_vector_09_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     P, I, I64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
     sig = {
@@ -55,11 +55,15 @@ def _load() -> ctypes.CDLL:
         "tq_quantize": [P, P, I, I64, I64, P, P],
         "tq_scores_workspace_size": [P, I, I, ctypes.POINTER(SZ)],
         "tq_scores": [P, P, I, I, I, I, I64, P, P, P, SZ, P],
+        "tq_scores_noalloc": [P, P, I, I, I, I, I64, P, P, P],
         "tq_attend_workspace_size": [P, P, I, I, I, I64, ctypes.POINTER(SZ)],
         "tq_attend": [P, P, P, I, I, I, I, I64, ctypes.c_float, P, P, P, SZ, P, P],
     }
     for name, args in sig.items():
-        fn = getattr(lib, name)
+        try:
+            fn = getattr(lib, name)
+        except AttributeError as e:
+            raise ImportError(f"{LIB_PATH} lacks {name}: rebuild it with `python kv_cache_vector_09_b200/build.py`") from e
         fn.argtypes = args
         fn.restype = ctypes.c_int
     lib.tq_status_string.argtypes = [ctypes.c_int]
@@ -202,6 +206,18 @@ def tq_scores(kc: Codec, q: torch.Tensor, B: int, Hq: int, Hkv: int, T: int, K: 
     _check(_lib.tq_scores(kc.handle, q.data_ptr(), _DTYPES[q.dtype], B, Hq, Hkv, T, ctypes.byref(st),
                           logits.data_ptr(), workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                           _stream(stream)), "tq_scores")
+    return logits
+
+
+def tq_scores_noalloc(kc: Codec, q: torch.Tensor, B: int, Hq: int, Hkv: int, T: int, K: Compressed,
+                      logits: torch.Tensor, stream=None) -> torch.Tensor:
+    """tq_scores without a workspace, for callers that cannot allocate device
+    memory: the library's built-in 2 MiB scratch is used instead.  Calls share
+    that scratch, so calls that may overlap on the GPU must be serialised."""
+    assert q.is_contiguous() and logits.is_contiguous() and logits.dtype == torch.float32
+    st = K.struct()
+    _check(_lib.tq_scores_noalloc(kc.handle, q.data_ptr(), _DTYPES[q.dtype], B, Hq, Hkv, T, ctypes.byref(st),
+                                  logits.data_ptr(), _stream(stream)), "tq_scores_noalloc")
     return logits
 
 

@@ -1,6 +1,6 @@
 """Build libtq.so in-tree with nvcc for sm_100a (B200).
 
-    python -m kv_cache_vector_09_b200.build [--force]
+    python kv_cache_vector_09_b200/build.py [--force] [-v]
 
 The shared library is written next to this file.  The CUDA runtime is linked
 statically, so the library depends only on the driver.
