@@ -334,6 +334,8 @@ def main():
         for _, fn in layer.stages():
             fn()
     torch.cuda.synchronize()
+    exact_k = tq.tq_codec_exact_rows(layer.kc, reset=True) / args.warmup
+    exact_v = tq.tq_codec_exact_rows(layer.vc, reset=True) / args.warmup
 
     clocks = ClockSampler(local)
     clocks.start()
@@ -416,6 +418,7 @@ def main():
         "tokens_quantised_per_s": w.B * w.T * world / ((stages["tq_quantize_K"]["ms"] + stages["tq_quantize_V"]["ms"])
                                                        * 1e-3),
         "stages": stages,
+        "exact_rows_per_call": {"K": exact_k, "V": exact_v, "of": w.n_keys},
         "roofline": roof(dom),
         "roofline_scores": roof("tq_scores"),
         "gpu_launches": args.steps * sum(Layer.LAUNCHES.values()),

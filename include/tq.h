@@ -217,6 +217,22 @@ TQ_API tq_status tq_attend(const tq_codec *kc, const tq_codec *vc, const void *q
                     const tq_compressed *V, void *workspace, size_t ws_bytes,
                     float *out, void *stream);
 
+/* Device-side health of a codec.  Kernels that wait on tensor-core or copy
+ * completion give up after a bounded time (about two seconds), record a
+ * nonzero code in the codec's device error word and return early.  This call
+ * synchronises `stream`, reads the word into *code (0 = healthy, 1 = an MMA
+ * completion wait timed out, 2 = a copy wait timed out), clears it, and
+ * returns TQ_ERR_DEVICE_ASSERT if it was set.                                */
+TQ_API tq_status tq_codec_device_error(const tq_codec *codec, void *stream,
+                                       uint32_t *code);
+
+/* Number of rows tq_quantize has re-evaluated in fp64 with this codec (rows
+ * whose fp32 evaluation left some code or sign decision within its error
+ * bound) since creation or the last reset.  Synchronises `stream`; reset != 0
+ * zeroes the counter after reading it.                                      */
+TQ_API tq_status tq_codec_exact_rows(const tq_codec *codec, void *stream,
+                                     int reset, uint64_t *rows);
+
 /* Human-readable status and the calling thread's last error detail.        */
 TQ_API const char *tq_status_string(tq_status status);
 TQ_API const char *tq_last_error_string(void);

@@ -58,6 +58,8 @@ def _load() -> ctypes.CDLL:
         "tq_scores_noalloc": [P, P, I, I, I, I, I64, P, P, P],
         "tq_attend_workspace_size": [P, P, I, I, I, I64, ctypes.POINTER(SZ)],
         "tq_attend": [P, P, P, I, I, I, I, I64, ctypes.c_float, P, P, P, SZ, P, P],
+        "tq_codec_device_error": [P, P, ctypes.POINTER(ctypes.c_uint32)],
+        "tq_codec_exact_rows": [P, P, I, ctypes.POINTER(ctypes.c_uint64)],
     }
     for name, args in sig.items():
         try:
@@ -238,6 +240,22 @@ def tq_attend(kc: Codec, vc: Codec, q: torch.Tensor, B: int, Hq: int, Hkv: int, 
                           workspace.numel() * workspace.element_size(), out.data_ptr(), _stream(stream)),
            "tq_attend")
     return out
+
+
+def tq_codec_device_error(codec: Codec, stream=None) -> int:
+    """Synchronise, read and clear the codec's device error word (0 = healthy)."""
+    v = ctypes.c_uint32()
+    st = _lib.tq_codec_device_error(codec.handle, _stream(stream), ctypes.byref(v))
+    if st not in (TQ_OK, 5):
+        _check(st, "tq_codec_device_error")
+    return v.value
+
+
+def tq_codec_exact_rows(codec: Codec, reset: bool = False, stream=None) -> int:
+    """Rows tq_quantize re-evaluated in fp64 with this codec (synchronises)."""
+    v = ctypes.c_uint64()
+    _check(_lib.tq_codec_exact_rows(codec.handle, _stream(stream), int(reset), ctypes.byref(v)), "tq_codec_exact_rows")
+    return v.value
 
 
 def workspace(nbytes: int, device) -> torch.Tensor:

@@ -1,5 +1,6 @@
 // Host side of libtq: random draws, Lloyd-Max codebooks, codec lifecycle, and
 // the argument checking in front of every kernel launch.
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -295,27 +296,49 @@ extern "C" tq_status tq_codec_create(const tq_spec* spec, int device, tq_codec**
       delete c;
       return tq_fail(TQ_ERR_INVALID_ARG, "device %d is not the current device (%d)", device, cur);
     }
-    // one block: S [m][d] | St [d][m] | s_l1 [m] | s_l2 [m] | dbits
+    // one block: S [m][d] | St [d][m] | s_l1 [m] | s_l2 [m] | dbits | bimg | dmask | sl1n | sl2n | err
     const int Q = m / 32;
-    std::vector<float> St((size_t)d * m), l1(m), l2(m);
+    std::vector<float> St((size_t)d * m), l1(m), l2(m), l1n(m), l2n(m);
+    for (int j = 0; j < m; ++j) {
+      double a1 = 0, a2 = 0;
+      for (int i = 0; i < d; ++i) {
+        const double v = c->S_host[(size_t)j * d + i];
+        a1 += std::fabs(v);
+        a2 += v * v;
+      }
+      l1n[j] = (float)(a1 * (1 + 1e-6));
+      l2n[j] = (float)(std::sqrt(a2) * (1 + 1e-6));
+    }
     for (int lane = 0; lane < 32; ++lane)
       for (int q = 0; q < Q; ++q) {
         const int j = lane + 32 * q, col = lane * Q + q;
-        double a1 = 0, a2 = 0;
-        for (int i = 0; i < d; ++i) {
-          const float v = c->S_host[(size_t)j * d + i];
-          St[(size_t)i * m + col] = v;
-          a1 += std::fabs((double)v);
-          a2 += (double)v * v;
-        }
-        l1[col] = (float)(a1 * (1 + 1e-6));
-        l2[col] = (float)(std::sqrt(a2) * (1 + 1e-6));
+        for (int i = 0; i < d; ++i) St[(size_t)i * m + col] = c->S_host[(size_t)j * d + i];
+        l1[col] = l1n[j];
+        l2[col] = l2n[j];
       }
+    // fp16 split S = S_hi + S_lo (+ error <= 2^-22 |S| + 2^-25) in the tensor-core operand layout
+    std::vector<uint16_t> bimg(2 * (size_t)m * d);
+    for (int j = 0; j < m; ++j)
+      for (int i = 0; i < d; ++i) {
+        const float v = c->S_host[(size_t)j * d + i];
+        const __half hi = __float2half_rn(v);
+        const __half lo = __float2half_rn(v - __half2float(hi));
+        const size_t off = ((size_t)(i / 8) * 16 * m + (size_t)(j / 8) * 128 + (j % 8) * 16 + (i % 8) * 2) / 2;
+        bimg[off] = __half_as_ushort(hi);
+        bimg[(size_t)m * d + off] = __half_as_ushort(lo);
+      }
+    std::vector<uint32_t> dmask(d);
+    for (int i = 0; i < d; ++i) dmask[i] = ((c->dbits_host[i / 32] >> (i % 32)) & 1u) ? 0x80000000u : 0u;
     const size_t oS = 0, oSt = align256(oS + sizeof(float) * (size_t)m * d);
     const size_t o1 = align256(oSt + sizeof(float) * (size_t)m * d);
     const size_t o2 = align256(o1 + sizeof(float) * m);
     const size_t oD = align256(o2 + sizeof(float) * m);
-    const size_t total = align256(oD + sizeof(uint32_t) * c->dbits_host.size());
+    const size_t oB = align256(oD + sizeof(uint32_t) * c->dbits_host.size());
+    const size_t oM = align256(oB + sizeof(uint16_t) * bimg.size());
+    const size_t o1n = align256(oM + sizeof(uint32_t) * d);
+    const size_t o2n = align256(o1n + sizeof(float) * m);
+    const size_t oE = align256(o2n + sizeof(float) * m);
+    const size_t total = align256(oE + 16);
     e = cudaMalloc(&c->dev_block, total);
     if (e != cudaSuccess) {
       delete c;
@@ -323,12 +346,18 @@ extern "C" tq_status tq_codec_create(const tq_spec* spec, int device, tq_codec**
       return tq_fail(TQ_ERR_NO_MEMORY, "cudaMalloc(%zu): %s", total, cudaGetErrorString(e));
     }
     char* base = (char*)c->dev_block;
-    e = cudaMemcpy(base + oD, c->dbits_host.data(), sizeof(uint32_t) * c->dbits_host.size(), cudaMemcpyHostToDevice);
+    e = cudaMemset(base, 0, total);
+    if (e == cudaSuccess)
+      e = cudaMemcpy(base + oD, c->dbits_host.data(), sizeof(uint32_t) * c->dbits_host.size(), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemcpy(base + oM, dmask.data(), sizeof(uint32_t) * d, cudaMemcpyHostToDevice);
     if (e == cudaSuccess && m > 0) {
       e = cudaMemcpy(base + oS, c->S_host.data(), sizeof(float) * (size_t)m * d, cudaMemcpyHostToDevice);
       if (e == cudaSuccess) e = cudaMemcpy(base + oSt, St.data(), sizeof(float) * St.size(), cudaMemcpyHostToDevice);
       if (e == cudaSuccess) e = cudaMemcpy(base + o1, l1.data(), sizeof(float) * m, cudaMemcpyHostToDevice);
       if (e == cudaSuccess) e = cudaMemcpy(base + o2, l2.data(), sizeof(float) * m, cudaMemcpyHostToDevice);
+      if (e == cudaSuccess) e = cudaMemcpy(base + oB, bimg.data(), sizeof(uint16_t) * bimg.size(), cudaMemcpyHostToDevice);
+      if (e == cudaSuccess) e = cudaMemcpy(base + o1n, l1n.data(), sizeof(float) * m, cudaMemcpyHostToDevice);
+      if (e == cudaSuccess) e = cudaMemcpy(base + o2n, l2n.data(), sizeof(float) * m, cudaMemcpyHostToDevice);
     }
     if (e != cudaSuccess) {
       cudaFree(c->dev_block);
@@ -340,6 +369,12 @@ extern "C" tq_status tq_codec_create(const tq_spec* spec, int device, tq_codec**
     p.s_l1 = (const float*)(base + o1);
     p.s_l2 = (const float*)(base + o2);
     p.dbits = (const uint32_t*)(base + oD);
+    p.bimg = (const uint16_t*)(base + oB);
+    p.dmask = (const uint32_t*)(base + oM);
+    p.sl1n = (const float*)(base + o1n);
+    p.sl2n = (const float*)(base + o2n);
+    p.err = (uint32_t*)(base + oE);
+    p.exact_rows = (unsigned long long*)(base + oE + 8);
   }
   *out = c;
   return TQ_OK;
@@ -430,7 +465,9 @@ extern "C" tq_status tq_quantize(const tq_codec* c, const void* x, tq_dtype dt, 
   if (n == 0) return TQ_OK;
   if (!x || !aligned16(x)) return tq_fail(TQ_ERR_INVALID_ARG, "tq_quantize: x null or not 16-byte aligned");
   if ((st = check_compressed(c, out, "out")) != TQ_OK) return st;
-  return launch_status(tq_launch_quantize(c->p, x, dt, n, ld, *out, (cudaStream_t)stream), "tq_quantize launch");
+  cudaError_t e = tq_launch_quantize_tc(c->p, x, dt, n, ld, *out, (cudaStream_t)stream);
+  if (e == cudaErrorNotSupported) e = tq_launch_quantize(c->p, x, dt, n, ld, *out, (cudaStream_t)stream);
+  return launch_status(e, "tq_quantize launch");
 }
 
 static size_t qprep_bytes(const tq_params& p, int nq) { return align256(sizeof(float) * (size_t)nq * (p.d + p.m)); }
@@ -522,4 +559,33 @@ extern "C" tq_status tq_attend(const tq_codec* kc, const tq_codec* vc, const voi
   if (e == cudaSuccess)
     e = tq_launch_attend(kc->p, vc->p, qprep, B, Hq, Hkv, T, scale, *K, *V, partials, nchunk, out, s);
   return launch_status(e, "tq_attend launch");
+}
+
+extern "C" tq_status tq_codec_device_error(const tq_codec* c, void* stream, uint32_t* code) {
+  tq_status st = check_device_codec(c, "tq_codec_device_error");
+  if (st != TQ_OK) return st;
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "tq_codec_device_error: stream sync");
+  uint32_t v = 0;
+  e = cudaMemcpy(&v, c->p.err, sizeof v, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "tq_codec_device_error: read");
+  if (v != 0) {
+    const uint32_t zero = 0;
+    e = cudaMemcpy(c->p.err, &zero, sizeof zero, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e, "tq_codec_device_error: clear");
+  }
+  if (code) *code = v;
+  if (v != 0) return tq_fail(TQ_ERR_DEVICE_ASSERT, "device error code %u (a bounded wait timed out)", v);
+  return TQ_OK;
+}
+
+extern "C" tq_status tq_codec_exact_rows(const tq_codec* c, void* stream, int reset, uint64_t* rows) {
+  tq_status st = check_device_codec(c, "tq_codec_exact_rows");
+  if (st != TQ_OK) return st;
+  if (!rows) return tq_fail(TQ_ERR_INVALID_ARG, "tq_codec_exact_rows: null output");
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e == cudaSuccess) e = cudaMemcpy(rows, c->p.exact_rows, sizeof(uint64_t), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && reset) e = cudaMemset(c->p.exact_rows, 0, sizeof(uint64_t));
+  if (e != cudaSuccess) return cuda_fail(e, "tq_codec_exact_rows");
+  return TQ_OK;
 }

@@ -38,6 +38,14 @@ struct tq_params {
   const float* s_l1;    // [m] sum_i |S_ji| (permuted like St's columns)
   const float* s_l2;    // [m] ||S_j||_2    (permuted like St's columns)
   const uint32_t* dbits;  // [ceil(d/32)] bit t of word w set <=> D_{32w+t} = -1
+  // tables of the tensor-core quantiser (m <= 256, d <= 128)
+  const uint16_t* bimg;   // fp16 S_hi then S_lo, each [m][d] in the K-major no-swizzle
+                          // core-matrix layout: (j, i) at (i/8)*16m + (j/8)*128 + (j%8)*16 + (i%8)*2 bytes
+  const uint32_t* dmask;  // [d] 0x80000000 where D_i = -1, else 0
+  const float* sl1n;      // [m] sum_i |S_ji| (natural row order)
+  const float* sl2n;      // [m] ||S_j||_2
+  uint32_t* err;          // device error word (bounded waits that gave up), zero when healthy
+  unsigned long long* exact_rows;  // rows re-evaluated in fp64 since the last reset
 };
 
 struct tq_codec {
@@ -59,6 +67,10 @@ tq_status tq_fail(tq_status st, const char* fmt, ...);
 // launchers implemented in the .cu files; arguments already validated
 cudaError_t tq_launch_quantize(const tq_params& p, const void* x, tq_dtype dt, int64_t n, int64_t ld,
                                const tq_compressed& out, cudaStream_t st);
+// tensor-core quantiser; returns cudaErrorNotSupported when the codec or dtype
+// has no tensor-core variant (the caller then uses the generic kernel)
+cudaError_t tq_launch_quantize_tc(const tq_params& p, const void* x, tq_dtype dt, int64_t n, int64_t ld,
+                                  const tq_compressed& out, cudaStream_t st);
 cudaError_t tq_launch_qprep(const tq_params& p, const void* q, tq_dtype dt, int nq, float* qprep,
                             cudaStream_t st);
 cudaError_t tq_launch_scores(const tq_params& p, const float* qprep, int B, int Hq, int Hkv, int64_t T,

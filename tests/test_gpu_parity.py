@@ -40,6 +40,7 @@ def gpu_quantize(codec, x_cpu: torch.Tensor, ld_pad: int = 0):
     out = tq.Compressed.empty(codec, n)
     tq.tq_quantize(codec, xg, out)
     torch.cuda.synchronize()
+    assert tq.tq_codec_device_error(codec) == 0
     return out
 
 
