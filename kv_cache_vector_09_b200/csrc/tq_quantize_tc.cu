@@ -1,51 +1,56 @@
-// Tensor-core quantiser: one thread per row, 128 rows per tile (= TMEM lanes).
+// Tensor-core quantiser for d in {64, 128}.
 //
-// Per row (thread): load x, apply the D signs, in-register Walsh-Hadamard
-// transform of the unnormalised vector w = H (D x), quantise every coordinate
-// against the boundaries scaled by the fp32 norm (z_i >= bnd_k  <=>  w_i >= nu
-// bnd_k), pack the bit planes, and form the residual r = w - nu cen[code].
-// The QJL sketch t = S r of the whole tile is one tensor-core product: r is
-// written to TMEM as fp16 hi + lo (r = hi + lo to 2^-22), S comes from shared
-// memory as fp16 hi + lo, and three passes (hi*hi, lo*hi, hi*lo) accumulate
-// t in fp32 TMEM.
+// A block owns tiles of 128 rows; TPR = d/32 threads share a row (4 for
+// d = 128), each holding 32 coordinates: chunks c = q + TPR k (k < 4) of 8
+// consecutive coordinates, q = thread index within the row.  Per row:
+//   load x (16-byte loads, a quad covers 64 contiguous bytes), apply the D
+//   signs, Walsh-Hadamard transform of the unnormalised w = H (D x) (five
+//   in-register butterfly stages over the chunk/element bits, log2 TPR
+//   shuffle stages over the thread bits), quantise every coordinate against the
+//   boundaries scaled by the fp32 norm (z >= bnd <=> w >= nu bnd) with a
+//   magnitude binary search, pack the bit planes into a shared-memory staging
+//   row, and (keys) form the residual r = w - nu cen[code] as fp16 hi + lo in
+//   the tensor-core operand layout.
+// The QJL sketch t = S r of the tile is one kind::f16 tcgen05.mma product
+// (A = residual tile, B = fp16 hi + lo image of S, both in shared memory;
+// passes hi*hi + lo*hi + hi*lo) with an fp32 accumulator in TMEM, read back by
+// the warps one 32-column sign word at a time.
 //
-// Every code and sign decision carries a rigorous bound on its fp32 error:
-//   w_i   : |dw| <= L u ||x||_1 <= L u sqrt(d) nu   (L = log2 d butterfly stages,
-//           each stage's nodes partition the inputs; u = 2^-24)
-//   nu    : relative error <= e_nu = (d/16 + 3) u    (8 partial sums + sqrt)
-//   code  : certain when |w_i - nu bnd_k| > A + B |w_i| for every boundary,
-//           A = 1.1 L u sqrt(d) nu, B = 1.1 (e_nu + 2u)
-//   t_j   : certain when |t_j| > 1.1 (||S_j||_1 E_r + 2^-17.8 ||S_j||_2 ||r|| + ...)
-//           with E_r the per-coordinate residual bound (see below).
-// Rows with any uncertain decision (and rows whose squared norm leaves
-// [1e-30, 1e30]) are recomputed in fp64 by a warp, after the tile.
+// Certified decisions (u = 2^-24, L = log2 d, nu the fp32 norm):
+//   code  : |w_i - nu bnd| > A + B |w_i| with A = 1.1 L u sqrt(d) nu (fp32 FWHT
+//           rounding: each stage's nodes partition the inputs, and
+//           ||x||_1 <= sqrt(d) nu), B = 1.1 (e_nu + 2u), e_nu = 10u
+//   sign  : |t_j| > ||S_j||_2 E + G, where E bounds ||dr||_2 of the scaled
+//           residual (FWHT: ||dw||_2 <= L u sqrt(d) nu, since every stage's
+//           rounding vector has norm <= u ||v_stage|| and the remaining
+//           butterflies scale norms by exactly sqrt(2) each; norm error
+//           (e_nu + u) ||cv||_2; subtraction u ||r||_2; fp16 split 2^-22 ||r||
+//           + 2^-25 sqrt(d)) plus the tensor-core terms (S split 2^-22, omitted
+//           lo*lo 2^-22, fp32 accumulation <= 2^-18 of sum |S r|) times ||r||.
+// A row with an uncertain code is recomputed entirely in fp64; a row with only
+// uncertain signs gets those sketch rows recomputed in fp64 (exact residual).
 #include <math.h>
 
 #include <algorithm>
+#include <type_traits>
 
 #include "tq_common.cuh"
 #include "tq_tc.cuh"
 
 namespace {
 
-constexpr int kTile = 128;
+constexpr int kRows = 128;                     // rows per tile (= MMA M)
 constexpr float kU = 5.9604644775390625e-08f;  // 2^-24
 
-struct QBook {  // codebook copy in shared memory
+struct QBook {
   float cen[2][TQ_MAX_LEVELS];
   float bnd[2][TQ_MAX_LEVELS];
 };
 
-// ---------------------------------------------------------------- helpers
-template <int BITS>
-struct Mag {
-  static constexpr int H = 1 << (BITS - 1);  // centroids per sign
-};
-
-// Magnitude search for one coordinate: a = |w|, mt[k] = nu * (k-th positive
-// boundary), k = 1..H-1.  Returns the magnitude cell m and the distance to the
-// nearest compared boundary (the zero boundary included): the compared
-// boundaries include both ends of the final cell.
+// Magnitude search: a = |w|, mt[k] = nu * (k-th positive boundary), k >= 1.
+// Returns the cell m and the distance to the nearest compared boundary (the
+// zero boundary included); the compared boundaries include both ends of the
+// final cell.
 template <int BITS>
 __device__ __forceinline__ void mag_search(float a, const float* mt, int& m, float& margin) {
   if constexpr (BITS == 1) {
@@ -78,19 +83,37 @@ __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
 }
 
 __device__ __forceinline__ float2 unpack_half2(uint32_t v) {
-  const __half2 h = *reinterpret_cast<const __half2*>(&v);
-  return __half22float2(h);
+  return __half22float2(*reinterpret_cast<const __half2*>(&v));
 }
 
-template <typename TIn>
-__device__ __forceinline__ void load_row(const TIn* __restrict__ xr, float* v, int D, const uint32_t* dm);
+// Shared-memory layout of one block (all offsets 16-byte aligned).
+struct QLayout {
+  uint32_t a_hi, a_lo, bimg, codes, signs, nu, gam, err, flag, fmask, scratch, total;
+  __host__ __device__ QLayout(int D, int m, int W, int nwarps) {
+    uint32_t o = 0;
+    const uint32_t atile = m > 0 ? (uint32_t)kRows * D * 2 : 0;
+    a_hi = o; o += atile;
+    a_lo = o; o += atile;
+    bimg = o; o += (uint32_t)m * D * 4;
+    codes = o; o += (uint32_t)kRows * W * 4;
+    signs = o; o += (uint32_t)kRows * 8 * 4;
+    nu = o; o += kRows * 4;
+    gam = o; o += kRows * 4;
+    err = o; o += kRows * 8;       // per row: E, G of the sign bound
+    flag = o; o += kRows * 4;      // per row: 1 = uncertain sign(s), 2 = uncertain code / range
+    fmask = o; o += kRows * 8 * 4; // per row: uncertain sign bits
+    scratch = o; o += (uint32_t)nwarps * D * 8;
+    total = (o + 127) & ~127u;
+  }
+};
 
-// --------------------------------------------------------- exact fp64 row
-// Warp-cooperative fp64 evaluation of one row (all decisions exact up to
-// ties at ~1e-16), writing every output of the row.
+// ------------------------------------------------------------ exact fp64
+// Warp-cooperative fp64 evaluation of one row, written straight to the
+// outputs.  full: every code, sign, nu and gamma is rewritten; otherwise the
+// codes are certified and only the sign bits in fmask (plus nu and gamma) are.
 template <int D, typename TIn>
-__device__ void exact_row_fp64(const tq_params& p, const QBook& qb, const TIn* __restrict__ xr, int64_t row,
-                               const tq_compressed& out, double* scratch) {
+__device__ void exact_row(const tq_params& p, const QBook& qb, const TIn* __restrict__ xr, int64_t row, bool full,
+                          const uint32_t* fmask, const tq_compressed& out, double* scratch) {
   constexpr int VPL = D / 32;
   const int lane = threadIdx.x & 31;
   double v[VPL];
@@ -108,7 +131,7 @@ __device__ void exact_row_fp64(const tq_params& p, const QBook& qb, const TIn* _
     const double u = v[k] * inv;
     v[k] = tq_dneg(p.dbits, k, lane) ? -u : u;
   }
-  tq_fwht_warp<VPL>(v, lane);  // v = z = H (D u) (p = d here)
+  tq_fwht_warp<VPL>(v, lane);  // z = H (D u)
   const double isd = 1.0 / sqrt((double)D);
   int code[VPL];
   double g2 = 0.0;
@@ -125,170 +148,208 @@ __device__ void exact_row_fp64(const tq_params& p, const QBook& qb, const TIn* _
   }
   g2 = tq_warp_sum(g2);
   __syncwarp();
-  const int Q = p.MS;
-  uint32_t signword = 0;
-  for (int q = 0; q < Q; ++q) {
-    const float* sc = p.St + lane * Q + q;
-    double t = 0.0;
-    for (int i = 0; i < D; ++i) t = fma((double)__ldg(sc + (size_t)i * p.m), scratch[i], t);
-    const uint32_t wv = __ballot_sync(TQ_FULL_MASK, t >= 0.0);
-    if (lane == q) signword = wv;
+  // sketch rows t_j = sum_i S_ji r_i: lanes split i, warp reduction
+  const int MS = p.MS;
+  for (int w = 0; w < MS; ++w) {
+    uint32_t todo = full ? 0xffffffffu : fmask[w];
+    if (!todo) continue;
+    uint32_t word = full ? 0u : out.signs[row * MS + w];
+    while (todo) {
+      const int jj = __ffs(todo) - 1;
+      todo &= todo - 1;
+      const float* Sj = p.S + (size_t)(32 * w + jj) * D;
+      double t = 0.0;
+#pragma unroll
+      for (int k = 0; k < VPL; ++k) t = fma((double)__ldg(Sj + lane + 32 * k), scratch[lane + 32 * k], t);
+      t = tq_warp_sum(t);
+      word = (word & ~(1u << jj)) | ((t >= 0.0 ? 1u : 0u) << jj);
+    }
+    if (lane == 0) out.signs[row * MS + w] = word;
   }
-  __syncwarp();
-  // pack: coordinate j = lane + 32k is bit `lane` of word k of its plane
-  constexpr int SLOTS = (VPL * 4 + 31) / 32;
-  uint32_t cw[SLOTS];
+  if (full) {
+    // coordinate j = lane + 32k is bit `lane` of word k of its plane
 #pragma unroll
-  for (int sl = 0; sl < SLOTS; ++sl) cw[sl] = 0;
-#pragma unroll
-  for (int k = 0; k < VPL; ++k) {
-    const int s = (p.nseg == 2 && k >= VPL / 2) ? 1 : 0;
-    const int kk = s ? k - VPL / 2 : k;
-    for (int pl = 0; pl < p.bits[s]; ++pl) {
-      const uint32_t wv = __ballot_sync(TQ_FULL_MASK, (code[k] >> pl) & 1);
-      const int widx = p.segbase[s] + pl * p.pw + kk;
-#pragma unroll
-      for (int sl = 0; sl < SLOTS; ++sl)
-        if (sl == (widx >> 5) && lane == (widx & 31)) cw[sl] = wv;
+    for (int k = 0; k < VPL; ++k) {
+      const int s = (p.nseg == 2 && k >= VPL / 2) ? 1 : 0;
+      const int kk = s ? k - VPL / 2 : k;
+      for (int pl = 0; pl < p.bits[s]; ++pl) {
+        const uint32_t wv = __ballot_sync(TQ_FULL_MASK, (code[k] >> pl) & 1);
+        if (lane == 0) out.codes[row * p.W + p.segbase[s] + pl * p.pw + kk] = wv;
+      }
     }
   }
-  uint32_t* orow = out.codes + row * p.W;
-#pragma unroll
-  for (int sl = 0; sl < SLOTS; ++sl)
-    if (sl * 32 + lane < p.W) orow[sl * 32 + lane] = cw[sl];
-  if (Q > 0) {
-    if (lane < Q) out.signs[row * Q + lane] = signword;
-    if (lane == 0) out.rnorms[row] = (float)sqrt(g2);
+  if (lane == 0) {
+    out.norms[row] = (float)nu;
+    if (MS > 0) out.rnorms[row] = (float)sqrt(g2);
   }
-  if (lane == 0) out.norms[row] = (float)nu;
+  __syncwarp();
 }
 
+struct FixEntry {
+  int64_t row;
+  int full;
+  uint32_t fmask[8];
+};
+constexpr int kFixCap = 256;
+
 // ---------------------------------------------------------------- kernel
-template <int D, int B0, int B1, typename TIn>
-__global__ void __launch_bounds__(kTile, 2)
-    tq_quantize_tc_kernel(const tq_params p, const TIn* __restrict__ x, const int64_t n, const int64_t ld,
-                          const tq_compressed out, const int64_t ntiles, const uint32_t tmem_cols) {
+template <int D, int B0, int B1, bool SK, typename TIn>
+__global__ void __launch_bounds__(kRows * (D / 32), SK ? 1 : 2)
+    tq_quantize_quad_kernel(const tq_params p, const TIn* __restrict__ x, const int64_t n, const int64_t ld,
+                            const tq_compressed out, const int64_t ntiles, const uint32_t tmem_cols) {
+  constexpr int TPR = D / 32;
+  constexpr int NT = kRows * TPR;
+  constexpr int NW = NT / 32;
   constexpr int NSEG = B1 > 0 ? 2 : 1;
-  constexpr int SEGLEN = D / NSEG;
-  constexpr int PW = SEGLEN / 32;
+  constexpr int NCH = D / 8;
+  constexpr int CHSEG = NCH / NSEG;
+  constexpr int PW = (D / NSEG) / 32;
   constexpr int W = (B0 + B1) * PW;
   constexpr int L = (D == 64) ? 6 : 7;
   constexpr int H0 = 1 << (B0 - 1);
   constexpr int H1 = B1 > 0 ? (1 << (B1 - 1)) : 1;
+  constexpr int LBO_A = (kRows / 8) * 128;
 
   extern __shared__ __align__(1024) unsigned char smem[];
   __shared__ QBook qb;
-  __shared__ uint32_t s_dmask[D];
-  __shared__ int s_list[kTile];
-  __shared__ int s_count;
+  __shared__ __align__(16) uint32_t s_dmask[D];
+  __shared__ FixEntry s_fix[kFixCap];
+  __shared__ int s_nfix;
   __shared__ int s_abort;
   __shared__ uint64_t s_bar;
   __shared__ uint32_t s_tmem;
 
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int m = p.m;
-  const bool sketch = m > 0;
-  // shared layout: B image (2 m D halves) | sl1 [m] | sl2 [m] | fp64 scratch [4][D]
-  uint16_t* s_bimg = reinterpret_cast<uint16_t*>(smem);
-  float* s_sl1 = reinterpret_cast<float*>(smem + (size_t)4 * m * D);
-  float* s_sl2 = s_sl1 + m;
-  double* s_scr = reinterpret_cast<double*>(smem + (size_t)4 * m * D + (size_t)8 * m) + (size_t)warp * D;
+  const int m = SK ? p.m : 0;
+  const QLayout ly(D, m, W, NW);
+  uint32_t* st_codes = reinterpret_cast<uint32_t*>(smem + ly.codes);
+  uint32_t* st_signs = reinterpret_cast<uint32_t*>(smem + ly.signs);
+  float* st_nu = reinterpret_cast<float*>(smem + ly.nu);
+  float* st_gam = reinterpret_cast<float*>(smem + ly.gam);
+  float2* st_err = reinterpret_cast<float2*>(smem + ly.err);
+  int* st_flag = reinterpret_cast<int*>(smem + ly.flag);
+  uint32_t* st_fmask = reinterpret_cast<uint32_t*>(smem + ly.fmask);
 
-  for (int i = tid; i < 2 * TQ_MAX_LEVELS; i += kTile) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int r = tid / TPR, q = tid % TPR;
+
+  for (int i = tid; i < 2 * TQ_MAX_LEVELS; i += NT) {
     qb.cen[i / TQ_MAX_LEVELS][i % TQ_MAX_LEVELS] = p.cen[i / TQ_MAX_LEVELS][i % TQ_MAX_LEVELS];
     qb.bnd[i / TQ_MAX_LEVELS][i % TQ_MAX_LEVELS] = p.bnd[i / TQ_MAX_LEVELS][i % TQ_MAX_LEVELS];
   }
-  for (int i = tid; i < D; i += kTile) s_dmask[i] = __ldg(p.dmask + i);
+  for (int i = tid; i < D; i += NT) s_dmask[i] = __ldg(p.dmask + i);
+  for (int i = tid; i < kRows; i += NT) st_flag[i] = 0;
   if (tid == 0) {
-    s_count = 0;
+    s_nfix = 0;
     s_abort = 0;
   }
-  if (sketch) {
+  if constexpr (SK) {
     const uint4* src = reinterpret_cast<const uint4*>(p.bimg);
-    uint4* dst = reinterpret_cast<uint4*>(s_bimg);
-    for (int i = tid; i < m * D * 4 / 16; i += kTile) dst[i] = __ldg(src + i);
-    for (int i = tid; i < m; i += kTile) {
-      s_sl1[i] = __ldg(p.sl1n + i);
-      s_sl2[i] = __ldg(p.sl2n + i);
-    }
+    uint4* dst = reinterpret_cast<uint4*>(smem + ly.bimg);
+    for (int i = tid; i < m * D * 4 / 16; i += NT) dst[i] = __ldg(src + i);
     if (tid == 0) {
       tqtc::mbar_init(&s_bar, 1);
       tqtc::fence_mbar_init();
     }
     if (warp == 0) tqtc::tmem_alloc(&s_tmem, tmem_cols);
-    tqtc::fence_proxy_async_smem();
   }
   tqtc::tc_fence_before();
   __syncthreads();
   tqtc::tc_fence_after();
-  const uint32_t tbase = sketch ? s_tmem : 0u;
-  const uint32_t lane_base = (uint32_t)(warp * 32);
-  const uint32_t col_lo = D / 2, col_d = D;
+  const uint32_t tbase = SK ? s_tmem : 0u;
   uint32_t phase = 0;
-
-  // positive boundaries qb.bnd[s][H + k - 1] (k >= 1) and positive centroids
-  // qb.cen[s][H + m] are read from shared memory
-  const float e_nu = (float)(D / 16 + 3) * kU;
+  const float e_nu = 10.f * kU;
   const float Bc = 1.1f * (e_nu + 2.f * kU);
   const float sqrtD = sqrtf((float)D);
-  const float cmax = p.cmax;
+  const float sgn1 = (q & 1) ? -1.f : 1.f;
+  const float sgn2 = (q & 2) ? -1.f : 1.f;
+  double* scr = reinterpret_cast<double*>(smem + ly.scratch) + (size_t)warp * D;
+  // fp64 re-evaluation of the queued rows, all warps at once (after the fast
+  // path of those rows has been written and made visible by a barrier)
+  auto drain = [&]() {
+    const int cnt = min(s_nfix, kFixCap);
+    if (tid == 0 && cnt > 0) atomicAdd(p.exact_rows, (unsigned long long)cnt);
+    for (int e = warp; e < cnt; e += NW) {
+      const FixEntry& f = s_fix[e];
+      exact_row<D, TIn>(p, qb, x + f.row * ld, f.row, f.full != 0, f.fmask, out, scr);
+    }
+    __syncthreads();
+    if (tid == 0) s_nfix = 0;
+    __syncthreads();
+  };
 
-  for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-    const int64_t row = tile * kTile + tid;
-    const bool valid = row < n;
-    // ---------------------------------------------------------- load
-    float v[D];
-    if (valid) {
-      const TIn* xr = x + row * ld;
-      if constexpr (sizeof(TIn) == 2) {
+  // prefetch of the first tile's rows
+  using Raw = typename std::conditional<sizeof(TIn) == 2, uint4, float4>::type;
+  constexpr int NRAW = sizeof(TIn) == 2 ? 4 : 8;
+  Raw raw[NRAW];
+  auto fetch = [&](int64_t t) {
+    const int64_t rw = t * kRows + r;
+    if (t < ntiles && rw < n) {
+      const TIn* xr = x + rw * ld;
 #pragma unroll
-        for (int c = 0; c < D / 8; ++c) {
-          const uint4 q = __ldg(reinterpret_cast<const uint4*>(xr) + c);
-          const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            const int i = 8 * c + 2 * h;
-            float lo, hi;
-            if constexpr (std::is_same<TIn, __nv_bfloat16>::value) {
-              lo = __uint_as_float((w4[h] << 16) ^ s_dmask[i]);
-              hi = __uint_as_float((w4[h] & 0xFFFF0000u) ^ s_dmask[i + 1]);
-            } else {
-              const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w4[h]));
-              lo = __uint_as_float(__float_as_uint(f.x) ^ s_dmask[i]);
-              hi = __uint_as_float(__float_as_uint(f.y) ^ s_dmask[i + 1]);
-            }
-            v[i] = lo;
-            v[i + 1] = hi;
-          }
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < D / 4; ++c) {
-          const float4 q = __ldg(reinterpret_cast<const float4*>(xr) + c);
-          v[4 * c + 0] = __uint_as_float(__float_as_uint(q.x) ^ s_dmask[4 * c + 0]);
-          v[4 * c + 1] = __uint_as_float(__float_as_uint(q.y) ^ s_dmask[4 * c + 1]);
-          v[4 * c + 2] = __uint_as_float(__float_as_uint(q.z) ^ s_dmask[4 * c + 2]);
-          v[4 * c + 3] = __uint_as_float(__float_as_uint(q.w) ^ s_dmask[4 * c + 3]);
+      for (int k = 0; k < 4; ++k) {
+        const int c = q + TPR * k;
+        if constexpr (sizeof(TIn) == 2) {
+          raw[k] = __ldg(reinterpret_cast<const uint4*>(xr + 8 * c));
+        } else {
+          raw[2 * k] = __ldg(reinterpret_cast<const float4*>(xr + 8 * c));
+          raw[2 * k + 1] = __ldg(reinterpret_cast<const float4*>(xr + 8 * c + 4));
         }
       }
     } else {
 #pragma unroll
-      for (int i = 0; i < D; ++i) v[i] = 0.f;
+      for (int k = 0; k < NRAW; ++k) raw[k] = Raw{0, 0, 0, 0};
     }
-    // ---------------------------------------------------------- norm
-    float acc8[8];
+  };
+  fetch(blockIdx.x);
+
+  for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    const int64_t row0 = tile * kRows;
+    const int64_t row = row0 + r;
+    const bool valid = row < n;
+    // ---------------------------------------------------------------- load
+    float v[32];
+    {
+      Raw cur[NRAW];
 #pragma unroll
-    for (int a = 0; a < 8; ++a) acc8[a] = 0.f;
+      for (int k = 0; k < NRAW; ++k) cur[k] = raw[k];
+      fetch(tile + gridDim.x);
 #pragma unroll
-    for (int i = 0; i < D; ++i) acc8[i & 7] = fmaf(v[i], v[i], acc8[i & 7]);
-    const float ss = ((acc8[0] + acc8[1]) + (acc8[2] + acc8[3])) + ((acc8[4] + acc8[5]) + (acc8[6] + acc8[7]));
-    bool flag = !(ss >= 1e-30f && ss <= 1e30f);
+      for (int k = 0; k < 4; ++k) {
+        const int c = q + TPR * k;
+        const uint4 dm0 = *reinterpret_cast<const uint4*>(s_dmask + 8 * c);
+        const uint4 dm1 = *reinterpret_cast<const uint4*>(s_dmask + 8 * c + 4);
+        const uint32_t dm[8] = {dm0.x, dm0.y, dm0.z, dm0.w, dm1.x, dm1.y, dm1.z, dm1.w};
+        if constexpr (sizeof(TIn) == 2) {
+          const uint4 qd = *reinterpret_cast<const uint4*>(&cur[k]);
+          const uint32_t w4[4] = {qd.x, qd.y, qd.z, qd.w};
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            v[8 * k + 2 * h] = __uint_as_float((w4[h] << 16) ^ dm[2 * h]);
+            v[8 * k + 2 * h + 1] = __uint_as_float((w4[h] & 0xFFFF0000u) ^ dm[2 * h + 1]);
+          }
+        } else {
+          const float4 a = *reinterpret_cast<const float4*>(&cur[2 * k]);
+          const float4 b = *reinterpret_cast<const float4*>(&cur[2 * k + 1]);
+          const float f[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v[8 * k + e] = __uint_as_float(__float_as_uint(f[e]) ^ dm[e]);
+        }
+      }
+    }
+    // ---------------------------------------------------------------- norm
+    float a4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int i = 0; i < 32; ++i) a4[i & 3] = fmaf(v[i], v[i], a4[i & 3]);
+    float ss = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+    ss += __shfl_xor_sync(TQ_FULL_MASK, ss, 1);
+    if constexpr (TPR == 4) ss += __shfl_xor_sync(TQ_FULL_MASK, ss, 2);
+    bool codeflag = !(ss >= 1e-30f && ss <= 1e30f);
     const float nu = sqrtf(ss);
-    // ---------------------------------------------------------- FWHT (in registers)
+    // ---------------------------------------------------------------- FWHT
 #pragma unroll
-    for (int h = 1; h < D; h <<= 1) {
+    for (int h = 1; h < 32; h <<= 1) {
 #pragma unroll
-      for (int i = 0; i < D; ++i) {
+      for (int i = 0; i < 32; ++i) {
         if ((i & h) == 0) {
           const float a = v[i], b = v[i + h];
           v[i] = a + b;
@@ -296,99 +357,123 @@ __global__ void __launch_bounds__(kTile, 2)
         }
       }
     }
-    // ---------------------------------------------------------- codes, residual
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = fmaf(sgn1, v[i], __shfl_xor_sync(TQ_FULL_MASK, v[i], 1));
+    if constexpr (TPR == 4) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = fmaf(sgn2, v[i], __shfl_xor_sync(TQ_FULL_MASK, v[i], 2));
+    }
+    // ---------------------------------------------------------------- codes
     float mt0[H0], mt1[H1];
     mt0[0] = mt1[0] = 0.f;
 #pragma unroll
     for (int k = 1; k < H0; ++k) mt0[k] = nu * qb.bnd[0][H0 + k - 1];
 #pragma unroll
-    for (int k = 1; k < H1; ++k) mt1[k] = B1 > 0 ? nu * qb.bnd[1][H1 + k - 1] : 0.f;
+    for (int k = 1; k < H1; ++k) mt1[k] = nu * qb.bnd[1][H1 + k - 1];
     const float A = 1.1f * kU * (float)L * sqrtD * nu;
-    float runmin = INFINITY;
-    float g2 = 0.f;
-    uint32_t cw[W];
+    int frexp_e;
+    frexpf(nu > 0.f ? nu : 1.f, &frexp_e);
+    frexp_e = max(-125, min(125, frexp_e));
+    const float rscale = ldexpf(1.f, -frexp_e);
+    float runmin = INFINITY, g2 = 0.f, cv2 = 0.f;
+    unsigned char* crow = reinterpret_cast<unsigned char*>(st_codes + r * W);
 #pragma unroll
-    for (int k = 0; k < W; ++k) cw[k] = 0u;
-    // fp16 scale of the residual: 2^-e with nu in [2^(e-1), 2^e)
-    int e2;
-    frexpf(nu > 0.f ? nu : 1.f, &e2);
-    e2 = max(-125, min(125, e2));
-    const float rscale = ldexpf(1.f, -e2);
+    for (int k = 0; k < 4; ++k) {
+      const int c = q + TPR * k;
+      const bool seg1 = NSEG == 2 && c >= CHSEG;
+      const int cs = seg1 ? c - CHSEG : c;
+      uint32_t pb[4] = {0u, 0u, 0u, 0u};
+      float rr[8];
 #pragma unroll
-    for (int c0 = 0; c0 < D; c0 += 16) {
-      uint32_t hi8[8], lo8[8];
-#pragma unroll
-      for (int ii = 0; ii < 16; ii += 2) {
-        float r2[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int i = c0 + ii + e;
-          const bool seg1 = NSEG == 2 && i >= SEGLEN;
-          const float w = v[i];
-          const float a = fabsf(w);
-          const bool pos = w >= 0.f;
-          int mcell;
-          float margin;
-          if (seg1) {
-            mag_search<(B1 > 0 ? B1 : 1)>(a, mt1, mcell, margin);
-          } else {
-            mag_search<B0>(a, mt0, mcell, margin);
-          }
-          const float cv = nu * (seg1 ? qb.cen[1][H1 + mcell] : qb.cen[0][H0 + mcell]);
-          runmin = fminf(runmin, fmaf(-Bc, a, margin));
-          const int bits = seg1 ? B1 : B0;
-          const int il = seg1 ? i - SEGLEN : i;
-          const int wbase = (seg1 ? B0 * PW : 0) + il / 32;
-          const uint32_t bit = 1u << (il & 31);
-          // plane bits: top plane = sign, lower planes = magnitude bits xor !sign
-#pragma unroll
-          for (int pl = 0; pl < 4; ++pl) {
-            if (pl < bits) {
-              bool b;
-              if (pl == bits - 1)
-                b = pos;
-              else
-                b = (((mcell >> pl) & 1) != 0) != !pos;
-              if (b) cw[wbase + pl * PW] |= bit;
-            }
-          }
-          const float r = w - copysignf(cv, w);
-          g2 = fmaf(r, r, g2);
-          r2[e] = r * rscale;
+      for (int e = 0; e < 8; ++e) {
+        const float w = v[8 * k + e];
+        const float a = fabsf(w);
+        const bool pos = w >= 0.f;
+        int mc;
+        float margin;
+        if (seg1) {
+          mag_search<(B1 > 0 ? B1 : 1)>(a, mt1, mc, margin);
+        } else {
+          mag_search<B0>(a, mt0, mc, margin);
         }
-        const uint32_t h = pack_half2(r2[0], r2[1]);
-        const float2 hf = unpack_half2(h);
-        hi8[ii / 2] = h;
-        lo8[ii / 2] = pack_half2(r2[0] - hf.x, r2[1] - hf.y);
+        runmin = fminf(runmin, fmaf(-Bc, a, margin));
+        const int bits = seg1 ? B1 : B0;
+#pragma unroll
+        for (int pl = 0; pl < 4; ++pl) {
+          if (pl < bits) {
+            const bool b = (pl == bits - 1) ? pos : ((((mc >> pl) & 1) != 0) != !pos);
+            pb[pl] |= (b ? 1u : 0u) << e;
+          }
+        }
+        if constexpr (SK) {
+          const float cvv = nu * (seg1 ? qb.cen[1][H1 + mc] : qb.cen[0][H0 + mc]);
+          const float rv = w - copysignf(cvv, w);
+          g2 = fmaf(rv, rv, g2);
+          cv2 = fmaf(cvv, cvv, cv2);
+          rr[e] = rv * rscale;
+        }
       }
-      if (sketch) {
-        tqtc::tmem_st8(tqtc::tmem_addr(tbase, lane_base, c0 / 2), hi8);
-        tqtc::tmem_st8(tqtc::tmem_addr(tbase, lane_base, col_lo + c0 / 2), lo8);
+      const int bits = seg1 ? B1 : B0;
+      const int wbase = seg1 ? B0 * PW : 0;
+#pragma unroll
+      for (int pl = 0; pl < 4; ++pl)
+        if (pl < bits) crow[(wbase + pl * PW) * 4 + cs] = (unsigned char)pb[pl];
+      if constexpr (SK) {
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int e = 0; e < 8; e += 2) {
+          const uint32_t h = pack_half2(rr[e], rr[e + 1]);
+          const float2 hf = unpack_half2(h);
+          hi[e / 2] = h;
+          lo[e / 2] = pack_half2(rr[e] - hf.x, rr[e + 1] - hf.y);
+        }
+        const uint32_t off = (uint32_t)c * LBO_A + (uint32_t)(r / 8) * 128 + (uint32_t)(r % 8) * 16;
+        *reinterpret_cast<uint4*>(smem + ly.a_hi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(smem + ly.a_lo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
       }
     }
-    flag |= runmin <= A;
-    // ---------------------------------------------------------- sketch
-    uint32_t sw[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) sw[k] = 0u;
-    if (sketch) {
-      tqtc::tmem_wait_st();
+    codeflag |= runmin <= A;
+    if (codeflag && valid) atomicOr(&st_flag[r], 2);
+    if constexpr (SK) {
+      g2 += __shfl_xor_sync(TQ_FULL_MASK, g2, 1);
+      cv2 += __shfl_xor_sync(TQ_FULL_MASK, cv2, 1);
+      if constexpr (TPR == 4) {
+        g2 += __shfl_xor_sync(TQ_FULL_MASK, g2, 2);
+        cv2 += __shfl_xor_sync(TQ_FULL_MASK, cv2, 2);
+      }
+    }
+    if (q == 0) {
+      st_nu[r] = nu;
+      if constexpr (SK) {
+        st_gam[r] = sqrtf(g2) / (nu * sqrtD);
+        const float R2 = rscale * sqrtf(g2) * 1.00001f;
+        const float E = 1.1f * (rscale * 1.1f * (kU * (float)L * sqrtD * nu + (e_nu + kU) * sqrtf(cv2) +
+                                                 kU * sqrtf(g2)) +
+                                2.4e-7f * R2 + 3.0e-8f * sqrtD) +
+                        1.1f * 4.3e-6f * R2;
+        st_err[r] = make_float2(E, 1.1f * 3.0e-8f * sqrtD * R2);
+      }
+    }
+    // ---------------------------------------------------------------- sketch
+    if constexpr (SK) {
+      tqtc::fence_proxy_async_smem();
       tqtc::tc_fence_before();
       __syncthreads();
       if (tid == 0) {
         tqtc::tc_fence_after();
-        const uint32_t idesc = tqtc::instr_desc(1, 0, 0, kTile, (uint32_t)m);
-        const uint32_t lbo = 16u * (uint32_t)m, sbo = 128u;
-        const uint32_t bhi = tqtc::smem_u32(s_bimg), blo = bhi + 2u * (uint32_t)m * D;
-        const uint32_t dcol = tbase + col_d;
+        const uint32_t idesc = tqtc::instr_desc(1, 0, 0, kRows, (uint32_t)m);
+        const uint32_t lbo_b = 16u * (uint32_t)m;
+        const uint32_t ahi = tqtc::smem_u32(smem + ly.a_hi), alo = tqtc::smem_u32(smem + ly.a_lo);
+        const uint32_t bhi = tqtc::smem_u32(smem + ly.bimg), blo = bhi + 2u * (uint32_t)m * D;
         bool accum = false;
 #pragma unroll
         for (int pass = 0; pass < 3; ++pass) {
-          const uint32_t acol = pass == 1 ? col_lo : 0u;
+          const uint32_t aa = pass == 1 ? alo : ahi;
           const uint32_t bb = pass == 2 ? blo : bhi;
 #pragma unroll
           for (int s = 0; s < D / 16; ++s) {
-            tqtc::mma_f16_ts(dcol, tbase + acol + 8u * s, tqtc::smem_desc(bb + 2u * s * lbo, lbo, sbo), idesc, accum);
+            tqtc::mma_f16_ss(tbase, tqtc::smem_desc(aa + 2u * s * LBO_A, LBO_A, 128),
+                             tqtc::smem_desc(bb + 2u * s * lbo_b, lbo_b, 128), idesc, accum);
             accum = true;
           }
         }
@@ -401,82 +486,69 @@ __global__ void __launch_bounds__(kTile, 2)
         s_abort = 1;
       }
       tqtc::tc_fence_after();
-      // bound of the residual error per coordinate, in scaled units
-      const float Er = rscale * 1.1f * (kU * (float)L * sqrtD * nu + (e_nu + kU) * nu * cmax +
-                                        kU * (sqrtD + cmax) * nu) +
-                       4.8e-7f * (sqrtD + cmax) + 2.98e-8f;
-      const float R2 = rscale * sqrtf(g2) * 1.00001f;
-      const float beta = 1.1f * (4.3e-6f * R2);
-      const float gam0 = 1.1f * 2.98e-8f * sqrtD * R2;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        if (c >= m / 32) break;
+      // epilogue: warp (lane quarter lq, word c) -> sign word c of rows 32 lq + lane
+      const int lq = warp & 3;
+      const int rr = 32 * lq + lane;
+      const float2 eg = st_err[rr];
+      for (int c = warp >> 2; c < m / 32; c += NW / 4) {
         uint32_t t16[2][16];
-        tqtc::tmem_ld16(tqtc::tmem_addr(tbase, lane_base, col_d + 32 * c), t16[0]);
-        tqtc::tmem_ld16(tqtc::tmem_addr(tbase, lane_base, col_d + 32 * c + 16), t16[1]);
+        tqtc::tmem_ld16(tqtc::tmem_addr(tbase, 32u * lq, 32u * c), t16[0]);
+        tqtc::tmem_ld16(tqtc::tmem_addr(tbase, 32u * lq, 32u * c + 16u), t16[1]);
         tqtc::tmem_wait_ld();
-        uint32_t word = 0;
+        uint32_t word = 0, unsure = 0;
 #pragma unroll
         for (int jj = 0; jj < 32; ++jj) {
           const float t = __uint_as_float(t16[jj >> 4][jj & 15]);
-          const int j = 32 * c + jj;
-          const float tau = 1.1f * s_sl1[j] * Er + beta * s_sl2[j] + gam0;
-          flag |= !(fabsf(t) > tau);
+          const float tau = fmaf(__ldg(p.sl2n + 32 * c + jj), eg.x, eg.y);
+          unsure |= (fabsf(t) > tau ? 0u : 1u) << jj;
           word |= (t >= 0.f ? 1u : 0u) << jj;
         }
-        sw[c] = word;
-      }
-    }
-    // ---------------------------------------------------------- store / defer
-    if (valid) {
-      if (!flag) {
-        uint32_t* orow = out.codes + row * W;
-        if constexpr (W % 4 == 0) {
-#pragma unroll
-          for (int k = 0; k < W; k += 4) *reinterpret_cast<uint4*>(orow + k) = make_uint4(cw[k], cw[k + 1], cw[k + 2], cw[k + 3]);
-        } else if constexpr (W % 2 == 0) {
-#pragma unroll
-          for (int k = 0; k < W; k += 2) *reinterpret_cast<uint2*>(orow + k) = make_uint2(cw[k], cw[k + 1]);
-        } else {
-#pragma unroll
-          for (int k = 0; k < W; ++k) orow[k] = cw[k];
-        }
-        out.norms[row] = nu;
-        if (sketch) {
-          const int MS = m / 32;
-          uint32_t* srow = out.signs + row * MS;
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
-            if (k < MS) srow[k] = sw[k];
-          out.rnorms[row] = sqrtf(g2) / (nu * sqrtD);
-        }
-      } else {
-        s_list[atomicAdd(&s_count, 1)] = tid;
+        st_signs[rr * 8 + c] = word;
+        st_fmask[rr * 8 + c] = unsure;
+        if (unsure && row0 + rr < n) atomicOr(&st_flag[rr], 1);
       }
     }
     tqtc::tc_fence_before();
     __syncthreads();
     if (s_abort) break;
-    // ---------------------------------------------------------- fp64 re-evaluation
-    const int cnt = s_count;
-    if (tid == 0 && cnt > 0) atomicAdd(p.exact_rows, (unsigned long long)cnt);
-    for (int e = warp; e < cnt; e += kTile / 32) {
-      const int64_t r = tile * kTile + s_list[e];
-      exact_row_fp64<D, TIn>(p, qb, x + r * ld, r, out, s_scr);
+    // ---------------------------------------------------------------- write out (fast path)
+    const int nrow = (int)((n - row0) < (int64_t)kRows ? (n - row0) : (int64_t)kRows);
+    {
+      uint32_t* gcodes = out.codes + row0 * W;
+      if constexpr (W % 4 == 0) {
+        for (int i = tid; i < nrow * W / 4; i += NT)
+          reinterpret_cast<uint4*>(gcodes)[i] = reinterpret_cast<const uint4*>(st_codes)[i];
+      } else {
+        for (int i = tid; i < nrow * W; i += NT) gcodes[i] = st_codes[i];
+      }
+      for (int i = tid; i < nrow; i += NT) out.norms[row0 + i] = st_nu[i];
+      if constexpr (SK) {
+        const int MS = m / 32;
+        for (int i = tid; i < nrow * MS; i += NT) out.signs[row0 * MS + i] = st_signs[(i / MS) * 8 + (i % MS)];
+        for (int i = tid; i < nrow; i += NT) out.rnorms[row0 + i] = st_gam[i];
+      }
+    }
+    // ---------------------------------------------------------------- queue uncertain rows
+    if (tid < kRows && st_flag[tid] != 0) {
+      const int e = atomicAdd(&s_nfix, 1);
+      FixEntry& f = s_fix[e];
+      f.row = row0 + tid;
+      f.full = (st_flag[tid] & 2) != 0;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) f.fmask[w] = st_fmask[tid * 8 + w];
     }
     __syncthreads();
-    if (tid == 0) s_count = 0;
+    if (s_nfix > kFixCap - kRows) drain();
+    for (int i = tid; i < kRows; i += NT) st_flag[i] = 0;
     __syncthreads();
     tqtc::tc_fence_after();
   }
   tqtc::tc_fence_before();
   __syncthreads();
-  if (sketch && warp == 0) tqtc::tmem_dealloc(tbase, tmem_cols);
-}
-
-template <typename Fn>
-cudaError_t set_smem_attr(Fn* fn, size_t bytes) {
-  return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (!s_abort) drain();
+  if constexpr (SK) {
+    if (warp == 0) tqtc::tmem_dealloc(tbase, tmem_cols);
+  }
 }
 
 int g_sms = 0;
@@ -490,22 +562,36 @@ int sm_count() {
   return g_sms;
 }
 
-template <int D, int B0, int B1, typename TIn>
-cudaError_t launch_tc(const tq_params& p, const void* x, int64_t n, int64_t ld, const tq_compressed& out,
-                      cudaStream_t st) {
-  const int m = p.m;
-  const size_t smem = (size_t)4 * m * D + (size_t)8 * m + (size_t)4 * D * sizeof(double);
-  auto fn = tq_quantize_tc_kernel<D, B0, B1, TIn>;
-  cudaError_t e = set_smem_attr(fn, smem);
+template <int D, int B0, int B1, bool SK, typename TIn>
+cudaError_t launch_quad(const tq_params& p, const void* x, int64_t n, int64_t ld, const tq_compressed& out,
+                        cudaStream_t st) {
+  constexpr int TPR = D / 32;
+  constexpr int NT = kRows * TPR;
+  constexpr int PW = (D / (B1 > 0 ? 2 : 1)) / 32;
+  constexpr int W = (B0 + B1) * PW;
+  const int m = SK ? p.m : 0;
+  const QLayout ly(D, m, W, NT / 32);
+  auto fn = tq_quantize_quad_kernel<D, B0, B1, SK, TIn>;
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ly.total);
   if (e != cudaSuccess) return e;
   uint32_t cols = 32;
-  while (cols < (uint32_t)(D + m)) cols <<= 1;
-  const int64_t ntiles = (n + kTile - 1) / kTile;
-  // at most two resident blocks per SM (TMEM: 2 x cols <= 512)
-  const int per_sm = (m > 0 && cols > 256) ? 1 : 2;
+  while (cols < (uint32_t)m) cols <<= 1;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, NT, ly.total);
+  if (e != cudaSuccess) return e;
+  if (SK) per_sm = std::min(per_sm, (int)(512 / cols));
+  per_sm = std::max(per_sm, 1);
+  const int64_t ntiles = (n + kRows - 1) / kRows;
   const int grid = (int)std::min<int64_t>(ntiles, (int64_t)sm_count() * per_sm);
-  fn<<<grid, kTile, smem, st>>>(p, (const TIn*)x, n, ld, out, ntiles, cols);
+  fn<<<grid, NT, ly.total, st>>>(p, (const TIn*)x, n, ld, out, ntiles, cols);
   return cudaGetLastError();
+}
+
+template <int D, int B0, int B1, typename TIn>
+cudaError_t launch_sk(const tq_params& p, const void* x, int64_t n, int64_t ld, const tq_compressed& out,
+                      cudaStream_t st) {
+  return p.m > 0 ? launch_quad<D, B0, B1, true, TIn>(p, x, n, ld, out, st)
+                 : launch_quad<D, B0, B1, false, TIn>(p, x, n, ld, out, st);
 }
 
 template <int D, typename TIn>
@@ -513,13 +599,13 @@ cudaError_t dispatch_bits(const tq_params& p, const void* x, int64_t n, int64_t 
                           cudaStream_t st) {
   if (p.nseg == 1) {
     switch (p.bits[0]) {
-      case 1: return launch_tc<D, 1, 0, TIn>(p, x, n, ld, out, st);
-      case 2: return launch_tc<D, 2, 0, TIn>(p, x, n, ld, out, st);
-      case 3: return launch_tc<D, 3, 0, TIn>(p, x, n, ld, out, st);
-      case 4: return launch_tc<D, 4, 0, TIn>(p, x, n, ld, out, st);
+      case 1: return launch_sk<D, 1, 0, TIn>(p, x, n, ld, out, st);
+      case 2: return launch_sk<D, 2, 0, TIn>(p, x, n, ld, out, st);
+      case 3: return launch_sk<D, 3, 0, TIn>(p, x, n, ld, out, st);
+      case 4: return launch_sk<D, 4, 0, TIn>(p, x, n, ld, out, st);
     }
   } else if (p.bits[0] == 2 && p.bits[1] == 3) {
-    return launch_tc<D, 2, 3, TIn>(p, x, n, ld, out, st);
+    return launch_sk<D, 2, 3, TIn>(p, x, n, ld, out, st);
   }
   return cudaErrorNotSupported;
 }
