@@ -172,7 +172,7 @@ class Layer:
         self.V = tq.Compressed.empty(self.vc, n, dev)
         self.logits = torch.empty((w.B, w.Hq, w.T), device=dev)
         self.out = torch.empty((w.B, w.Hq, d), device=dev)
-        self.ws_s = tq.workspace(tq.tq_scores_workspace_size(self.kc, w.B, w.Hq), dev)
+        self.ws_s = tq.workspace(tq.tq_scores_workspace_size(self.kc, w.B, w.Hq, w.Hkv), dev)
         self.ws_a = tq.workspace(tq.tq_attend_workspace_size(self.kc, self.vc, w.B, w.Hq, w.Hkv, w.T), dev)
 
     def stages(self, k=None, v=None, q=None):

@@ -164,16 +164,17 @@ TQ_API tq_status tq_quantize(const tq_codec *codec, const void *x, tq_dtype dtyp
                       int64_t n, int64_t ld, const tq_compressed *out,
                       void *stream);
 
-/* Workspace bytes for tq_scores with B batches of Hq query heads.           */
+/* Workspace bytes for tq_scores with B batches of Hq query heads over Hkv KV
+ * heads (the query side is prepared per (batch, KV head) group).            */
 TQ_API tq_status tq_scores_workspace_size(const tq_codec *kc, int B, int Hq,
-                                   size_t *bytes);
+                                          int Hkv, size_t *bytes);
 
 /* Attention logits over compressed keys (unscaled estimator above).
  *   q       [B][Hq][d] of `dtype`, contiguous
  *   K       compressed keys, B*Hkv*T rows; key (b, h_kv, t) is row
  *           (b*Hkv + h_kv)*T + t
  *   logits  [B][Hq][T] fp32 out; query head h uses KV head h / (Hq / Hkv)
- *   workspace, ws_bytes  >= tq_scores_workspace_size(kc, B, Hq)
+ *   workspace, ws_bytes  >= tq_scores_workspace_size(kc, B, Hq, Hkv)
  * Hq must be a multiple of Hkv, Hq / Hkv <= 32.  T = 0 is a no-op.          */
 TQ_API tq_status tq_scores(const tq_codec *kc, const void *q, tq_dtype dtype, int B,
                     int Hq, int Hkv, int64_t T, const tq_compressed *K,
@@ -187,8 +188,8 @@ TQ_API tq_status tq_scores(const tq_codec *kc, const void *q, tq_dtype dtype, in
  * arguments and result as tq_scores, minus the workspace: the scratch is a
  * 2 MiB array inside libtq (held on every GPU that loads the library until
  * the process exits).
- *   - Calls needing more scratch than that (tq_scores_workspace_size(kc, B, Hq)
- *     above 2 MiB) return TQ_ERR_UNSUPPORTED and write nothing.
+ *   - Calls needing more scratch than that (tq_scores_workspace_size(kc, B, Hq,
+ *     Hkv) above 2 MiB) return TQ_ERR_UNSUPPORTED and write nothing.
  *   - The first call on a device looks up the array's device address; make it
  *     before any stream capture.
  *   - Every call shares the one array: calls whose kernels may overlap on the

@@ -53,7 +53,7 @@ def _load() -> ctypes.CDLL:
         "tq_codec_export": [P, P, P, P, P],
         "tq_codec_layout": [P, ctypes.POINTER(I), ctypes.POINTER(I)],
         "tq_quantize": [P, P, I, I64, I64, P, P],
-        "tq_scores_workspace_size": [P, I, I, ctypes.POINTER(SZ)],
+        "tq_scores_workspace_size": [P, I, I, I, ctypes.POINTER(SZ)],
         "tq_scores": [P, P, I, I, I, I, I64, P, P, P, SZ, P],
         "tq_scores_noalloc": [P, P, I, I, I, I, I64, P, P, P],
         "tq_attend_workspace_size": [P, P, I, I, I, I64, ctypes.POINTER(SZ)],
@@ -195,9 +195,9 @@ def tq_quantize(codec: Codec, x: torch.Tensor, out: Compressed, stream=None) -> 
     return out
 
 
-def tq_scores_workspace_size(kc: Codec, B: int, Hq: int) -> int:
+def tq_scores_workspace_size(kc: Codec, B: int, Hq: int, Hkv: int) -> int:
     v = ctypes.c_size_t()
-    _check(_lib.tq_scores_workspace_size(kc.handle, B, Hq, ctypes.byref(v)), "tq_scores_workspace_size")
+    _check(_lib.tq_scores_workspace_size(kc.handle, B, Hq, Hkv, ctypes.byref(v)), "tq_scores_workspace_size")
     return v.value
 
 

@@ -282,6 +282,32 @@ extern "C" tq_status tq_codec_create(const tq_spec* spec, int device, tq_codec**
     }
   }
   p.W = W;
+  // plane-identity coefficients: alpha_t = 2^-b sum_c cen[c] prod_{k in t} s_k(c)
+  p.plane_ok = 1;
+  for (int s = 0; s < spec->nseg; ++s) {
+    const int bits = spec->seg_bits[s], L = 1 << bits;
+    p.nterms[s] = tq_term_count[bits];
+    for (int t = 0; t < p.nterms[s]; ++t) {
+      double a = 0.0;
+      for (int code = 0; code < L; ++code) {
+        double prod = 1.0;
+        for (int k = 0; k < bits; ++k)
+          if ((tq_term_mask[bits][t] >> k) & 1) prod *= ((code >> k) & 1) ? 1.0 : -1.0;
+        a += (double)c->cen_host[s][code] * prod;
+      }
+      p.alpha[s][t] = (float)(a / L);
+    }
+    for (int code = 0; code < L; ++code) {
+      double rec = 0.0;
+      for (int t = 0; t < p.nterms[s]; ++t) {
+        double prod = 1.0;
+        for (int k = 0; k < bits; ++k)
+          if ((tq_term_mask[bits][t] >> k) & 1) prod *= ((code >> k) & 1) ? 1.0 : -1.0;
+        rec += (double)p.alpha[s][t] * prod;
+      }
+      if (std::fabs(rec - c->cen_host[s][code]) > 1e-6 * (1.0 + std::fabs(c->cen_host[s][code]))) p.plane_ok = 0;
+    }
+  }
   draw_signs(spec->seed, d, c->dbits_host);
   if (m > 0) draw_sketch(spec->seed, m, d, c->S_host);
 
@@ -472,10 +498,15 @@ extern "C" tq_status tq_quantize(const tq_codec* c, const void* x, tq_dtype dt, 
 
 static size_t qprep_bytes(const tq_params& p, int nq) { return align256(sizeof(float) * (size_t)nq * (p.d + p.m)); }
 
-extern "C" tq_status tq_scores_workspace_size(const tq_codec* kc, int B, int Hq, size_t* bytes) {
+static size_t scores_bytes(const tq_params& p, int B, int Hq, int Hkv) {
+  return qprep_bytes(p, B * Hq) + align256(tq_scores_tc_bytes(p, B, Hq, Hkv));
+}
+
+extern "C" tq_status tq_scores_workspace_size(const tq_codec* kc, int B, int Hq, int Hkv, size_t* bytes) {
   if (!kc || !bytes) return tq_fail(TQ_ERR_INVALID_ARG, "tq_scores_workspace_size: null argument");
-  if (B < 0 || Hq < 0) return tq_fail(TQ_ERR_INVALID_ARG, "tq_scores_workspace_size: negative size");
-  *bytes = qprep_bytes(kc->p, B * Hq);
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv)
+    return tq_fail(TQ_ERR_INVALID_ARG, "tq_scores_workspace_size: bad shape B=%d Hq=%d Hkv=%d", B, Hq, Hkv);
+  *bytes = scores_bytes(kc->p, B, Hq, Hkv);
   return TQ_OK;
 }
 
@@ -499,13 +530,17 @@ extern "C" tq_status tq_scores(const tq_codec* kc, const void* q, tq_dtype dt, i
   if (!q || !aligned16(q)) return tq_fail(TQ_ERR_INVALID_ARG, "tq_scores: q null or not 16-byte aligned");
   if (!logits || !aligned16(logits)) return tq_fail(TQ_ERR_INVALID_ARG, "tq_scores: logits null or not 16-byte aligned");
   if ((st = check_compressed(kc, K, "K")) != TQ_OK) return st;
-  const size_t need = qprep_bytes(kc->p, B * Hq);
+  const size_t need = scores_bytes(kc->p, B, Hq, Hkv);
   if (!workspace || !aligned16(workspace) || ws_bytes < need)
     return tq_fail(TQ_ERR_INVALID_ARG, "tq_scores: workspace null, misaligned or smaller than %zu bytes", need);
   const cudaStream_t s = (cudaStream_t)stream;
   float* qprep = (float*)workspace;
   cudaError_t e = tq_launch_qprep(kc->p, q, dt, B * Hq, qprep, s);
-  if (e == cudaSuccess) e = tq_launch_scores(kc->p, qprep, B, Hq, Hkv, T, *K, logits, s);
+  if (e == cudaSuccess) {
+    void* ws_tc = (char*)workspace + qprep_bytes(kc->p, B * Hq);
+    e = tq_launch_scores_tc(kc->p, qprep, B, Hq, Hkv, T, *K, logits, ws_tc, s);
+    if (e == cudaErrorNotSupported) e = tq_launch_scores(kc->p, qprep, B, Hq, Hkv, T, *K, logits, s);
+  }
   return launch_status(e, "tq_scores launch");
 }
 

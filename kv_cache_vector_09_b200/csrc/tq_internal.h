@@ -46,7 +46,19 @@ struct tq_params {
   const float* sl2n;      // [m] ||S_j||_2
   uint32_t* err;          // device error word (bounded waits that gave up), zero when healthy
   unsigned long long* exact_rows;  // rows re-evaluated in fp64 since the last reset
+  // plane identity of the symmetric codebooks: with s_k = 2 bit_k - 1,
+  //   cen[code] = sum_t alpha[seg][t] * prod_{k in term t} s_k,
+  // over the odd subsets of planes (term masks tq_term_mask[bits][t]); the
+  // product of an odd subset equals 2 * xor(bits) - 1.
+  int nterms[2];
+  float alpha[2][8];
+  int plane_ok;   // 1 if the identity reproduces every centroid (always, for
+                  // exactly symmetric codebooks)
 };
+
+// odd subsets of the bit planes, as bit masks, per bit width (1..4)
+static const int tq_term_mask[5][8] = {{0}, {1}, {1, 2}, {1, 2, 4, 7}, {1, 2, 4, 8, 7, 11, 13, 14}};
+static const int tq_term_count[5] = {0, 1, 2, 4, 8};
 
 struct tq_codec {
   tq_spec spec;
@@ -71,6 +83,11 @@ cudaError_t tq_launch_quantize(const tq_params& p, const void* x, tq_dtype dt, i
 // has no tensor-core variant (the caller then uses the generic kernel)
 cudaError_t tq_launch_quantize_tc(const tq_params& p, const void* x, tq_dtype dt, int64_t n, int64_t ld,
                                   const tq_compressed& out, cudaStream_t st);
+// tensor-core scorer: workspace bytes it needs after the query-prep block (0
+// if the configuration has no tensor-core variant), and the launch
+size_t tq_scores_tc_bytes(const tq_params& p, int B, int Hq, int Hkv);
+cudaError_t tq_launch_scores_tc(const tq_params& p, const float* qprep, int B, int Hq, int Hkv, int64_t T,
+                                const tq_compressed& K, float* logits, void* ws_tc, cudaStream_t st);
 cudaError_t tq_launch_qprep(const tq_params& p, const void* q, tq_dtype dt, int nq, float* qprep,
                             cudaStream_t st);
 cudaError_t tq_launch_scores(const tq_params& p, const float* qprep, int B, int Hq, int Hkv, int64_t T,

@@ -60,13 +60,13 @@ extern "C" tq_status tq_scores_noalloc(const tq_codec* kc, const void* q, tq_dty
   if (!kc) return tq_fail(TQ_ERR_INVALID_ARG, "tq_scores_noalloc: null codec");
   if (kc->device < 0) return tq_fail(TQ_ERR_INVALID_ARG, "tq_scores_noalloc: host-only codec");
   size_t need = 0;
-  tq_status st = tq_scores_workspace_size(kc, B, Hq, &need);
+  tq_status st = tq_scores_workspace_size(kc, B, Hq, Hkv, &need);
   if (st != TQ_OK) return st;
   if (need > TQ_SCORES_NOALLOC_SCRATCH)
     return tq_fail(TQ_ERR_UNSUPPORTED,
-                   "tq_scores_noalloc: B=%d, Hq=%d needs %zu bytes of scratch, above the built-in %u bytes; "
-                   "use tq_scores with a workspace",
-                   B, Hq, need, (unsigned)TQ_SCORES_NOALLOC_SCRATCH);
+                   "tq_scores_noalloc: B=%d, Hq=%d, Hkv=%d needs %zu bytes of scratch, above the built-in %u "
+                   "bytes; use tq_scores with a workspace",
+                   B, Hq, Hkv, need, (unsigned)TQ_SCORES_NOALLOC_SCRATCH);
   int cur = -1;
   const cudaError_t e = cudaGetDevice(&cur);
   if (e != cudaSuccess) return tq_fail(TQ_ERR_CUDA, "tq_scores_noalloc: cudaGetDevice: %s", cudaGetErrorString(e));

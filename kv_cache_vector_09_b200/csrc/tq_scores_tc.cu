@@ -1,0 +1,555 @@
+// Tensor-core scoring of compressed keys (kind::i8 tcgen05.mma).
+//
+// The estimator's two dot products per (key, query) are sums of query values
+// selected by key bits:
+//   <q', cen[code]> = sum_{segment s, odd plane subset t} alpha_st <q'_s, sigma_t>
+//   <w, sign>       = sum_j w_j sigma_j,       sigma = 2 bit - 1
+// (the plane identity: a symmetric codebook's centroid is an odd multilinear
+// function of the code's bit signs, and the product of an odd set of bit signs
+// is 2 * xor(bits) - 1).  With sigma = 2b - 1 both become
+//   sum_k b_k v_k - corr,   v_k = 2 alpha q'_i  (or 2 w_j),
+// a 0/1-by-real contraction over K = 32 * (source words) per key.
+//
+// A (keys, M = 128 per tile) goes to TMEM as u8 bytes: source word u (a plane
+// word, an xor of plane words, or a sign word) becomes eight 32-bit columns
+// word & (0x01010101 << r), r < 8, so K index k = 32u + 4r + j holds
+// 2^r * bit(r + 8j).  B (queries, N = 4 limbs x G queries, padded to 16)
+// holds round(v_k 2^(e - r)) split into four balanced base-256 s8 limbs, in
+// shared memory.  The s32 accumulation is exact; the epilogue rebuilds
+// I = sum_l 256^l D_l, scales by 2^-e and subtracts corr.
+#include <math.h>
+
+#include <algorithm>
+
+#include "tq_common.cuh"
+#include "tq_tc.cuh"
+
+namespace {
+
+constexpr int kKeys = 128;
+
+__host__ __device__ constexpr int term_mask(int bits, int t) {
+  return bits == 1 ? 1
+         : bits == 2 ? (t == 0 ? 1 : 2)
+         : bits == 3 ? (t < 3 ? (1 << t) : 7)
+                     : (t < 4 ? (1 << t) : (t == 4 ? 7 : t == 5 ? 11 : t == 6 ? 13 : 14));
+}
+
+__host__ __device__ inline int ncols_for(int G) { return ((4 * G + 15) / 16) * 16; }
+
+struct Geom {
+  int U_mse, U, Kt, N, G, lbo, bbytes, gstride;
+  __host__ __device__ Geom(const tq_params& p, int G_) {
+    U_mse = 0;
+    for (int s = 0; s < p.nseg; ++s) U_mse += p.nterms[s] * p.pw;
+    U = U_mse + p.MS;
+    Kt = 32 * U;
+    G = G_;
+    N = ncols_for(G_);
+    lbo = (N / 8) * 128;
+    bbytes = Kt * N;
+    gstride = ((bbytes + 16 * G_ + 127) / 128) * 128;  // B image + 4 floats per query
+  }
+};
+
+// ------------------------------------------------------------ B operand
+// One block per (batch, KV head) group.  qprep rows are [q' (d) | w (m)].
+__global__ void __launch_bounds__(256) tq_scores_bbuild_kernel(const tq_params p, const float* __restrict__ qprep,
+                                                               const int Hq, const int Hkv, uint8_t* __restrict__ ws) {
+  const Geom g(p, Hq / Hkv);
+  const int grp = blockIdx.x, b = grp / Hkv, hk = grp % Hkv;
+  const int d = p.d, m = p.m, L = p.seg_len;
+  __shared__ int s_xmse[32], s_xqjl[32];    // exponents e
+  uint8_t* out = ws + (size_t)grp * g.gstride;
+  float* consts = reinterpret_cast<float*>(out + g.bbytes);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int gq = warp; gq < g.G; gq += blockDim.x / 32) {
+    const float* qv = qprep + (size_t)(b * Hq + hk * g.G + gq) * (d + m);
+    float mx = 0.f, corr = 0.f;
+    for (int s = 0; s < p.nseg; ++s) {
+      float amax = 0.f, qmax = 0.f, qsum = 0.f;
+      for (int t = 0; t < p.nterms[s]; ++t) amax = fmaxf(amax, fabsf(p.alpha[s][t]));
+      float asum = 0.f;
+      for (int t = 0; t < p.nterms[s]; ++t) asum += p.alpha[s][t];
+      for (int i = lane; i < L; i += 32) {
+        const float v = qv[s * L + i];
+        qmax = fmaxf(qmax, fabsf(v));
+        qsum += v;
+      }
+      qmax = tq_warp_max(qmax);
+      qsum = tq_warp_sum(qsum);
+      mx = fmaxf(mx, 2.f * amax * qmax);
+      corr += asum * qsum;
+    }
+    float wmax = 0.f, wsum = 0.f;
+    for (int j = lane; j < m; j += 32) {
+      const float v = qv[d + j];
+      wmax = fmaxf(wmax, fabsf(v));
+      wsum += v;
+    }
+    wmax = tq_warp_max(wmax);
+    wsum = tq_warp_sum(wsum);
+    if (lane == 0) {
+      int ex;
+      frexpf(mx > 0.f ? mx : 1.f, &ex);
+      const int em = 30 - ex;  // |v| 2^em < 2^30
+      frexpf(wmax > 0.f ? 2.f * wmax : 1.f, &ex);
+      const int eq = 30 - ex;
+      s_xmse[gq] = em;
+      s_xqjl[gq] = eq;
+      consts[4 * gq + 0] = ldexpf(1.f, -em);
+      consts[4 * gq + 1] = corr;
+      consts[4 * gq + 2] = ldexpf(1.f, -eq);
+      consts[4 * gq + 3] = wsum;
+    }
+  }
+  __syncthreads();
+  const int u0 = p.nterms[0] * p.pw;
+  for (int idx = threadIdx.x; idx < g.Kt * g.N; idx += blockDim.x) {
+    const int n = idx / g.Kt, k = idx % g.Kt;
+    const int gq = n / 4, l = n % 4;
+    int8_t limb = 0;
+    if (gq < g.G) {
+      const float* qv = qprep + (size_t)(b * Hq + hk * g.G + gq) * (d + m);
+      const int u = k / 32, r = (k % 32) / 4, j = k % 4, bp = r + 8 * j;
+      float v;
+      int e;
+      if (u < g.U_mse) {
+        const int s = (p.nseg == 2 && u >= u0) ? 1 : 0;
+        const int uu = s ? u - u0 : u;
+        const int t = uu / p.pw, w = uu % p.pw;
+        v = 2.f * p.alpha[s][t] * qv[s * L + 32 * w + bp];
+        e = s_xmse[gq];
+      } else {
+        v = 2.f * qv[d + 32 * (u - g.U_mse) + bp];
+        e = s_xqjl[gq];
+      }
+      int x = __float2int_rn(ldexpf(v, e - r));
+      // balanced base-256 digits
+      int lv = 0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int dq = (int)(int8_t)(x & 0xFF);
+        if (q == l) lv = dq;
+        x = (x - dq) >> 8;
+      }
+      limb = (int8_t)lv;
+    }
+    const int off = (k / 16) * g.lbo + (n / 8) * 128 + (n % 8) * 16 + (k % 16);
+    out[off] = (uint8_t)limb;
+  }
+}
+
+// ------------------------------------------------------------ scoring
+// Warp-specialised, one block per SM, tiles of 128 keys of one (batch, KV
+// head) group; a block owns a contiguous range of tiles.
+//   warps 0-3  expansion: read a tile's codes/signs from the ring, build the u8
+//              planes in TMEM A[i % 2] (warp w owns lanes 32w..32w+31)
+//   warps 4-7  epilogue: read accumulator D[i % 2], rebuild the two sums, write
+//              the logits
+//   warp 8     producer: bulk copies of key tiles into a 4-stage ring and of
+//              each group's query operand into one of two buffers
+//   warp 9     MMA issue: U tcgen05.mma (kind::i8, A from TMEM) per tile
+// mbarriers: ring_full/ring_empty (producer <-> expansion), a_full (expansion
+// -> MMA), mma_done (MMA commit -> expansion for A reuse, epilogue for D),
+// d_empty (epilogue -> MMA), b_full/b_empty (producer <-> MMA, query operand).
+constexpr int kStages = 4;
+constexpr int kThreads = 320;
+
+__host__ __device__ inline int ring_stage_bytes(int W, int MS) { return kKeys * (W + MS) * 4; }
+
+template <int D, int B0, int B1, bool RING>
+__global__ void __launch_bounds__(kThreads, 1)
+    tq_scores_tc_kernel(const tq_params p, const tq_compressed K, float* __restrict__ logits,
+                        const uint8_t* __restrict__ ws, const int Hq, const int Hkv, const int64_t T,
+                        const int64_t tiles_per_group, const int64_t ntiles) {
+  constexpr int NSEG = B1 > 0 ? 2 : 1;
+  constexpr int PW = (D / NSEG) / 32;
+  constexpr int W = (B0 + B1) * PW;
+  constexpr int NT0 = B0 == 1 ? 1 : B0 == 2 ? 2 : B0 == 3 ? 4 : 8;
+  constexpr int NT1 = B1 == 0 ? 0 : B1 == 1 ? 1 : B1 == 2 ? 2 : B1 == 3 ? 4 : 8;
+  constexpr int U_MSE = (NT0 + NT1) * PW;
+
+  extern __shared__ __align__(1024) unsigned char smem[];
+  __shared__ uint64_t ring_full[kStages], ring_empty[kStages];
+  __shared__ uint64_t a_full[2], mma_done[2], d_empty[2], b_full[2], b_empty[2], drained;
+  __shared__ uint32_t s_tmem;
+  __shared__ volatile int s_abort;
+
+  const Geom g(p, Hq / Hkv);
+  const int MS = p.MS;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bstride = ((g.bbytes + 16 * g.G + 127) / 128) * 128;  // one query-operand buffer
+  unsigned char* bbuf = smem;                                     // [2][bstride]
+  unsigned char* ring = smem + 2 * bstride;                       // [kStages][ring_stage_bytes]
+  const int sbytes = ring_stage_bytes(W, MS);
+  const uint32_t acols = 8u * (uint32_t)g.U, dcols = 2u * (uint32_t)g.N;
+
+  const int64_t t_begin = (int64_t)blockIdx.x * ntiles / gridDim.x;
+  const int64_t t_end = (int64_t)(blockIdx.x + 1) * ntiles / gridDim.x;
+  const int64_t ntl = t_end - t_begin;
+
+  if (tid == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      tqtc::mbar_init(&ring_full[i], 1);
+      tqtc::mbar_init(&ring_empty[i], 128);
+    }
+    for (int i = 0; i < 2; ++i) {
+      tqtc::mbar_init(&a_full[i], 128);
+      tqtc::mbar_init(&mma_done[i], 1);
+      tqtc::mbar_init(&d_empty[i], 128);
+      tqtc::mbar_init(&b_full[i], 1);
+      tqtc::mbar_init(&b_empty[i], 1);
+    }
+    tqtc::mbar_init(&drained, 1);
+    tqtc::fence_mbar_init();
+    s_abort = 0;
+  }
+  if (warp == 0) tqtc::tmem_alloc(&s_tmem, 512);
+  tqtc::tc_fence_before();
+  __syncthreads();
+  tqtc::tc_fence_after();
+  const uint32_t tbase = s_tmem;
+  auto fail = [&](uint32_t code) {
+    atomicExch(p.err, code);
+    s_abort = 1;
+  };
+
+  if (warp == 8) {
+    // ---------------------------------------------------------- producer
+    if (lane == 0) {
+      int64_t cur = -1, issued = 0;
+      int gi = -1;
+      for (int64_t i = 0; i < ntl && !s_abort; ++i) {
+        const int64_t tile = t_begin + i;
+        const int64_t grp = tile / tiles_per_group;
+        if (grp != cur) {
+          cur = grp;
+          ++gi;
+          const int gb = gi & 1;
+          if (gi >= 2 && !tqtc::mbar_wait_or_abort(&b_empty[gb], (uint32_t)((gi / 2 - 1) & 1), &s_abort)) {
+            fail(tqtc::kErrCopyWait);
+            break;
+          }
+          tqtc::mbar_arrive_expect_tx(&b_full[gb], (uint32_t)bstride);
+          tqtc::bulk_g2s(bbuf + gb * bstride, ws + (size_t)grp * g.gstride, (uint32_t)bstride, &b_full[gb]);
+        }
+        if (RING) {
+          const int st = (int)(i % kStages);
+          if (i >= kStages &&
+              !tqtc::mbar_wait_or_abort(&ring_empty[st], (uint32_t)((i / kStages - 1) & 1), &s_abort)) {
+            fail(tqtc::kErrCopyWait);
+            break;
+          }
+          const int64_t t0 = (tile % tiles_per_group) * kKeys;
+          const int64_t rows = (T - t0) < kKeys ? (T - t0) : kKeys;
+          const int64_t row0 = grp * T + t0;
+          unsigned char* dst = ring + (size_t)st * sbytes;
+          const uint32_t bc = (uint32_t)(rows * W * 4), bs = (uint32_t)(rows * MS * 4);
+          tqtc::mbar_arrive_expect_tx(&ring_full[st], bc + bs);
+          tqtc::bulk_g2s(dst, K.codes + row0 * W, bc, &ring_full[st]);
+          if (MS > 0) tqtc::bulk_g2s(dst + kKeys * W * 4, K.signs + row0 * MS, bs, &ring_full[st]);
+          issued = i + 1;
+        }
+      }
+      // let every copy still in flight land before the block exits (bounded)
+      for (int64_t i = issued > kStages ? issued - kStages : 0; i < issued; ++i)
+        if (!tqtc::mbar_wait_or_abort(&ring_full[i % kStages], (uint32_t)((i / kStages) & 1), nullptr))
+          atomicExch(p.err, tqtc::kErrCopyWait);
+      for (int j = gi > 0 ? gi - 1 : 0; j <= gi; ++j)
+        if (!tqtc::mbar_wait_or_abort(&b_full[j & 1], (uint32_t)((j / 2) & 1), nullptr))
+          atomicExch(p.err, tqtc::kErrCopyWait);
+    }
+  } else if (warp == 9) {
+    // ---------------------------------------------------------- MMA issue
+    if (lane == 0) {
+      const uint32_t idesc = tqtc::instr_desc(2, 0, 1, kKeys, (uint32_t)g.N);
+      int64_t cur = -1;
+      int gi = -1;
+      for (int64_t i = 0; i < ntl && !s_abort; ++i) {
+        const int64_t tile = t_begin + i;
+        const int64_t grp = tile / tiles_per_group;
+        const int b = (int)(i & 1);
+        if (grp != cur) {
+          if (gi >= 0) tqtc::mma_commit(&b_empty[gi & 1]);  // previous group's operand is free once done
+          cur = grp;
+          ++gi;
+          if (!tqtc::mbar_wait_or_abort(&b_full[gi & 1], (uint32_t)((gi / 2) & 1), &s_abort)) {
+            fail(tqtc::kErrCopyWait);
+            break;
+          }
+        }
+        if (!tqtc::mbar_wait_or_abort(&a_full[b], (uint32_t)((i / 2) & 1), &s_abort)) {
+          fail(tqtc::kErrMmaWait);
+          break;
+        }
+        if (i >= 2 && !tqtc::mbar_wait_or_abort(&d_empty[b], (uint32_t)((i / 2 - 1) & 1), &s_abort)) {
+          fail(tqtc::kErrMmaWait);
+          break;
+        }
+        tqtc::tc_fence_after();
+        const uint32_t a0 = tbase + (uint32_t)b * acols;
+        const uint32_t d_mse = tbase + 2u * acols + (uint32_t)b * dcols, d_qjl = d_mse + (uint32_t)g.N;
+        uint64_t desc = tqtc::smem_desc(tqtc::smem_u32(bbuf + (gi & 1) * bstride), (uint32_t)g.lbo, 128);
+        const uint64_t step = (uint64_t)((2u * (uint32_t)g.lbo) >> 4);
+        for (int u = 0; u < g.U; ++u) {
+          const bool qjl = u >= g.U_mse;
+          tqtc::mma_i8_ts(qjl ? d_qjl : d_mse, a0 + 8u * (uint32_t)u, desc, idesc, !(u == 0 || u == g.U_mse));
+          desc += step;
+        }
+        tqtc::mma_commit(&mma_done[b]);
+      }
+      // every MMA issued has completed before TMEM is released (bounded)
+      tqtc::mma_commit(&drained);
+      if (!tqtc::mbar_wait_or_abort(&drained, 0, nullptr)) atomicExch(p.err, tqtc::kErrMmaWait);
+    }
+  } else if (warp < 4) {
+    // ---------------------------------------------------------- expansion
+    const uint32_t lane_base = 32u * (uint32_t)warp;
+    for (int64_t i = 0; i < ntl; ++i) {
+      const int64_t tile = t_begin + i;
+      const int64_t grp = tile / tiles_per_group;
+      const int64_t t0 = (tile % tiles_per_group) * kKeys;
+      const int b = (int)(i & 1);
+      const bool valid = t0 + tid < T;
+      uint32_t kcw[W], ksw[8];
+#pragma unroll
+      for (int k = 0; k < W; ++k) kcw[k] = 0u;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) ksw[k] = 0u;
+      if constexpr (RING) {
+        const int st = (int)(i % kStages);
+        if (!tqtc::mbar_wait_or_abort(&ring_full[st], (uint32_t)((i / kStages) & 1), &s_abort)) {
+          fail(tqtc::kErrCopyWait);
+          break;
+        }
+        if (valid) {
+          const unsigned char* src = ring + (size_t)st * sbytes;
+          const uint32_t* c32 = reinterpret_cast<const uint32_t*>(src) + tid * W;
+          if constexpr (W % 4 == 0) {
+#pragma unroll
+            for (int k = 0; k < W; k += 4) {
+              const uint4 q4 = *reinterpret_cast<const uint4*>(c32 + k);
+              kcw[k] = q4.x; kcw[k + 1] = q4.y; kcw[k + 2] = q4.z; kcw[k + 3] = q4.w;
+            }
+          } else if constexpr (W % 2 == 0) {
+#pragma unroll
+            for (int k = 0; k < W; k += 2) {
+              const uint2 q2 = *reinterpret_cast<const uint2*>(c32 + k);
+              kcw[k] = q2.x; kcw[k + 1] = q2.y;
+            }
+          } else {
+#pragma unroll
+            for (int k = 0; k < W; ++k) kcw[k] = c32[k];
+          }
+          const uint32_t* s32 = reinterpret_cast<const uint32_t*>(src + kKeys * W * 4) + tid * MS;
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            if (k < MS) ksw[k] = s32[k];
+        }
+        tqtc::mbar_arrive(&ring_empty[st]);
+      } else if (valid) {
+        const int64_t row = grp * T + t0 + tid;
+#pragma unroll
+        for (int k = 0; k < W; ++k) kcw[k] = __ldg(K.codes + row * W + k);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          if (k < MS) ksw[k] = __ldg(K.signs + row * MS + k);
+      }
+      // A[b] is free once the MMAs of tile i - 2 are done
+      if (i >= 2 && !tqtc::mbar_wait_or_abort(&mma_done[b], (uint32_t)((i / 2 - 1) & 1), &s_abort)) {
+        fail(tqtc::kErrMmaWait);
+        break;
+      }
+      tqtc::tc_fence_after();
+      const uint32_t a0 = (uint32_t)b * acols;
+      auto emit = [&](int u, uint32_t word) {
+        uint32_t regs[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) regs[r] = word & (0x01010101u << r);
+        tqtc::tmem_st8(tqtc::tmem_addr(tbase, lane_base, a0 + 8u * (uint32_t)u), regs);
+      };
+#pragma unroll
+      for (int s = 0; s < NSEG; ++s) {
+        const int bits = s ? B1 : B0;
+        const int base = s ? B0 * PW : 0;
+        const int nt = s ? NT1 : NT0;
+        const int ubase = s ? NT0 * PW : 0;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          if (t < nt) {
+            const int mask = term_mask(bits, t);
+#pragma unroll
+            for (int w = 0; w < PW; ++w) {
+              uint32_t word = 0u;
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                if ((mask >> k) & 1) word ^= kcw[base + k * PW + w];
+              emit(ubase + t * PW + w, word);
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (k < MS) emit(U_MSE + k, ksw[k]);
+      tqtc::tmem_wait_st();
+      tqtc::tc_fence_before();
+      tqtc::mbar_arrive(&a_full[b]);
+    }
+  } else {
+    // ---------------------------------------------------------- epilogue (warps 4-7)
+    const int et = tid - 128;
+    const uint32_t lane_base = 32u * (uint32_t)(warp - 4);
+    for (int64_t i = 0; i < ntl; ++i) {
+      const int64_t tile = t_begin + i;
+      const int64_t grp = tile / tiles_per_group;
+      const int64_t t0 = (tile % tiles_per_group) * kKeys;
+      const int b = (int)(i & 1);
+      const int64_t t = t0 + et;
+      const bool valid = t < T;
+      const int64_t row = grp * T + t;
+      const float knu = valid ? __ldg(K.norms + row) : 0.f;
+      const float kgam = (valid && MS > 0) ? __ldg(K.rnorms + row) : 0.f;
+      const float* cs_all = reinterpret_cast<const float*>(ws + (size_t)grp * g.gstride + g.bbytes);
+      if (!tqtc::mbar_wait_or_abort(&mma_done[b], (uint32_t)((i / 2) & 1), &s_abort)) {
+        fail(tqtc::kErrMmaWait);
+        break;
+      }
+      tqtc::tc_fence_after();
+      const uint32_t d_mse = 2u * acols + (uint32_t)b * dcols, d_qjl = d_mse + (uint32_t)g.N;
+      const int bq = (int)(grp / Hkv), hk = (int)(grp % Hkv);
+      const float cq = kgam * p.qjl_coef;
+      for (int qc = 0; qc < g.N / 16; ++qc) {
+        uint32_t dm[16], dq[16];
+        tqtc::tmem_ld16(tqtc::tmem_addr(tbase, lane_base, d_mse + 16u * qc), dm);
+        if (MS > 0) tqtc::tmem_ld16(tqtc::tmem_addr(tbase, lane_base, d_qjl + 16u * qc), dq);
+        tqtc::tmem_wait_ld();
+        if (qc == g.N / 16 - 1) {
+          tqtc::tc_fence_before();
+          tqtc::mbar_arrive(&d_empty[b]);
+        }
+#pragma unroll
+        for (int g4 = 0; g4 < 4; ++g4) {
+          const int gq = 4 * qc + g4;
+          if (gq < g.G && valid) {
+            const float4 cs = __ldg(reinterpret_cast<const float4*>(cs_all) + gq);
+            float im = (float)(int)dm[4 * g4 + 3];
+            im = fmaf(im, 256.f, (float)(int)dm[4 * g4 + 2]);
+            im = fmaf(im, 256.f, (float)(int)dm[4 * g4 + 1]);
+            im = fmaf(im, 256.f, (float)(int)dm[4 * g4 + 0]);
+            float val = fmaf(im, cs.x, -cs.y) * p.inv_sqrt_d;
+            if (MS > 0) {
+              float iq = (float)(int)dq[4 * g4 + 3];
+              iq = fmaf(iq, 256.f, (float)(int)dq[4 * g4 + 2]);
+              iq = fmaf(iq, 256.f, (float)(int)dq[4 * g4 + 1]);
+              iq = fmaf(iq, 256.f, (float)(int)dq[4 * g4 + 0]);
+              val = fmaf(cq, fmaf(iq, cs.z, -cs.w), val);
+            }
+            logits[((int64_t)bq * Hq + hk * g.G + gq) * T + t] = knu * val;
+          }
+        }
+      }
+    }
+  }
+  tqtc::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tqtc::tmem_dealloc(tbase, 512);
+}
+
+int g_sms = 0;
+int sm_count() {
+  if (!g_sms) {
+    int dev = 0, v = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+    g_sms = v;
+  }
+  return g_sms;
+}
+
+int smem_per_sm() {
+  static int v = 0;
+  if (!v) {
+    int dev = 0, x = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&x, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess || x <= 0)
+      x = 228 * 1024;
+    v = x;
+  }
+  return v;
+}
+
+bool supported(const tq_params& p, int G, uint32_t* cols_out) {
+  if (!p.plane_ok || (p.d != 64 && p.d != 128)) return false;
+  if (p.m > 256) return false;
+  if (!(p.nseg == 1 || (p.bits[0] == 2 && p.bits[1] == 3))) return false;
+  const Geom g(p, G);
+  if (g.bbytes > 64 * 1024 || g.N > 128) return false;
+  const uint32_t need = 2u * (8u * g.U + 2u * g.N);  // double-buffered A and accumulators
+  if (need > 512) return false;
+  if (cols_out) *cols_out = 512;
+  return true;
+}
+
+template <int D, int B0, int B1, bool RING>
+cudaError_t launch_scores_t(const tq_params& p, const tq_compressed& K, float* logits, const uint8_t* ws, int B,
+                            int Hq, int Hkv, int64_t T, cudaStream_t st) {
+  constexpr int W = (B0 + B1) * ((D / (B1 > 0 ? 2 : 1)) / 32);
+  const Geom g(p, Hq / Hkv);
+  const size_t bstride = (size_t)((g.bbytes + 16 * g.G + 127) / 128) * 128;
+  size_t smem = 2 * bstride + (RING ? (size_t)kStages * ring_stage_bytes(W, p.MS) : 0);
+  // the block takes all 512 TMEM columns: ask for more than half of the SM's
+  // shared memory so that a second block never waits on the allocation
+  smem = std::max(smem, (size_t)(smem_per_sm() / 2 + 1024));
+  auto fn = tq_scores_tc_kernel<D, B0, B1, RING>;
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int64_t tpg = (T + kKeys - 1) / kKeys;
+  const int64_t ntiles = (int64_t)B * Hkv * tpg;
+  const int grid = (int)std::min<int64_t>(ntiles, (int64_t)sm_count());
+  fn<<<grid, kThreads, smem, st>>>(p, K, logits, ws, Hq, Hkv, T, tpg, ntiles);
+  return cudaGetLastError();
+}
+
+template <int D, int B0, int B1>
+cudaError_t launch_scores(const tq_params& p, const tq_compressed& K, float* logits, const uint8_t* ws, int B,
+                          int Hq, int Hkv, int64_t T, uint32_t cols, cudaStream_t st) {
+  (void)cols;
+  // bulk copies need 16-byte aligned tile starts and sizes: T a multiple of 4
+  const bool ring = (T % 4) == 0 && (uintptr_t)K.codes % 16 == 0 && (p.MS == 0 || (uintptr_t)K.signs % 16 == 0);
+  return ring ? launch_scores_t<D, B0, B1, true>(p, K, logits, ws, B, Hq, Hkv, T, st)
+              : launch_scores_t<D, B0, B1, false>(p, K, logits, ws, B, Hq, Hkv, T, st);
+}
+
+}  // namespace
+
+size_t tq_scores_tc_bytes(const tq_params& p, int B, int Hq, int Hkv) {
+  if (Hkv <= 0 || Hq % Hkv) return 0;
+  if (!supported(p, Hq / Hkv, nullptr)) return 0;
+  const Geom g(p, Hq / Hkv);
+  return (size_t)B * Hkv * g.gstride;
+}
+
+cudaError_t tq_launch_scores_tc(const tq_params& p, const float* qprep, int B, int Hq, int Hkv, int64_t T,
+                                const tq_compressed& K, float* logits, void* ws_tc, cudaStream_t st) {
+  uint32_t cols = 0;
+  if (!supported(p, Hq / Hkv, &cols)) return cudaErrorNotSupported;
+  uint8_t* ws = reinterpret_cast<uint8_t*>(ws_tc);
+  tq_scores_bbuild_kernel<<<B * Hkv, 256, 0, st>>>(p, qprep, Hq, Hkv, ws);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  switch (p.d * 100 + p.bits[0] * 10 + (p.nseg == 2 ? p.bits[1] : 0)) {
+    case 12810: return launch_scores<128, 1, 0>(p, K, logits, ws, B, Hq, Hkv, T, cols, st);
+    case 12820: return launch_scores<128, 2, 0>(p, K, logits, ws, B, Hq, Hkv, T, cols, st);
+    case 12830: return launch_scores<128, 3, 0>(p, K, logits, ws, B, Hq, Hkv, T, cols, st);
+    case 12840: return launch_scores<128, 4, 0>(p, K, logits, ws, B, Hq, Hkv, T, cols, st);
+    case 12823: return launch_scores<128, 2, 3>(p, K, logits, ws, B, Hq, Hkv, T, cols, st);
+    case 6410: return launch_scores<64, 1, 0>(p, K, logits, ws, B, Hq, Hkv, T, cols, st);
+    case 6420: return launch_scores<64, 2, 0>(p, K, logits, ws, B, Hq, Hkv, T, cols, st);
+    case 6430: return launch_scores<64, 3, 0>(p, K, logits, ws, B, Hq, Hkv, T, cols, st);
+    case 6440: return launch_scores<64, 4, 0>(p, K, logits, ws, B, Hq, Hkv, T, cols, st);
+    case 6423: return launch_scores<64, 2, 3>(p, K, logits, ws, B, Hq, Hkv, T, cols, st);
+  }
+  return cudaErrorNotSupported;
+}

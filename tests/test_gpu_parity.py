@@ -162,7 +162,7 @@ def test_scores_match_oracle(case):
     # end to end: each side quantises and scores on its own
     K = gpu_quantize(kc, k.reshape(-1, d))
     qg = q.to(DEV).contiguous()
-    ws = tq.workspace(tq.tq_scores_workspace_size(kc, B, Hq), DEV)
+    ws = tq.workspace(tq.tq_scores_workspace_size(kc, B, Hq, Hkv), DEV)
     logits = torch.empty((B, Hq, T), device=DEV)
     tq.tq_scores(kc, qg, B, Hq, Hkv, T, K, logits, ws)
     torch.cuda.synchronize()
@@ -278,7 +278,7 @@ def test_full_size_sampled(wname):
         return
     q = synth.queries(w)
     qg = q.to(DEV).contiguous()
-    ws = tq.workspace(tq.tq_scores_workspace_size(kc, w.B, w.Hq), DEV)
+    ws = tq.workspace(tq.tq_scores_workspace_size(kc, w.B, w.Hq, w.Hkv), DEV)
     logits = torch.empty((w.B, w.Hq, w.T), device=DEV)
     tq.tq_scores(kc, qg, w.B, w.Hq, w.Hkv, w.T, K, logits, ws)
     torch.cuda.synchronize()

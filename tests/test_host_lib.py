@@ -77,7 +77,7 @@ def test_invalid_arguments_are_rejected_on_the_host():
     st = lib.tq_quantize(c.handle, None, 1, 1, 128, ctypes.byref(comp), None)
     assert st == 1 and "host-only" in tq.tq_last_error_string()
     v = ctypes.c_size_t()
-    assert lib.tq_scores_workspace_size(c.handle, 8, 32, ctypes.byref(v)) == 0 and v.value >= 8 * 32 * (128 + 64) * 4
+    assert lib.tq_scores_workspace_size(c.handle, 8, 32, 8, ctypes.byref(v)) == 0 and v.value >= 8 * 32 * (128 + 64) * 4
     assert lib.tq_codec_destroy(None) == 0
     c.close()
     c.close()

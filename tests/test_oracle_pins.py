@@ -433,3 +433,29 @@ def test_topk_order_and_ties():
     for i in range(3):
         want = sorted(range(200), key=lambda j: (-sc[i, j], j))[:10]
         assert list(idx[i]) == want
+
+
+@pytest.mark.parametrize("bits,d", [(1, 128), (2, 128), (3, 128), (4, 128), (2, 64), (3, 1536)])
+def test_plane_identity_of_symmetric_codebooks(bits, d):
+    # With s_k = 2 bit_k - 1, every function of the code is a multilinear
+    # polynomial in the s_k (Walsh expansion); a codebook with
+    # cen[c] = -cen[2^b - 1 - c] has only odd-degree terms, and the product of
+    # an odd set of s_k equals 2 * xor(bits) - 1.  Checked exhaustively.
+    cen = O.published_codebook(bits, d)[0].astype(np.float64)
+    L = 1 << bits
+    sgn = np.array([[1.0 if (c >> k) & 1 else -1.0 for k in range(bits)] for c in range(L)])
+    coef = {}
+    for S in range(1, L):
+        prod = np.prod(np.where([(S >> k) & 1 for k in range(bits)], sgn, 1.0), axis=1)
+        coef[S] = float(cen @ prod) / L
+    assert abs(float(cen.sum()) / L) == 0.0
+    for S, a in coef.items():
+        if bin(S).count("1") % 2 == 0:
+            assert a == 0.0, (S, a)
+    for c in range(L):
+        rec = 0.0
+        for S, a in coef.items():
+            if bin(S).count("1") % 2 == 1:
+                par = bin(c & S).count("1") & 1
+                rec += a * (2.0 * par - 1.0 if bin(S).count("1") % 2 else 1.0)
+        assert abs(rec - cen[c]) < 1e-12 * (1 + abs(cen[c]))

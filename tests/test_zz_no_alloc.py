@@ -41,7 +41,7 @@ def _case(B, Hq, Hkv, T, d, bits, m, dtype, seed):
     K = tq.Compressed.empty(kc, B * Hkv * T)
     tq.tq_quantize(kc, k, K)
     ref = torch.empty((B, Hq, T), device=dev)
-    ws = tq.workspace(tq.tq_scores_workspace_size(kc, B, Hq), dev)
+    ws = tq.workspace(tq.tq_scores_workspace_size(kc, B, Hq, Hkv), dev)
     tq.tq_scores(kc, q, B, Hq, Hkv, T, K, ref, ws)
     return kc, q, K, ref
 
@@ -79,7 +79,7 @@ def test_noalloc_rejects_requests_above_its_scratch():
     d, m = 128, 128
     kc = tq.Codec(d, (2,), m, 0)
     B, Hq, Hkv, T = 64, 64, 64, 4           # 4096 queries x (d + m) floats = 4 MiB of scratch
-    assert tq.tq_scores_workspace_size(kc, B, Hq) > (2 << 20)
+    assert tq.tq_scores_workspace_size(kc, B, Hq, Hkv) > (2 << 20)
     dev = torch.device("cuda", 0)
     q = torch.zeros((B, Hq, d), device=dev)
     K = tq.Compressed.empty(kc, B * Hkv * T)
