@@ -93,6 +93,10 @@ cudaError_t tq_launch_qprep(const tq_params& p, const void* q, tq_dtype dt, int 
 cudaError_t tq_launch_scores(const tq_params& p, const float* qprep, int B, int Hq, int Hkv, int64_t T,
                              const tq_compressed& K, float* logits, cudaStream_t st);
 int tq_attend_chunks(int B, int Hq, int Hkv, int64_t T, int num_sms);
+// fused attention (tq_attend.cu): d in {64, 128}, m <= 256; cudaErrorNotSupported otherwise
+cudaError_t tq_launch_attend_fused(const tq_params& kp, const tq_params& vp, const float* qprep, int B, int Hq,
+                                   int Hkv, int64_t T, float scale, const tq_compressed& K, const tq_compressed& V,
+                                   float* partials, int nchunk, cudaStream_t st);
 cudaError_t tq_launch_attend(const tq_params& kp, const tq_params& vp, const float* qprep, int B, int Hq,
                              int Hkv, int64_t T, float scale, const tq_compressed& K, const tq_compressed& V,
                              float* partials, int nchunk, float* out, cudaStream_t st);

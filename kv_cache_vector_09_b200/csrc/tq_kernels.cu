@@ -657,8 +657,8 @@ int tq_attend_chunks(int B, int Hq, int Hkv, int64_t T, int sms) {
 cudaError_t tq_launch_attend(const tq_params& kp, const tq_params& vp, const float* qprep, int B, int Hq, int Hkv,
                              int64_t T, float scale, const tq_compressed& K, const tq_compressed& V, float* partials,
                              int nchunk, float* out, cudaStream_t st) {
-  cudaError_t e;
-  {
+  cudaError_t e = tq_launch_attend_fused(kp, vp, qprep, B, Hq, Hkv, T, scale, K, V, partials, nchunk, st);
+  if (e == cudaErrorNotSupported) {
     auto run = [&]() -> cudaError_t {
       TQ_DISPATCH_NG(Hq / Hkv, (launch_attend_g<NG>(kp, vp, qprep, B, Hq, Hkv, T, scale, K, V, partials, nchunk, st)));
     };
