@@ -218,6 +218,29 @@ TQ_API tq_status tq_attend(const tq_codec *kc, const tq_codec *vc, const void *q
                     const tq_compressed *V, void *workspace, size_t ws_bytes,
                     float *out, void *stream);
 
+/* Workspace bytes for tq_search_topk with nq queries and top-k (k >= 1). */
+TQ_API tq_status tq_search_workspace_size(const tq_codec *codec, int nq, int k,
+                                          size_t *bytes);
+
+/* Nearest-neighbour search over a compressed index (the vector-search use
+ * the "Google acelera LLMs em 8 vezes" page names: an index of quantised
+ * embeddings searched by inner product, with no indexing beyond quantising).
+ * For every query i < nq (q: [nq][d], dtype as tq_scores) and every index row
+ * t < n (index: n rows written by tq_quantize with the same codec), the score
+ * is the tq_scores estimate
+ *   s(i, t) = nu_t (<q'_i, cen[c_t]> / sqrt(d) + gamma_t sqrt(pi/2)/m <S q'_i, 2 b_t - 1>)
+ * and idx[i][0..k) / score[i][0..k) (device, int32 / fp32, row-major) receive
+ * the k best rows in descending score, ties to the lower row index.  The
+ * scores are never stored in full: tensor-core tiles of 128 rows x 256
+ * queries feed per-query top-k lists.  Requires one segment (nseg = 1),
+ * d a multiple of 32 with 64 <= d <= 2048, m <= 512, k <= 32, 1 <= k <= n,
+ * n < 2^31.  The workspace (device, 256-byte aligned) is sized by
+ * tq_search_workspace_size.                                                 */
+TQ_API tq_status tq_search_topk(const tq_codec *codec, const void *q, tq_dtype dtype,
+                                int nq, const tq_compressed *index, int64_t n, int k,
+                                int32_t *idx, float *score, void *workspace,
+                                size_t ws_bytes, void *stream);
+
 /* Device-side health of a codec.  Kernels that wait on tensor-core or copy
  * completion give up after a bounded time (about two seconds), record a
  * nonzero code in the codec's device error word and return early.  This call

@@ -58,6 +58,8 @@ def _load() -> ctypes.CDLL:
         "tq_scores_noalloc": [P, P, I, I, I, I, I64, P, P, P],
         "tq_attend_workspace_size": [P, P, I, I, I, I64, ctypes.POINTER(SZ)],
         "tq_attend": [P, P, P, I, I, I, I, I64, ctypes.c_float, P, P, P, SZ, P, P],
+        "tq_search_workspace_size": [P, I, I, ctypes.POINTER(SZ)],
+        "tq_search_topk": [P, P, I, I, P, I64, I, P, P, P, SZ, P],
         "tq_codec_device_error": [P, P, ctypes.POINTER(ctypes.c_uint32)],
         "tq_codec_exact_rows": [P, P, I, ctypes.POINTER(ctypes.c_uint64)],
     }
@@ -240,6 +242,25 @@ def tq_attend(kc: Codec, vc: Codec, q: torch.Tensor, B: int, Hq: int, Hkv: int, 
                           workspace.numel() * workspace.element_size(), out.data_ptr(), _stream(stream)),
            "tq_attend")
     return out
+
+
+def tq_search_workspace_size(codec: Codec, nq: int, k: int) -> int:
+    v = ctypes.c_size_t()
+    _check(_lib.tq_search_workspace_size(codec.handle, nq, k, ctypes.byref(v)), "tq_search_workspace_size")
+    return v.value
+
+
+def tq_search_topk(codec: Codec, q: torch.Tensor, index: Compressed, n: int, k: int, idx: torch.Tensor,
+                   score: torch.Tensor, workspace: torch.Tensor, stream=None):
+    """Top-k index rows per query (idx int32 [nq, k], score fp32 [nq, k])."""
+    assert q.is_contiguous() and q.dim() == 2
+    assert idx.dtype == torch.int32 and score.dtype == torch.float32 and idx.is_contiguous() and score.is_contiguous()
+    xs = index.struct()
+    _check(_lib.tq_search_topk(codec.handle, q.data_ptr(), _DTYPES[q.dtype], q.shape[0], ctypes.byref(xs), n, k,
+                               idx.data_ptr(), score.data_ptr(), workspace.data_ptr(),
+                               workspace.numel() * workspace.element_size(), _stream(stream)),
+           "tq_search_topk")
+    return idx, score
 
 
 def tq_codec_device_error(codec: Codec, stream=None) -> int:

@@ -7,6 +7,7 @@ statically, so the library depends only on the driver.
 """
 from __future__ import annotations
 
+import concurrent.futures
 import hashlib
 import os
 import shutil
@@ -63,7 +64,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     nvcc = _nvcc()
     objdir = os.path.join(HERE, "_build")
     os.makedirs(objdir, exist_ok=True)
-    objs = []
+    jobs = []
     for src in sources():
         obj = os.path.join(objdir, os.path.basename(src) + ".o")
         cmd = [nvcc, *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), "-c", src, "-o", obj]
@@ -71,8 +72,14 @@ def build(force: bool = False, verbose: bool = False) -> str:
             cmd = [nvcc, "-x", "cu", *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), "-c", src, "-o", obj]
         if verbose:
             print(" ".join(cmd), flush=True)
-        subprocess.run(cmd, check=True)
-        objs.append(obj)
+        jobs.append((cmd, obj))
+    # one nvcc process per translation unit, run side by side
+    workers = max(1, min(len(jobs), os.cpu_count() or 1))
+    with concurrent.futures.ThreadPoolExecutor(max_workers=workers) as ex:
+        for r in ex.map(lambda j: subprocess.run(j[0]), jobs):
+            if r.returncode != 0:
+                raise subprocess.CalledProcessError(r.returncode, r.args)
+    objs = [obj for _, obj in jobs]
     tmp = LIB + ".tmp"
     cmd = [nvcc, *NVCC_FLAGS, "-shared", "-cudart", "static", "-o", tmp, *objs]
     if verbose:

@@ -596,6 +596,55 @@ extern "C" tq_status tq_attend(const tq_codec* kc, const tq_codec* vc, const voi
   return launch_status(e, "tq_attend launch");
 }
 
+// ---------------------------------------------------------------- search
+static tq_status check_search_codec(const tq_codec* c, const char* name) {
+  if (c->p.nseg != 1) return tq_fail(TQ_ERR_UNSUPPORTED, "%s: needs one segment (nseg = %d)", name, c->p.nseg);
+  if (c->p.d % 32 != 0 || c->p.d < 64 || c->p.d > 2048)
+    return tq_fail(TQ_ERR_UNSUPPORTED, "%s: d = %d (needs a multiple of 32 in [64, 2048])", name, c->p.d);
+  if (c->p.m > 512) return tq_fail(TQ_ERR_UNSUPPORTED, "%s: m = %d above 512", name, c->p.m);
+  return TQ_OK;
+}
+
+extern "C" tq_status tq_search_workspace_size(const tq_codec* c, int nq, int k, size_t* bytes) {
+  if (!c || !bytes) return tq_fail(TQ_ERR_INVALID_ARG, "tq_search_workspace_size: null argument");
+  if (nq < 0 || k < 1 || k > 32) return tq_fail(TQ_ERR_INVALID_ARG, "tq_search_workspace_size: nq = %d, k = %d", nq, k);
+  tq_status st = check_search_codec(c, "tq_search_workspace_size");
+  if (st != TQ_OK) return st;
+  *bytes = tq_search_bytes(c->p, nq > 0 ? nq : 1, k, device_sms(c->device < 0 ? 0 : c->device));
+  return TQ_OK;
+}
+
+extern "C" tq_status tq_search_topk(const tq_codec* c, const void* q, tq_dtype dt, int nq, const tq_compressed* X,
+                                    int64_t n, int k, int32_t* idx, float* score, void* workspace, size_t ws_bytes,
+                                    void* stream) {
+  tq_status st = check_device_codec(c, "tq_search_topk");
+  if (st != TQ_OK) return st;
+  if ((st = check_search_codec(c, "tq_search_topk")) != TQ_OK) return st;
+  if ((st = check_dtype(dt)) != TQ_OK) return st;
+  if (nq < 0) return tq_fail(TQ_ERR_INVALID_ARG, "tq_search_topk: nq = %d", nq);
+  if (k < 1 || k > 32) return tq_fail(TQ_ERR_INVALID_ARG, "tq_search_topk: k = %d outside [1, 32]", k);
+  if (n < k || n >= ((int64_t)1 << 31))
+    return tq_fail(TQ_ERR_INVALID_ARG, "tq_search_topk: n = %lld (needs k <= n < 2^31)", (long long)n);
+  if (nq == 0) return TQ_OK;
+  if (!q || !aligned16(q)) return tq_fail(TQ_ERR_INVALID_ARG, "tq_search_topk: q null or not 16-byte aligned");
+  if (!idx || !score) return tq_fail(TQ_ERR_INVALID_ARG, "tq_search_topk: idx / score null");
+  if ((st = check_compressed(c, X, "index")) != TQ_OK) return st;
+  const size_t need = tq_search_bytes(c->p, nq, k, device_sms(c->device));
+  if (!workspace || ((uintptr_t)workspace & 255u) != 0 || ws_bytes < need)
+    return tq_fail(TQ_ERR_INVALID_ARG, "tq_search_topk: workspace null, not 256-byte aligned or smaller than %zu bytes",
+                   need);
+  const cudaStream_t s = (cudaStream_t)stream;
+  const int nb = tq_search_batch(nq, k);
+  const size_t esz = dtype_size(dt);
+  for (int q0 = 0; q0 < nq; q0 += nb) {
+    const int cnt = std::min(nb, nq - q0);
+    cudaError_t e = tq_launch_qprep(c->p, (const char*)q + (size_t)q0 * c->p.d * esz, dt, cnt, (float*)workspace, s);
+    if (e == cudaSuccess) e = tq_launch_search(c->p, (const float*)workspace, cnt, q0, *X, n, k, idx, score, workspace, s);
+    if (e != cudaSuccess) return launch_status(e, "tq_search_topk launch");
+  }
+  return TQ_OK;
+}
+
 extern "C" tq_status tq_codec_device_error(const tq_codec* c, void* stream, uint32_t* code) {
   tq_status st = check_device_codec(c, "tq_codec_device_error");
   if (st != TQ_OK) return st;

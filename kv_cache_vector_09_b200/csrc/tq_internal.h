@@ -93,6 +93,12 @@ cudaError_t tq_launch_qprep(const tq_params& p, const void* q, tq_dtype dt, int 
 cudaError_t tq_launch_scores(const tq_params& p, const float* qprep, int B, int Hq, int Hkv, int64_t T,
                              const tq_compressed& K, float* logits, cudaStream_t st);
 int tq_attend_chunks(int B, int Hq, int Hkv, int64_t T, int num_sms);
+// top-k search (tq_search.cu): queries per batch, workspace bytes, and one
+// batch of nq queries (qprep at the start of ws, written by the caller)
+int tq_search_batch(int nq, int k);
+size_t tq_search_bytes(const tq_params& p, int nq, int k, int nsm);
+cudaError_t tq_launch_search(const tq_params& p, const float* qprep, int nq, int q0, const tq_compressed& X,
+                             int64_t n, int k, int32_t* idx, float* score, void* ws, cudaStream_t st);
 // fused attention (tq_attend.cu): d in {64, 128}, m <= 256; cudaErrorNotSupported otherwise
 cudaError_t tq_launch_attend_fused(const tq_params& kp, const tq_params& vp, const float* qprep, int B, int Hq,
                                    int Hkv, int64_t T, float scale, const tq_compressed& K, const tq_compressed& V,

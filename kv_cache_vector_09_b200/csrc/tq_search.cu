@@ -1,0 +1,556 @@
+// Top-k search over a compressed index on the tensor cores (kind::f16
+// tcgen05.mma, fp32 accumulation in TMEM).
+//
+// The score of query i and index row t is the estimator of tq_scores,
+//   s = nu_t / sqrt(d) * ( sum_c q'_c cen[code_c] + g_t sum_j w_j sgn_j ),
+//   g_t = gamma_t sqrt(pi/2) / m * sqrt(d),   w = S q',   sgn = 2 bit - 1,
+// a dense contraction of the dequantised row against the query.  Both sides
+// are split into fp16 hi + lo parts and three products per element are
+// accumulated (hi*hi + lo*hi + hi*lo; the omitted lo*lo is below 2^-22 of
+// the term), in K groups of 16 elements:
+//   group of 16 coordinates:  A = [cen_hi | cen_lo | cen_hi],  B = [q_hi | q_hi | q_lo]
+//   group of 16 sketch rows:  A = [g_hi s | g_lo s | g_hi s],  B = [w_hi | w_hi | w_lo]
+// with B scaled per query by 2^e (w by 2^(e-6), g by 2^6) to keep the fp16
+// parts normal.  A is built per 128-row tile by CUDA-core warps straight
+// into TMEM (codes -> centroid hi/lo pairs), B is a per-query image built
+// once per call and streamed from L2 by bulk copies.  One block per SM:
+//   warps 0-7   A builders (warps 0-3 even groups, 4-7 odd groups; warp w
+//               writes TMEM lanes 32 (w % 4) ..)
+//   warp 8      B producer (bulk copies into a 4-stage ring)
+//   warp 9      MMA issue: 3 MMAs (M = 128, N = 256, K = 16) per group
+//   warps 10-13 epilogue: scores of the tile -> per-query top-k lists in
+//               shared memory (insertions under a per-query lock)
+// A final kernel merges the blocks' lists.  Every mbarrier wait is bounded.
+#include <math.h>
+
+#include <algorithm>
+
+#include "tq_common.cuh"
+#include "tq_internal.h"
+#include "tq_tc.cuh"
+
+namespace {
+
+constexpr int kRowsT = 128;                // index rows per tile (MMA M)
+constexpr int kQT = 256;                   // queries per tile (MMA N)
+constexpr int kStepBytes = kQT * 16 * 2;   // one K = 16 step of B: 8 KB
+constexpr int kGroupBytes = 3 * kStepBytes;
+constexpr int kBStages = 4;
+constexpr int kASlots = 8;                 // TMEM A ring, 32 columns per slot
+constexpr int kThreads = 448;
+constexpr float kQjlGain = 64.f;           // 2^6 on the A side of the sketch groups
+
+__device__ __forceinline__ uint32_t spread4(uint32_t x) { return (x * 0x00204081u) & 0x01010101u; }
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t half_bits(float v) { return (uint32_t)__half_as_ushort(__float2half_rn(v)); }
+
+__device__ __forceinline__ bool better(float s, int r, float ts, int tr) { return s > ts || (s == ts && r < tr); }
+
+// ---------------------------------------------------------------- query side
+// Per-query exponent e: max(|q'|, |w| 2^-6) 2^e < 2^14.
+__global__ void __launch_bounds__(256) search_qexp_kernel(const float* __restrict__ qprep, int nq, int d, int m,
+                                                          int* __restrict__ qexp, float* __restrict__ qscale) {
+  const int lane = threadIdx.x & 31;
+  const int qi = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (qi >= nq) return;
+  const float* row = qprep + (size_t)qi * (d + m);
+  float mx = 0.f;
+  for (int i = lane; i < d; i += 32) mx = fmaxf(mx, fabsf(row[i]));
+  for (int j = lane; j < m; j += 32) mx = fmaxf(mx, fabsf(row[d + j]) * (1.f / kQjlGain));
+  mx = tq_warp_max(mx);
+  if (lane == 0) {
+    int ex = 0;
+    frexpf(mx > 0.f ? mx : 1.f, &ex);
+    const int e = 14 - ex;
+    qexp[qi] = e;
+    qscale[qi] = ldexpf(1.f, -e);
+  }
+}
+
+// B image: [query tile][group][step][8 KB], one thread per (query, group).
+// Within a step: element (n, kk) at (kk / 8) * 4096 + (n / 8) * 128 + (n % 8) * 16 + (kk % 8) * 2.
+__global__ void __launch_bounds__(256) search_bimg_kernel(const float* __restrict__ qprep, const int* __restrict__ qexp,
+                                                          int nq, int nqt, int d, int m, uint8_t* __restrict__ img) {
+  const int ngroups = d / 16 + m / 16;
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (int64_t)nqt * kQT * ngroups) return;
+  const int n_all = (int)(idx % (nqt * kQT));
+  const int g = (int)(idx / (nqt * kQT));
+  const int qt = n_all / kQT, n = n_all % kQT;
+  uint32_t hi[8], lo[8];
+  if (n_all < nq) {
+    const float* row = qprep + (size_t)n_all * (d + m);
+    const int e = qexp[n_all];
+    const bool sk = g >= d / 16;
+    const float* src = sk ? row + d + 16 * (g - d / 16) : row + 16 * g;
+    const int es = sk ? e - 6 : e;
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      uint32_t h2 = 0u, l2 = 0u;
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const float v = ldexpf(src[2 * p + t], es);
+        const __half h = __float2half_rn(v);
+        const float r = v - __half2float(h);
+        h2 |= (uint32_t)__half_as_ushort(h) << (16 * t);
+        l2 |= half_bits(r) << (16 * t);
+      }
+      hi[p] = h2;
+      lo[p] = l2;
+    }
+  } else {
+#pragma unroll
+    for (int p = 0; p < 8; ++p) hi[p] = lo[p] = 0u;
+  }
+  uint8_t* gbase = img + ((size_t)qt * ngroups + g) * kGroupBytes;
+  const uint32_t off = (uint32_t)(n / 8) * 128u + (uint32_t)(n % 8) * 16u;
+  const uint32_t* parts[3] = {hi, hi, lo};
+#pragma unroll
+  for (int s = 0; s < 3; ++s) {
+    const uint32_t* v = parts[s];
+    *reinterpret_cast<uint4*>(gbase + s * kStepBytes + off) = make_uint4(v[0], v[1], v[2], v[3]);
+    *reinterpret_cast<uint4*>(gbase + s * kStepBytes + 4096 + off) = make_uint4(v[4], v[5], v[6], v[7]);
+  }
+}
+
+// ---------------------------------------------------------------- search
+struct SearchArgs {
+  const uint32_t* codes;
+  const uint32_t* signs;
+  const float* norms;
+  const float* rnorms;
+  int64_t n;
+  int nq;          // queries in this batch
+  int nqt;         // query tiles
+  int k;
+  const uint8_t* img;
+  const float* qscale;
+  float* part_s;   // [grid][nq][k]
+  int* part_i;
+};
+
+__device__ __forceinline__ int64_t unit_begin(int64_t units, int b, int g) { return units * b / g; }
+
+template <int BITS>
+__global__ void __launch_bounds__(kThreads, 1)
+    search_kernel(const tq_params p, const SearchArgs a) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  __shared__ uint64_t a_full[kASlots], a_empty[kASlots], b_full[kBStages], b_empty[kBStages];
+  __shared__ uint64_t d_full, d_empty, drained;
+  __shared__ uint32_t s_tmem;
+  __shared__ volatile int s_abort;
+  __shared__ uint32_t s_cen[16];  // fp16 cen hi | lo << 16, by code
+
+  const int d = p.d, m = p.m, W = p.W, MS = p.MS, PW = p.pw;
+  const int gc = d / 16, ngroups = gc + m / 16;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nq = a.nq, k = a.k;
+
+  unsigned char* bring = smem;                                        // [kBStages][kGroupBytes]
+  float* tops = reinterpret_cast<float*>(smem + kBStages * kGroupBytes);  // [nq][k]
+  int* tidx = reinterpret_cast<int*>(tops + (size_t)nq * k);              // [nq][k]
+  int* locks = tidx + (size_t)nq * k;                                     // [nq]
+
+  const int64_t nkt = (a.n + kRowsT - 1) / kRowsT;
+  const int64_t units = nkt * a.nqt;
+  const int64_t u0 = unit_begin(units, blockIdx.x, gridDim.x), u1 = unit_begin(units, blockIdx.x + 1, gridDim.x);
+  const int64_t nul = u1 - u0;
+
+  for (int i = tid; i < nq * k; i += kThreads) {
+    tops[i] = -INFINITY;
+    tidx[i] = 0x7FFFFFFF;
+  }
+  for (int i = tid; i < nq; i += kThreads) locks[i] = 0;
+  if (tid < 16) {
+    const float c = tid < (1 << BITS) ? p.cen[0][tid] : 0.f;
+    const __half h = __float2half_rn(c);
+    s_cen[tid] = (uint32_t)__half_as_ushort(h) | (half_bits(c - __half2float(h)) << 16);
+  }
+  if (tid == 0) {
+    for (int i = 0; i < kASlots; ++i) {
+      tqtc::mbar_init(&a_full[i], 128);
+      tqtc::mbar_init(&a_empty[i], 1);
+    }
+    for (int i = 0; i < kBStages; ++i) {
+      tqtc::mbar_init(&b_full[i], 1);
+      tqtc::mbar_init(&b_empty[i], 1);
+    }
+    tqtc::mbar_init(&d_full, 1);
+    tqtc::mbar_init(&d_empty, 128);
+    tqtc::mbar_init(&drained, 1);
+    tqtc::fence_mbar_init();
+    s_abort = 0;
+  }
+  if (warp == 0) tqtc::tmem_alloc(&s_tmem, 512);
+  tqtc::tc_fence_before();
+  __syncthreads();
+  tqtc::tc_fence_after();
+  const uint32_t tbase = s_tmem;  // D: columns [0, 256); A ring: [256, 512)
+  auto fail = [&](uint32_t code) {
+    atomicExch(p.err, code);
+    s_abort = 1;
+  };
+
+  if (warp < 8) {
+    // ---------------------------------------------------------- A builders
+    const int set = warp >> 2;
+    const uint32_t lane_base = 32u * (uint32_t)(warp & 3);
+    const int rloc = 32 * (warp & 3) + lane;
+    const float gk = p.qjl_coef * sqrtf((float)d) * kQjlGain;
+    for (int64_t ul = 0; ul < nul && !s_abort; ++ul) {
+      const int64_t kt = (u0 + ul) / a.nqt;
+      const int64_t row = kt * kRowsT + rloc;
+      const bool valid = row < a.n;
+      const uint32_t* crow = a.codes + (valid ? row : 0) * W;
+      const uint32_t* srow = a.signs + (valid ? row : 0) * MS;
+      uint32_t ghi2 = 0u, glo2 = 0u;
+      if (m > 0) {
+        const float g = valid ? __ldg(a.rnorms + row) * gk : 0.f;
+        const __half h = __float2half_rn(g);
+        const uint32_t hb = __half_as_ushort(h), lb = half_bits(g - __half2float(h));
+        ghi2 = hb | (hb << 16);
+        glo2 = lb | (lb << 16);
+      }
+      for (int g = set; g < ngroups; g += 2) {
+        const int64_t x = ul * ngroups + g;
+        const int slot = (int)(x % kASlots);
+        uint32_t hi[8], lo[8];
+        if (g < gc) {
+          const int w = g >> 1, sh = 16 * (g & 1);
+          uint32_t pl[BITS];
+#pragma unroll
+          for (int b = 0; b < BITS; ++b) pl[b] = valid ? (__ldg(crow + b * PW + w) >> sh) : 0u;
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            uint32_t y = 0u;  // byte r = 4 * code of coordinate 16 g + 4 t + r
+#pragma unroll
+            for (int b = 0; b < BITS; ++b) y |= spread4((pl[b] >> (4 * t)) & 0xFu) << (b + 2);
+            uint32_t hl[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+              hl[r] = *reinterpret_cast<const uint32_t*>(reinterpret_cast<const char*>(s_cen) + ((y >> (8 * r)) & 0xFFu));
+            hi[2 * t] = prmt(hl[0], hl[1], 0x5410);
+            lo[2 * t] = prmt(hl[0], hl[1], 0x7632);
+            hi[2 * t + 1] = prmt(hl[2], hl[3], 0x5410);
+            lo[2 * t + 1] = prmt(hl[2], hl[3], 0x7632);
+          }
+        } else {
+          const int j0 = 16 * (g - gc);
+          const uint32_t bits = valid ? (__ldg(srow + (j0 >> 5)) >> (j0 & 16)) : 0xFFFFu;
+#pragma unroll
+          for (int pp = 0; pp < 8; ++pp) {
+            // sign bit 0 -> negative: flip the fp16 sign bits
+            const uint32_t nb = ~bits >> (2 * pp);
+            const uint32_t mask = ((nb & 1u) << 15) | ((nb & 2u) << 30);
+            hi[pp] = ghi2 ^ mask;
+            lo[pp] = glo2 ^ mask;
+          }
+        }
+        if (x >= kASlots &&
+            !tqtc::mbar_wait_or_abort(&a_empty[slot], (uint32_t)((x / kASlots - 1) & 1), &s_abort)) {
+          fail(tqtc::kErrMmaWait);
+          break;
+        }
+        tqtc::tc_fence_after();
+        const uint32_t col = 256u + 32u * (uint32_t)slot;
+        tqtc::tmem_st8(tqtc::tmem_addr(tbase, lane_base, col), hi);
+        tqtc::tmem_st8(tqtc::tmem_addr(tbase, lane_base, col + 8u), lo);
+        tqtc::tmem_st8(tqtc::tmem_addr(tbase, lane_base, col + 16u), hi);
+        tqtc::tmem_wait_st();
+        tqtc::tc_fence_before();
+        tqtc::mbar_arrive(&a_full[slot]);
+      }
+    }
+  } else if (warp == 8) {
+    // ---------------------------------------------------------- B producer
+    if (lane == 0) {
+      int64_t issued = 0;
+      for (int64_t ul = 0; ul < nul && !s_abort; ++ul) {
+        const int64_t qt = (u0 + ul) % a.nqt;
+        const uint8_t* src = a.img + (size_t)qt * ngroups * kGroupBytes;
+        for (int g = 0; g < ngroups; ++g) {
+          const int64_t x = ul * ngroups + g;
+          const int st = (int)(x % kBStages);
+          if (x >= kBStages &&
+              !tqtc::mbar_wait_or_abort(&b_empty[st], (uint32_t)((x / kBStages - 1) & 1), &s_abort)) {
+            fail(tqtc::kErrCopyWait);
+            break;
+          }
+          tqtc::mbar_arrive_expect_tx(&b_full[st], (uint32_t)kGroupBytes);
+          tqtc::bulk_g2s(bring + (size_t)st * kGroupBytes, src + (size_t)g * kGroupBytes, (uint32_t)kGroupBytes,
+                         &b_full[st]);
+          issued = x + 1;
+        }
+      }
+      // let every copy still in flight land before the block exits (bounded)
+      for (int64_t x = issued > kBStages ? issued - kBStages : 0; x < issued; ++x)
+        if (!tqtc::mbar_wait_or_abort(&b_full[x % kBStages], (uint32_t)((x / kBStages) & 1), nullptr))
+          atomicExch(p.err, tqtc::kErrCopyWait);
+    }
+  } else if (warp == 9) {
+    // ---------------------------------------------------------- MMA issue
+    if (lane == 0) {
+      const uint32_t idesc = tqtc::instr_desc(1, 0, 0, kRowsT, kQT);
+      const uint32_t bbase = tqtc::smem_u32(bring);
+      for (int64_t ul = 0; ul < nul && !s_abort; ++ul) {
+        if (ul >= 1 && !tqtc::mbar_wait_or_abort(&d_empty, (uint32_t)((ul - 1) & 1), &s_abort)) {
+          fail(tqtc::kErrMmaWait);
+          break;
+        }
+        bool ok = true;
+        for (int g = 0; g < ngroups; ++g) {
+          const int64_t x = ul * ngroups + g;
+          const int slot = (int)(x % kASlots), st = (int)(x % kBStages);
+          if (!tqtc::mbar_wait_or_abort(&a_full[slot], (uint32_t)((x / kASlots) & 1), &s_abort) ||
+              !tqtc::mbar_wait_or_abort(&b_full[st], (uint32_t)((x / kBStages) & 1), &s_abort)) {
+            fail(tqtc::kErrMmaWait);
+            ok = false;
+            break;
+          }
+          tqtc::tc_fence_after();
+          const uint32_t acol = tbase + 256u + 32u * (uint32_t)slot;
+          const uint32_t b0 = bbase + (uint32_t)st * kGroupBytes;
+#pragma unroll
+          for (int s = 0; s < 3; ++s)
+            tqtc::mma_f16_ts(tbase, acol + 8u * (uint32_t)s,
+                             tqtc::smem_desc(b0 + (uint32_t)s * kStepBytes, 4096u, 128u), idesc, g > 0 || s > 0);
+          tqtc::mma_commit(&a_empty[slot]);
+          tqtc::mma_commit(&b_empty[st]);
+        }
+        if (!ok) break;
+        tqtc::mma_commit(&d_full);
+      }
+      tqtc::mma_commit(&drained);
+      if (!tqtc::mbar_wait_or_abort(&drained, 0, nullptr)) atomicExch(p.err, tqtc::kErrMmaWait);
+    }
+  } else {
+    // ---------------------------------------------------------- epilogue
+    const uint32_t quarter = (uint32_t)(warp & 3);
+    const int rloc = 32 * (int)quarter + lane;
+    const float inv_sqrt_d = p.inv_sqrt_d;
+    for (int64_t ul = 0; ul < nul; ++ul) {
+      const int64_t kt = (u0 + ul) / a.nqt, qt = (u0 + ul) % a.nqt;
+      const int64_t row = kt * kRowsT + rloc;
+      const bool valid = row < a.n;
+      const float rs = valid ? __ldg(a.norms + row) * inv_sqrt_d : 0.f;
+      if (!tqtc::mbar_wait_or_abort(&d_full, (uint32_t)(ul & 1), &s_abort)) {
+        fail(tqtc::kErrMmaWait);
+        break;
+      }
+      tqtc::tc_fence_after();
+      for (int c = 0; c < kQT / 32; ++c) {
+        uint32_t dv[32];
+        tqtc::tmem_ld16(tqtc::tmem_addr(tbase, 32u * quarter, 32u * c), *reinterpret_cast<uint32_t(*)[16]>(dv));
+        tqtc::tmem_ld16(tqtc::tmem_addr(tbase, 32u * quarter, 32u * c + 16u),
+                        *reinterpret_cast<uint32_t(*)[16]>(dv + 16));
+        tqtc::tmem_wait_ld();
+        if (c == kQT / 32 - 1) {
+          tqtc::tc_fence_before();
+          tqtc::mbar_arrive(&d_empty);
+        }
+        const int qbase = (int)qt * kQT + 32 * c;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int qi = qbase + j;
+          if (qi >= nq) continue;
+          const float s = __uint_as_float(dv[j]) * rs * __ldg(a.qscale + qi);
+          float* tq = tops + (size_t)qi * k;
+          int* ti = tidx + (size_t)qi * k;
+          const volatile float* vtq = tq;
+          const volatile int* vti = ti;
+          bool cand = valid && better(s, (int)row, vtq[k - 1], vti[k - 1]);
+          unsigned mask = __ballot_sync(0xFFFFFFFFu, cand);
+          while (mask) {
+            const int leader = __ffs(mask) - 1;
+            if (lane == leader) {
+              bool done = false;
+              for (int spin = 0; spin < (1 << 22) && !done; ++spin) {
+                if (atomicCAS(&locks[qi], 0, 1) == 0) {
+                  __threadfence_block();
+                  if (better(s, (int)row, vtq[k - 1], vti[k - 1])) {
+                    int pos = k - 1;
+                    while (pos > 0 && better(s, (int)row, vtq[pos - 1], vti[pos - 1])) {
+                      tq[pos] = vtq[pos - 1];
+                      ti[pos] = vti[pos - 1];
+                      --pos;
+                    }
+                    tq[pos] = s;
+                    ti[pos] = (int)row;
+                  }
+                  __threadfence_block();
+                  atomicExch(&locks[qi], 0);
+                  done = true;
+                }
+              }
+              if (!done) fail(tqtc::kErrMmaWait);
+            }
+            mask &= mask - 1;
+            __syncwarp();
+          }
+        }
+      }
+    }
+  }
+  tqtc::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tqtc::tmem_dealloc(tbase, 512);
+  // this block's lists
+  float* ps = a.part_s + (size_t)blockIdx.x * nq * k;
+  int* pi = a.part_i + (size_t)blockIdx.x * nq * k;
+  for (int i = tid; i < nq * k; i += kThreads) {
+    ps[i] = tops[i];
+    pi[i] = tidx[i];
+  }
+}
+
+// Merge the blocks' lists: one warp per query, k rounds of a warp argmax
+// over the candidates ranked below the previous pick.
+__global__ void __launch_bounds__(256) search_merge_kernel(const float* __restrict__ part_s,
+                                                           const int* __restrict__ part_i, int nblk, int nq, int k,
+                                                           int q0, int32_t* __restrict__ idx, float* __restrict__ score) {
+  const int lane = threadIdx.x & 31;
+  const int qi = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (qi >= nq) return;
+  float ps = INFINITY;
+  int pr = -1;
+  for (int r = 0; r < k; ++r) {
+    float bs = -INFINITY;
+    int br = 0x7FFFFFFF;
+    for (int c = lane; c < nblk * k; c += 32) {
+      const int blk = c / k, j = c % k;
+      const float s = part_s[((size_t)blk * nq + qi) * k + j];
+      const int rr = part_i[((size_t)blk * nq + qi) * k + j];
+      if (rr == 0x7FFFFFFF) continue;
+      if (better(ps, pr, s, rr) && better(s, rr, bs, br)) {
+        bs = s;
+        br = rr;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float os = __shfl_xor_sync(0xFFFFFFFFu, bs, o);
+      const int orr = __shfl_xor_sync(0xFFFFFFFFu, br, o);
+      if (better(os, orr, bs, br)) {
+        bs = os;
+        br = orr;
+      }
+    }
+    if (lane == 0) {
+      idx[(size_t)(q0 + qi) * k + r] = br;
+      score[(size_t)(q0 + qi) * k + r] = bs;
+    }
+    ps = bs;
+    pr = br;
+  }
+}
+
+int g_sms_search = 0;
+int sms() {
+  if (!g_sms_search) {
+    int dev = 0, v = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+    g_sms_search = v;
+  }
+  return g_sms_search;
+}
+
+}  // namespace
+
+// query batch: the largest multiple of 256 (or nq) whose lists fit 104 KB
+int tq_search_batch(int nq, int k) {
+  const int per = 8 * k + 4;
+  int nb = (104 * 1024 / per) / kQT * kQT;
+  if (nb < kQT) nb = kQT;
+  return nq < nb ? nq : nb;
+}
+
+size_t tq_search_bytes(const tq_params& p, int nq, int k, int nsm) {
+  const int nb = tq_search_batch(nq, k);
+  const int nqt = (nb + kQT - 1) / kQT;
+  const int ngroups = p.d / 16 + p.m / 16;
+  auto al = [](size_t x) { return (x + 255) / 256 * 256; };
+  return al(sizeof(float) * (size_t)nb * (p.d + p.m)) + al(sizeof(int) * nb) + al(sizeof(float) * nb) +
+         al((size_t)nqt * ngroups * kGroupBytes) + 2 * al(sizeof(float) * (size_t)nsm * nb * k);
+}
+
+int tq_search_sms() { return sms(); }
+
+cudaError_t tq_launch_search(const tq_params& p, const float* qprep, int nq, int q0, const tq_compressed& X,
+                             int64_t n, int k, int32_t* idx, float* score, void* ws, cudaStream_t st) {
+  const int nb = nq;  // this batch (<= tq_search_batch)
+  const int nqt = (nb + kQT - 1) / kQT;
+  const int ngroups = p.d / 16 + p.m / 16;
+  const int nsm = sms();
+  auto al = [](size_t x) { return (x + 255) / 256 * 256; };
+  uint8_t* w = reinterpret_cast<uint8_t*>(ws);
+  // qprep sits at the start of the workspace (written by the caller)
+  w += al(sizeof(float) * (size_t)tq_search_batch(nb, k) * (p.d + p.m));
+  int* qexp = reinterpret_cast<int*>(w);
+  w += al(sizeof(int) * tq_search_batch(nb, k));
+  float* qscale = reinterpret_cast<float*>(w);
+  w += al(sizeof(float) * tq_search_batch(nb, k));
+  uint8_t* img = w;
+  w += al((size_t)nqt * ngroups * kGroupBytes);
+  const int64_t nkt = (n + kRowsT - 1) / kRowsT;
+  const int grid = (int)std::min<int64_t>((int64_t)nsm, nkt * nqt);
+  float* part_s = reinterpret_cast<float*>(w);
+  w += al(sizeof(float) * (size_t)nsm * tq_search_batch(nb, k) * k);
+  int* part_i = reinterpret_cast<int*>(w);
+
+  search_qexp_kernel<<<(nb + 7) / 8, 256, 0, st>>>(qprep, nb, p.d, p.m, qexp, qscale);
+  const int64_t nth = (int64_t)nqt * kQT * ngroups;
+  search_bimg_kernel<<<(unsigned)((nth + 255) / 256), 256, 0, st>>>(qprep, qexp, nb, nqt, p.d, p.m, img);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+
+  SearchArgs a;
+  a.codes = X.codes;
+  a.signs = X.signs;
+  a.norms = X.norms;
+  a.rnorms = X.rnorms;
+  a.n = n;
+  a.nq = nb;
+  a.nqt = nqt;
+  a.k = k;
+  a.img = img;
+  a.qscale = qscale;
+  a.part_s = part_s;
+  a.part_i = part_i;
+  size_t smem = (size_t)kBStages * kGroupBytes + (size_t)nb * k * 8 + (size_t)nb * 4;
+  // the block takes all 512 TMEM columns: ask for more than half of the SM's
+  // shared memory so that a second block never waits on the allocation
+  {
+    int dev = 0, per_sm = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess || per_sm <= 0)
+      per_sm = 228 * 1024;
+    smem = std::max(smem, (size_t)(per_sm / 2 + 1024));
+  }
+  switch (p.bits[0]) {
+#define TQ_SEARCH_CASE(B)                                                                                  \
+  case B: {                                                                                                \
+    auto fn = search_kernel<B>;                                                                            \
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);                  \
+    if (e != cudaSuccess) return e;                                                                        \
+    fn<<<grid, kThreads, smem, st>>>(p, a);                                                                \
+    break;                                                                                                 \
+  }
+    TQ_SEARCH_CASE(1)
+    TQ_SEARCH_CASE(2)
+    TQ_SEARCH_CASE(3)
+    TQ_SEARCH_CASE(4)
+#undef TQ_SEARCH_CASE
+    default: return cudaErrorNotSupported;
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  search_merge_kernel<<<(nb + 7) / 8, 256, 0, st>>>(part_s, part_i, grid, nb, k, q0, idx, score);
+  return cudaGetLastError();
+}
