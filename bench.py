@@ -277,6 +277,24 @@ def run_reference(args, rank, world):
     """The oracle as the reference arm: rank 0 only, bounded samples per step."""
     if rank != 0:
         return 0
+    if args.workload == "vsearch":
+        w = synth.VSEARCH
+        times, pairs_total = [], 0
+        for s in range(args.warmup + args.steps):
+            pps, secs, pairs, threads, desc = cpu_search_sample(w, args.ref_step_seconds)
+            if s >= args.warmup:
+                times.append(secs)
+                pairs_total += pairs
+        value = pairs_total / sum(times)
+        print(json.dumps({
+            "metric": SEARCH_METRIC, "value": value, "unit": "pairs/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * sum(times) / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": w.name, "n": w.n, "nq": w.nq, "d": w.d, "bits": list(w.bits), "m": w.m, "k": w.k,
+                       "step": "oracle top-k on a bounded sample per step"},
+            "cpu_baseline": {"value": value, "unit": "pairs/s", "cores": threads, "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": "pairs/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}), flush=True)
+        return 0
     w = synth.WORKLOADS[args.workload]
     times, keys_total = [], 0
     for s in range(args.warmup + args.steps):
@@ -296,6 +314,126 @@ def run_reference(args, rank, world):
         "cpu_baseline": {"value": value, "unit": "keys/s", "cores": threads, "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": "keys/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------- vector search
+SEARCH_METRIC = "query-row pairs scored/s, top-10 search over a 1M-row compressed index (d=1536)"
+
+
+def load_tensor_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["bf16_tflops"]), "measured bf16_tflops (burst; fp16 has the same dense rate)"
+    except Exception:
+        return 1590.0, "fallback 1.59 PFLOP/s"
+
+
+def cpu_search_sample(w, budget_s: float):
+    """The oracle's top-k on a bounded sample: a few queries against the first
+    rows of the index (quantised by the oracle).  Returns (pairs/s, seconds,
+    pairs, threads, description)."""
+    import oracle as O
+    oc = O.make_codec(w.d, w.bits, w.m, w.codec_seed)
+    rows = 4096
+    x = synth.search_rows(w, 0, rows).numpy()
+    X = O.quantize(x, oc)
+    q = synth.search_queries(w)[:64].numpy()
+    t0 = time.perf_counter()
+    done = 0
+    while True:
+        O.search_topk(q[done % 64:done % 64 + 4], X, oc, w.k)
+        done += 4
+        if time.perf_counter() - t0 > budget_s:
+            break
+    secs = time.perf_counter() - t0
+    pairs = done * rows
+    return pairs / secs, secs, pairs, torch.get_num_threads(), \
+        f"{done} queries x {rows} rows of the index (oracle top-{w.k}, quantised by the oracle)"
+
+
+def run_search(args, tq, dev, rank, world, pg):
+    w = synth.VSEARCH
+    codec = tq.Codec(w.d, w.bits, w.m, w.codec_seed, device=dev.index)
+    X = tq.Compressed.empty(codec, w.n, dev)
+    for r0 in range(0, w.n, w.row_block):
+        r1 = min(w.n, r0 + w.row_block)
+        tq.tq_quantize(codec, synth.search_rows(w, r0, r1).to(dev), X.rows(r0, r1))
+    q_host = synth.search_queries(w)
+    q = q_host.to(dev).contiguous()
+    idx = torch.empty((w.nq, w.k), dtype=torch.int32, device=dev)
+    sc = torch.empty((w.nq, w.k), dtype=torch.float32, device=dev)
+    ws = tq.workspace(tq.tq_search_workspace_size(codec, w.nq, w.k), dev)
+    stage = [("tq_search_topk", lambda: tq.tq_search_topk(codec, q, X, w.n, w.k, idx, sc, ws))]
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        stage[0][1]()
+    torch.cuda.synchronize()
+    assert tq.tq_codec_device_error(codec) == 0
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.perf_counter()
+    total_ms, per = time_steps(None, args.steps, stream, stage)
+    t_wall1 = time.perf_counter()
+    clocks.stop()
+    ms_step = max_over_ranks(pg, total_ms / args.steps, dev)
+    pairs = w.nq * w.n
+    value = whole_job_value(pairs, world, ms_step)
+    # end to end: queries from pinned host memory in, top-k lists out (the
+    # index is the stored database and stays resident)
+    qh = q_host.pin_memory()
+    ih = torch.empty(idx.shape, dtype=torch.int32).pin_memory()
+    sh = torch.empty(sc.shape, dtype=torch.float32).pin_memory()
+    qd = torch.empty_like(q)
+
+    def pre():
+        qd.copy_(qh, non_blocking=True)
+
+    def post():
+        ih.copy_(idx, non_blocking=True)
+        sh.copy_(sc, non_blocking=True)
+
+    e2e_stage = [("tq_search_topk", lambda: tq.tq_search_topk(codec, qd, X, w.n, w.k, idx, sc, ws))]
+    time_steps(None, 1, stream, e2e_stage, pre, post)
+    e2e_steps = args.e2e_steps or args.steps
+    e2e_ms, _ = time_steps(None, e2e_steps, stream, e2e_stage, pre, post)
+    e2e_ms = max_over_ranks(pg, e2e_ms / e2e_steps, dev)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank != 0:
+        return 0
+    peak, peak_src = load_tensor_peak()
+    ms = statistics.mean(per["tq_search_topk"])
+    alg_flops = 2.0 * (w.d + w.m) * pairs          # the dequantised contraction
+    exec_flops = 3.0 * alg_flops                     # hi*hi + lo*hi + hi*lo
+    ach = alg_flops / (ms * 1e-3) / 1e12
+    line = {
+        "metric": SEARCH_METRIC, "value": value, "unit": "pairs/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16x3 (fp32 accumulate)", "data": "synthetic",
+        "config": {"workload": w.name, "n": w.n, "nq": w.nq, "d": w.d, "bits": list(w.bits), "m": w.m, "k": w.k,
+                   "parallelism": f"dp{world} (each rank searches its own copy)",
+                   "l2": "index 616 MB read per step, larger than L2"},
+        "queries_per_s": w.nq * world / (ms_step * 1e-3),
+        "roofline": {"kernel": "tq_search_topk", "bound": "tensor", "achieved": round(ach, 1), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(ach / peak, 4), "traffic": None, "peak_source": peak_src,
+                     "flops_per_launch": alg_flops, "executed_tensor_flops_per_launch": exec_flops},
+        "gpu_launches": args.steps * 5,
+        "e2e": {"value": whole_job_value(pairs, world, e2e_ms), "unit": "pairs/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": qh.numel() * 4, "d2h_bytes_per_step": ih.numel() * 4 + sh.numel() * 4},
+        "clocks": clocks.summary(t_wall0, t_wall1),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        pps, secs, npairs, threads, desc = cpu_search_sample(w, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": pps, "unit": "pairs/s", "cores": threads, "kind": "oracle", "sample": desc,
+                                "seconds": round(secs, 2)}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -326,6 +464,8 @@ def main():
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
         pg = dist
+    if args.workload == "vsearch":
+        return run_search(args, tq, dev, rank, world, pg)
     w = synth.WORKLOADS[args.workload]
     layer = Layer(tq, w, dev, rank)
     stream = torch.cuda.current_stream()

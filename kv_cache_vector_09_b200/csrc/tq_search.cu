@@ -19,7 +19,7 @@
 //   warp 8      B producer (bulk copies into a 4-stage ring)
 //   warp 9      MMA issue: 3 MMAs (M = 128, N = 256, K = 16) per group
 //   warps 10-13 epilogue: scores of the tile -> per-query top-k lists in
-//               shared memory (insertions under a per-query lock)
+//               shared memory (each query's list updated by one warp)
 // A final kernel merges the blocks' lists.  Every mbarrier wait is bounded.
 #include <math.h>
 
@@ -142,7 +142,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     search_kernel(const tq_params p, const SearchArgs a) {
   extern __shared__ __align__(1024) unsigned char smem[];
   __shared__ uint64_t a_full[kASlots], a_empty[kASlots], b_full[kBStages], b_empty[kBStages];
-  __shared__ uint64_t d_full, d_empty, drained;
+  __shared__ uint64_t d_full, d_empty, drained, epi_bar;
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_abort;
   __shared__ uint32_t s_cen[16];  // fp16 cen hi | lo << 16, by code
@@ -153,9 +153,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nq = a.nq, k = a.k;
 
   unsigned char* bring = smem;                                        // [kBStages][kGroupBytes]
-  float* tops = reinterpret_cast<float*>(smem + kBStages * kGroupBytes);  // [nq][k]
+  float* stg = reinterpret_cast<float*>(smem + kBStages * kGroupBytes);   // [32][kRowsT] score staging
+  float* s_qscale = stg + 32 * kRowsT;                                    // [nq]
+  float* tops = s_qscale + nq;                                            // [nq][k]
   int* tidx = reinterpret_cast<int*>(tops + (size_t)nq * k);              // [nq][k]
-  int* locks = tidx + (size_t)nq * k;                                     // [nq]
 
   const int64_t nkt = (a.n + kRowsT - 1) / kRowsT;
   const int64_t units = nkt * a.nqt;
@@ -166,7 +167,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tops[i] = -INFINITY;
     tidx[i] = 0x7FFFFFFF;
   }
-  for (int i = tid; i < nq; i += kThreads) locks[i] = 0;
+  for (int i = tid; i < nq; i += kThreads) s_qscale[i] = __ldg(a.qscale + i);
   if (tid < 16) {
     const float c = tid < (1 << BITS) ? p.cen[0][tid] : 0.f;
     const __half h = __float2half_rn(c);
@@ -184,6 +185,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tqtc::mbar_init(&d_full, 1);
     tqtc::mbar_init(&d_empty, 128);
     tqtc::mbar_init(&drained, 1);
+    tqtc::mbar_init(&epi_bar, 128);
     tqtc::fence_mbar_init();
     s_abort = 0;
   }
@@ -203,46 +205,101 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = 32u * (uint32_t)(warp & 3);
     const int rloc = 32 * (warp & 3) + lane;
     const float gk = p.qjl_coef * sqrtf((float)d) * kQjlGain;
-    for (int64_t ul = 0; ul < nul && !s_abort; ++ul) {
+    // emit one group: wait for its ring slot, store [hi | lo | hi], signal
+    auto emit = [&](int64_t x, const uint32_t (&hi)[8], const uint32_t (&lo)[8]) -> bool {
+      const int slot = (int)(x % kASlots);
+      if (x >= kASlots &&
+          !tqtc::mbar_wait_or_abort(&a_empty[slot], (uint32_t)((x / kASlots - 1) & 1), &s_abort)) {
+        fail(tqtc::kErrMmaWait);
+        return false;
+      }
+      tqtc::tc_fence_after();
+      const uint32_t col = 256u + 32u * (uint32_t)slot;
+      tqtc::tmem_st8(tqtc::tmem_addr(tbase, lane_base, col), hi);
+      tqtc::tmem_st8(tqtc::tmem_addr(tbase, lane_base, col + 8u), lo);
+      tqtc::tmem_st8(tqtc::tmem_addr(tbase, lane_base, col + 16u), hi);
+      tqtc::tmem_wait_st();
+      tqtc::tc_fence_before();
+      tqtc::mbar_arrive(&a_full[slot]);
+      return true;
+    };
+    // 16 codes (one 16-bit half of each plane word) -> centroid hi / lo pairs
+    auto decode16 = [&](const uint32_t (&pl)[BITS], uint32_t (&hi)[8], uint32_t (&lo)[8]) {
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        uint32_t y = 0u;  // byte r = 4 * code of coordinate 4 t + r
+#pragma unroll
+        for (int b = 0; b < BITS; ++b) y |= spread4((pl[b] >> (4 * t)) & 0xFu) << (b + 2);
+        uint32_t hl[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+          hl[r] = *reinterpret_cast<const uint32_t*>(reinterpret_cast<const char*>(s_cen) + ((y >> (8 * r)) & 0xFFu));
+        hi[2 * t] = prmt(hl[0], hl[1], 0x5410);
+        lo[2 * t] = prmt(hl[0], hl[1], 0x7632);
+        hi[2 * t + 1] = prmt(hl[2], hl[3], 0x5410);
+        lo[2 * t + 1] = prmt(hl[2], hl[3], 0x7632);
+      }
+    };
+    bool alive = true;
+    for (int64_t ul = 0; ul < nul && alive && !s_abort; ++ul) {
       const int64_t kt = (u0 + ul) / a.nqt;
       const int64_t row = kt * kRowsT + rloc;
       const bool valid = row < a.n;
       const uint32_t* crow = a.codes + (valid ? row : 0) * W;
       const uint32_t* srow = a.signs + (valid ? row : 0) * MS;
-      uint32_t ghi2 = 0u, glo2 = 0u;
-      if (m > 0) {
-        const float g = valid ? __ldg(a.rnorms + row) * gk : 0.f;
-        const __half h = __float2half_rn(g);
-        const uint32_t hb = __half_as_ushort(h), lb = half_bits(g - __half2float(h));
-        ghi2 = hb | (hb << 16);
-        glo2 = lb | (lb << 16);
-      }
-      for (int g = set; g < ngroups; g += 2) {
-        const int64_t x = ul * ngroups + g;
-        const int slot = (int)(x % kASlots);
-        uint32_t hi[8], lo[8];
-        if (g < gc) {
-          const int w = g >> 1, sh = 16 * (g & 1);
+      const int64_t x0 = ul * ngroups;
+      const int sh = 16 * set;  // groups of this set take this half of every word
+      if (PW % 4 == 0) {
+        // coordinate groups in blocks of four words per plane (one 16-byte
+        // load each), the next block loaded while this one is built
+        uint4 cur[BITS], nxt[BITS];
+#pragma unroll
+        for (int b = 0; b < BITS; ++b)
+          cur[b] = valid ? __ldg(reinterpret_cast<const uint4*>(crow + b * PW)) : make_uint4(0u, 0u, 0u, 0u);
+        for (int blk = 0; blk < PW / 4 && alive; ++blk) {
+          if (blk + 1 < PW / 4) {
+#pragma unroll
+            for (int b = 0; b < BITS; ++b)
+              nxt[b] = valid ? __ldg(reinterpret_cast<const uint4*>(crow + b * PW + 4 * blk + 4))
+                             : make_uint4(0u, 0u, 0u, 0u);
+          }
+#pragma unroll
+          for (int ww = 0; ww < 4; ++ww) {
+            uint32_t pl[BITS];
+#pragma unroll
+            for (int b = 0; b < BITS; ++b) {
+              const uint32_t v = ww == 0 ? cur[b].x : ww == 1 ? cur[b].y : ww == 2 ? cur[b].z : cur[b].w;
+              pl[b] = v >> sh;
+            }
+            uint32_t hi[8], lo[8];
+            decode16(pl, hi, lo);
+            if (!emit(x0 + 2 * (4 * blk + ww) + set, hi, lo)) {
+              alive = false;
+              break;
+            }
+          }
+#pragma unroll
+          for (int b = 0; b < BITS; ++b) cur[b] = nxt[b];
+        }
+      } else {
+        for (int g = set; g < gc && alive; g += 2) {
           uint32_t pl[BITS];
 #pragma unroll
-          for (int b = 0; b < BITS; ++b) pl[b] = valid ? (__ldg(crow + b * PW + w) >> sh) : 0u;
-#pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            uint32_t y = 0u;  // byte r = 4 * code of coordinate 16 g + 4 t + r
-#pragma unroll
-            for (int b = 0; b < BITS; ++b) y |= spread4((pl[b] >> (4 * t)) & 0xFu) << (b + 2);
-            uint32_t hl[4];
-#pragma unroll
-            for (int r = 0; r < 4; ++r)
-              hl[r] = *reinterpret_cast<const uint32_t*>(reinterpret_cast<const char*>(s_cen) + ((y >> (8 * r)) & 0xFFu));
-            hi[2 * t] = prmt(hl[0], hl[1], 0x5410);
-            lo[2 * t] = prmt(hl[0], hl[1], 0x7632);
-            hi[2 * t + 1] = prmt(hl[2], hl[3], 0x5410);
-            lo[2 * t + 1] = prmt(hl[2], hl[3], 0x7632);
-          }
-        } else {
-          const int j0 = 16 * (g - gc);
-          const uint32_t bits = valid ? (__ldg(srow + (j0 >> 5)) >> (j0 & 16)) : 0xFFFFu;
+          for (int b = 0; b < BITS; ++b) pl[b] = valid ? (__ldg(crow + b * PW + (g >> 1)) >> sh) : 0u;
+          uint32_t hi[8], lo[8];
+          decode16(pl, hi, lo);
+          alive = emit(x0 + g, hi, lo);
+        }
+      }
+      if (m > 0 && alive) {
+        const float gv = valid ? __ldg(a.rnorms + row) * gk : 0.f;
+        const __half h = __float2half_rn(gv);
+        const uint32_t hb = __half_as_ushort(h), lb = half_bits(gv - __half2float(h));
+        const uint32_t ghi2 = hb | (hb << 16), glo2 = lb | (lb << 16);
+        // sketch groups of this set: this half of every sign word
+        for (int u = 0; u < MS && alive; ++u) {
+          const uint32_t bits = valid ? (__ldg(srow + u) >> sh) : 0xFFFFu;
+          uint32_t hi[8], lo[8];
 #pragma unroll
           for (int pp = 0; pp < 8; ++pp) {
             // sign bit 0 -> negative: flip the fp16 sign bits
@@ -251,20 +308,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             hi[pp] = ghi2 ^ mask;
             lo[pp] = glo2 ^ mask;
           }
+          alive = emit(x0 + gc + 2 * u + set, hi, lo);
         }
-        if (x >= kASlots &&
-            !tqtc::mbar_wait_or_abort(&a_empty[slot], (uint32_t)((x / kASlots - 1) & 1), &s_abort)) {
-          fail(tqtc::kErrMmaWait);
-          break;
-        }
-        tqtc::tc_fence_after();
-        const uint32_t col = 256u + 32u * (uint32_t)slot;
-        tqtc::tmem_st8(tqtc::tmem_addr(tbase, lane_base, col), hi);
-        tqtc::tmem_st8(tqtc::tmem_addr(tbase, lane_base, col + 8u), lo);
-        tqtc::tmem_st8(tqtc::tmem_addr(tbase, lane_base, col + 16u), hi);
-        tqtc::tmem_wait_st();
-        tqtc::tc_fence_before();
-        tqtc::mbar_arrive(&a_full[slot]);
       }
     }
   } else if (warp == 8) {
@@ -331,10 +376,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------------------------------------------------- epilogue
+    // Per 32-column chunk of the accumulator: every thread (one index row)
+    // scales its 32 scores into the staging tile, then each warp owns 8 of
+    // the chunk's queries and updates their lists alone: few candidates are
+    // inserted one by one, many are merged by k rounds of a warp argmax.
     const uint32_t quarter = (uint32_t)(warp & 3);
+    const int ew = warp - 10;  // 0..3
     const int rloc = 32 * (int)quarter + lane;
     const float inv_sqrt_d = p.inv_sqrt_d;
-    for (int64_t ul = 0; ul < nul; ++ul) {
+    // bounded barrier of the four epilogue warps (an mbarrier phase each)
+    uint32_t ephase = 0u;
+    auto epi_sync = [&]() -> bool {
+      tqtc::mbar_arrive(&epi_bar);
+      const bool ok = tqtc::mbar_wait_or_abort(&epi_bar, ephase, &s_abort);
+      ephase ^= 1u;
+      if (!ok) fail(tqtc::kErrMmaWait);
+      return ok;
+    };
+    bool alive = true;
+    for (int64_t ul = 0; ul < nul && alive; ++ul) {
       const int64_t kt = (u0 + ul) / a.nqt, qt = (u0 + ul) % a.nqt;
       const int64_t row = kt * kRowsT + rloc;
       const bool valid = row < a.n;
@@ -344,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tqtc::tc_fence_after();
-      for (int c = 0; c < kQT / 32; ++c) {
+      for (int c = 0; c < kQT / 32 && alive; ++c) {
         uint32_t dv[32];
         tqtc::tmem_ld16(tqtc::tmem_addr(tbase, 32u * quarter, 32u * c), *reinterpret_cast<uint32_t(*)[16]>(dv));
         tqtc::tmem_ld16(tqtc::tmem_addr(tbase, 32u * quarter, 32u * c + 16u),
@@ -358,42 +418,100 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           const int qi = qbase + j;
+          const float sc = qi < nq ? s_qscale[qi] : 0.f;
+          stg[j * kRowsT + rloc] = valid ? __uint_as_float(dv[j]) * rs * sc : -INFINITY;
+        }
+        if (!(alive = epi_sync())) break;
+        for (int jj = 0; jj < 8; ++jj) {
+          const int j = ew * 8 + jj, qi = qbase + j;
           if (qi >= nq) continue;
-          const float s = __uint_as_float(dv[j]) * rs * __ldg(a.qscale + qi);
           float* tq = tops + (size_t)qi * k;
           int* ti = tidx + (size_t)qi * k;
-          const volatile float* vtq = tq;
-          const volatile int* vti = ti;
-          bool cand = valid && better(s, (int)row, vtq[k - 1], vti[k - 1]);
-          unsigned mask = __ballot_sync(0xFFFFFFFFu, cand);
-          while (mask) {
-            const int leader = __ffs(mask) - 1;
-            if (lane == leader) {
-              bool done = false;
-              for (int spin = 0; spin < (1 << 22) && !done; ++spin) {
-                if (atomicCAS(&locks[qi], 0, 1) == 0) {
-                  __threadfence_block();
-                  if (better(s, (int)row, vtq[k - 1], vti[k - 1])) {
-                    int pos = k - 1;
-                    while (pos > 0 && better(s, (int)row, vtq[pos - 1], vti[pos - 1])) {
-                      tq[pos] = vtq[pos - 1];
-                      ti[pos] = vti[pos - 1];
-                      --pos;
-                    }
-                    tq[pos] = s;
-                    ti[pos] = (int)row;
+          const float ths = tq[k - 1];
+          const int thr = ti[k - 1];
+          float v[4];
+          int r[4];
+          unsigned cm = 0u;  // candidate bits of this lane
+          int cnt = 0;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            v[i] = stg[j * kRowsT + lane + 32 * i];
+            r[i] = (int)(kt * kRowsT) + lane + 32 * i;
+            const bool cand = r[i] < a.n && better(v[i], r[i], ths, thr);
+            cm |= (cand ? 1u : 0u) << i;
+            cnt += __popc(__ballot_sync(0xFFFFFFFFu, cand));
+          }
+          if (cnt == 0) continue;
+          if (cnt <= 4) {
+            // one by one, in lane order
+            for (int i = 0; i < 4; ++i) {
+              unsigned mask = __ballot_sync(0xFFFFFFFFu, (cm >> i) & 1u);
+              while (mask) {
+                const int leader = __ffs(mask) - 1;
+                if (lane == leader && better(v[i], r[i], tq[k - 1], ti[k - 1])) {
+                  int pos = k - 1;
+                  while (pos > 0 && better(v[i], r[i], tq[pos - 1], ti[pos - 1])) {
+                    tq[pos] = tq[pos - 1];
+                    ti[pos] = ti[pos - 1];
+                    --pos;
                   }
-                  __threadfence_block();
-                  atomicExch(&locks[qi], 0);
-                  done = true;
+                  tq[pos] = v[i];
+                  ti[pos] = r[i];
+                }
+                mask &= mask - 1;
+                __syncwarp();
+              }
+            }
+          } else {
+            // merge: lanes < k hold the current list; k rounds of a warp argmax
+            float ls = lane < k ? tq[lane] : -INFINITY;
+            int lr = lane < k ? ti[lane] : 0x7FFFFFFF;
+            bool lused = lane >= k;
+            float outs = -INFINITY;
+            int outr = 0x7FFFFFFF;
+            for (int rnd = 0; rnd < k; ++rnd) {
+              float bs = -INFINITY;
+              int br = 0x7FFFFFFF;
+              if (!lused && better(ls, lr, bs, br)) {
+                bs = ls;
+                br = lr;
+              }
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                if (((cm >> i) & 1u) && better(v[i], r[i], bs, br)) {
+                  bs = v[i];
+                  br = r[i];
+                }
+              float ws = bs;
+              int wr = br;
+#pragma unroll
+              for (int o = 16; o > 0; o >>= 1) {
+                const float os = __shfl_xor_sync(0xFFFFFFFFu, ws, o);
+                const int orr = __shfl_xor_sync(0xFFFFFFFFu, wr, o);
+                if (better(os, orr, ws, wr)) {
+                  ws = os;
+                  wr = orr;
                 }
               }
-              if (!done) fail(tqtc::kErrMmaWait);
+              if (lane == rnd) {
+                outs = ws;
+                outr = wr;
+              }
+              // the owner retires the winner (rows are distinct)
+              if (!lused && lr == wr) lused = true;
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                if (((cm >> i) & 1u) && r[i] == wr) cm &= ~(1u << i);
             }
-            mask &= mask - 1;
+            __syncwarp();
+            if (lane < k) {
+              tq[lane] = outs;
+              ti[lane] = outr;
+            }
             __syncwarp();
           }
         }
+        alive = epi_sync();
       }
     }
   }
@@ -523,7 +641,7 @@ cudaError_t tq_launch_search(const tq_params& p, const float* qprep, int nq, int
   a.qscale = qscale;
   a.part_s = part_s;
   a.part_i = part_i;
-  size_t smem = (size_t)kBStages * kGroupBytes + (size_t)nb * k * 8 + (size_t)nb * 4;
+  size_t smem = (size_t)kBStages * kGroupBytes + 32 * kRowsT * 4 + (size_t)nb * 4 + (size_t)nb * k * 8;
   // the block takes all 512 TMEM columns: ask for more than half of the SM's
   // shared memory so that a second block never waits on the allocation
   {
