@@ -8,17 +8,17 @@
 // are split into fp16 hi + lo parts and three products per element are
 // accumulated (hi*hi + lo*hi + hi*lo; the omitted lo*lo is below 2^-22 of
 // the term), in K groups of 16 elements:
-//   group of 16 coordinates:  A = [cen_hi | cen_lo | cen_hi],  B = [q_hi | q_hi | q_lo]
-//   group of 16 sketch rows:  A = [g_hi s | g_lo s | g_hi s],  B = [w_hi | w_hi | w_lo]
+//   group of 16 coordinates:  A = [cen_hi | cen_lo],  B = [q_hi | q_lo]
+//   group of 16 sketch rows:  A = [g_hi s | g_lo s],  B = [w_hi | w_lo]
+// and the three MMAs of a group pair (A_hi, B_hi), (A_lo, B_hi), (A_hi, B_lo)
 // with B scaled per query by 2^e (w by 2^(e-6), g by 2^6) to keep the fp16
 // parts normal.  A is built per 128-row tile by CUDA-core warps straight
 // into TMEM (codes -> centroid hi/lo pairs), B is a per-query image built
 // once per call and streamed from L2 by bulk copies.  One block per SM:
-//   warps 0-7   A builders (warps 0-3 even groups, 4-7 odd groups; warp w
-//               writes TMEM lanes 32 (w % 4) ..)
-//   warp 8      B producer (bulk copies into a 4-stage ring)
-//   warp 9      MMA issue: 3 MMAs (M = 128, N = 256, K = 16) per group
-//   warps 10-13 epilogue: scores of the tile -> per-query top-k lists in
+//   warps 0-3   A builders (warp w writes TMEM lanes 32 w ..)
+//   warp 4      B producer (bulk copies into a 4-stage ring)
+//   warp 5      MMA issue: 3 MMAs (M = 128, N = 256, K = 16) per group
+//   warps 6-13  epilogue: scores of the tile -> per-query top-k lists in
 //               shared memory (each query's list updated by one warp)
 // A final kernel merges the blocks' lists.  Every mbarrier wait is bounded.
 #include <math.h>
@@ -34,9 +34,10 @@ namespace {
 constexpr int kRowsT = 128;                // index rows per tile (MMA M)
 constexpr int kQT = 256;                   // queries per tile (MMA N)
 constexpr int kStepBytes = kQT * 16 * 2;   // one K = 16 step of B: 8 KB
-constexpr int kGroupBytes = 3 * kStepBytes;
+constexpr int kGroupBytes = 2 * kStepBytes;  // [hi | lo]
 constexpr int kBStages = 4;
-constexpr int kASlots = 8;                 // TMEM A ring, 32 columns per slot
+constexpr int kCandCap = 2048;             // candidate buffer of the epilogue (entries)
+constexpr int kASlots = 16;                // TMEM A ring, 16 columns per slot ([hi | lo])
 constexpr int kThreads = 448;
 constexpr float kQjlGain = 64.f;           // 2^6 on the A side of the sketch groups
 
@@ -73,7 +74,7 @@ __global__ void __launch_bounds__(256) search_qexp_kernel(const float* __restric
   }
 }
 
-// B image: [query tile][group][step][8 KB], one thread per (query, group).
+// B image: [query tile][group][hi, lo][8 KB], one thread per (query, group).
 // Within a step: element (n, kk) at (kk / 8) * 4096 + (n / 8) * 128 + (n % 8) * 16 + (kk % 8) * 2.
 __global__ void __launch_bounds__(256) search_bimg_kernel(const float* __restrict__ qprep, const int* __restrict__ qexp,
                                                           int nq, int nqt, int d, int m, uint8_t* __restrict__ img) {
@@ -110,9 +111,9 @@ __global__ void __launch_bounds__(256) search_bimg_kernel(const float* __restric
   }
   uint8_t* gbase = img + ((size_t)qt * ngroups + g) * kGroupBytes;
   const uint32_t off = (uint32_t)(n / 8) * 128u + (uint32_t)(n % 8) * 16u;
-  const uint32_t* parts[3] = {hi, hi, lo};
+  const uint32_t* parts[2] = {hi, lo};
 #pragma unroll
-  for (int s = 0; s < 3; ++s) {
+  for (int s = 0; s < 2; ++s) {
     const uint32_t* v = parts[s];
     *reinterpret_cast<uint4*>(gbase + s * kStepBytes + off) = make_uint4(v[0], v[1], v[2], v[3]);
     *reinterpret_cast<uint4*>(gbase + s * kStepBytes + 4096 + off) = make_uint4(v[4], v[5], v[6], v[7]);
@@ -143,6 +144,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ __align__(1024) unsigned char smem[];
   __shared__ uint64_t a_full[kASlots], a_empty[kASlots], b_full[kBStages], b_empty[kBStages];
   __shared__ uint64_t d_full, d_empty, drained, epi_bar;
+  __shared__ int s_ncand[2];
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_abort;
   __shared__ uint32_t s_cen[16];  // fp16 cen hi | lo << 16, by code
@@ -153,8 +155,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nq = a.nq, k = a.k;
 
   unsigned char* bring = smem;                                        // [kBStages][kGroupBytes]
-  float* stg = reinterpret_cast<float*>(smem + kBStages * kGroupBytes);   // [32][kRowsT] score staging
-  float* s_qscale = stg + 32 * kRowsT;                                    // [nq]
+  float* stg = reinterpret_cast<float*>(smem + kBStages * kGroupBytes);   // [2][32][kRowsT] score staging
+  int* cand_q = reinterpret_cast<int*>(stg + 2 * 32 * kRowsT);           // [kCandCap] candidates: query,
+  int* cand_r = cand_q + kCandCap;                                        //   row,
+  float* cand_s = reinterpret_cast<float*>(cand_r + kCandCap);            //   score
+  float* s_qscale = cand_s + kCandCap;                                    // [nq]
   float* tops = s_qscale + nq;                                            // [nq][k]
   int* tidx = reinterpret_cast<int*>(tops + (size_t)nq * k);              // [nq][k]
 
@@ -183,11 +188,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       tqtc::mbar_init(&b_empty[i], 1);
     }
     tqtc::mbar_init(&d_full, 1);
-    tqtc::mbar_init(&d_empty, 128);
+    tqtc::mbar_init(&d_empty, 256);
     tqtc::mbar_init(&drained, 1);
-    tqtc::mbar_init(&epi_bar, 128);
+    tqtc::mbar_init(&epi_bar, 256);
     tqtc::fence_mbar_init();
     s_abort = 0;
+    s_ncand[0] = s_ncand[1] = 0;
   }
   if (warp == 0) tqtc::tmem_alloc(&s_tmem, 512);
   tqtc::tc_fence_before();
@@ -199,29 +205,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     s_abort = 1;
   };
 
-  if (warp < 8) {
+  if (warp < 4) {
     // ---------------------------------------------------------- A builders
-    const int set = warp >> 2;
-    const uint32_t lane_base = 32u * (uint32_t)(warp & 3);
-    const int rloc = 32 * (warp & 3) + lane;
+    const uint32_t lane_base = 32u * (uint32_t)warp;
+    const int rloc = 32 * warp + lane;
     const float gk = p.qjl_coef * sqrtf((float)d) * kQjlGain;
-    // emit one group: wait for its ring slot, store [hi | lo | hi], signal
-    auto emit = [&](int64_t x, const uint32_t (&hi)[8], const uint32_t (&lo)[8]) -> bool {
+    // put one group into its ring slot (after the slot's previous MMAs are
+    // done); groups are signalled in batches: one wait for the stores, then
+    // an arrival per slot
+    auto put = [&](int64_t x, const uint32_t (&hi)[8], const uint32_t (&lo)[8]) -> bool {
       const int slot = (int)(x % kASlots);
       if (x >= kASlots &&
-          !tqtc::mbar_wait_or_abort(&a_empty[slot], (uint32_t)((x / kASlots - 1) & 1), &s_abort)) {
+          !tqtc::mbar_wait_sleep_or_abort(&a_empty[slot], (uint32_t)((x / kASlots - 1) & 1), &s_abort, 128)) {
         fail(tqtc::kErrMmaWait);
         return false;
       }
       tqtc::tc_fence_after();
-      const uint32_t col = 256u + 32u * (uint32_t)slot;
+      const uint32_t col = 256u + 16u * (uint32_t)slot;
       tqtc::tmem_st8(tqtc::tmem_addr(tbase, lane_base, col), hi);
       tqtc::tmem_st8(tqtc::tmem_addr(tbase, lane_base, col + 8u), lo);
-      tqtc::tmem_st8(tqtc::tmem_addr(tbase, lane_base, col + 16u), hi);
+      return true;
+    };
+    // signal groups x0 .. x0 + cnt - 1
+    auto signal = [&](int64_t x0, int cnt) {
       tqtc::tmem_wait_st();
       tqtc::tc_fence_before();
-      tqtc::mbar_arrive(&a_full[slot]);
-      return true;
+      for (int i = 0; i < cnt; ++i) tqtc::mbar_arrive(&a_full[(int)((x0 + i) % kASlots)]);
     };
     // 16 codes (one 16-bit half of each plane word) -> centroid hi / lo pairs
     auto decode16 = [&](const uint32_t (&pl)[BITS], uint32_t (&hi)[8], uint32_t (&lo)[8]) {
@@ -248,10 +257,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t* crow = a.codes + (valid ? row : 0) * W;
       const uint32_t* srow = a.signs + (valid ? row : 0) * MS;
       const int64_t x0 = ul * ngroups;
-      const int sh = 16 * set;  // groups of this set take this half of every word
       if (PW % 4 == 0) {
         // coordinate groups in blocks of four words per plane (one 16-byte
-        // load each), the next block loaded while this one is built
+        // load each, eight groups), the next block loaded while this one is
+        // built
         uint4 cur[BITS], nxt[BITS];
 #pragma unroll
         for (int b = 0; b < BITS; ++b)
@@ -265,30 +274,32 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
 #pragma unroll
           for (int ww = 0; ww < 4; ++ww) {
-            uint32_t pl[BITS];
 #pragma unroll
-            for (int b = 0; b < BITS; ++b) {
-              const uint32_t v = ww == 0 ? cur[b].x : ww == 1 ? cur[b].y : ww == 2 ? cur[b].z : cur[b].w;
-              pl[b] = v >> sh;
-            }
-            uint32_t hi[8], lo[8];
-            decode16(pl, hi, lo);
-            if (!emit(x0 + 2 * (4 * blk + ww) + set, hi, lo)) {
-              alive = false;
-              break;
+            for (int hh = 0; hh < 2; ++hh) {
+              uint32_t pl[BITS];
+#pragma unroll
+              for (int b = 0; b < BITS; ++b) {
+                const uint32_t v = ww == 0 ? cur[b].x : ww == 1 ? cur[b].y : ww == 2 ? cur[b].z : cur[b].w;
+                pl[b] = v >> (16 * hh);
+              }
+              uint32_t hi[8], lo[8];
+              decode16(pl, hi, lo);
+              if (alive && !put(x0 + 2 * (4 * blk + ww) + hh, hi, lo)) alive = false;
             }
           }
+          if (!alive) break;
+          signal(x0 + 8 * blk, 8);
 #pragma unroll
           for (int b = 0; b < BITS; ++b) cur[b] = nxt[b];
         }
       } else {
-        for (int g = set; g < gc && alive; g += 2) {
+        for (int g = 0; g < gc && alive; ++g) {
           uint32_t pl[BITS];
 #pragma unroll
-          for (int b = 0; b < BITS; ++b) pl[b] = valid ? (__ldg(crow + b * PW + (g >> 1)) >> sh) : 0u;
+          for (int b = 0; b < BITS; ++b) pl[b] = valid ? (__ldg(crow + b * PW + (g >> 1)) >> (16 * (g & 1))) : 0u;
           uint32_t hi[8], lo[8];
           decode16(pl, hi, lo);
-          alive = emit(x0 + g, hi, lo);
+          if ((alive = put(x0 + g, hi, lo))) signal(x0 + g, 1);
         }
       }
       if (m > 0 && alive) {
@@ -296,9 +307,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const __half h = __float2half_rn(gv);
         const uint32_t hb = __half_as_ushort(h), lb = half_bits(gv - __half2float(h));
         const uint32_t ghi2 = hb | (hb << 16), glo2 = lb | (lb << 16);
-        // sketch groups of this set: this half of every sign word
-        for (int u = 0; u < MS && alive; ++u) {
-          const uint32_t bits = valid ? (__ldg(srow + u) >> sh) : 0xFFFFu;
+        // sketch groups: the two halves of every sign word
+        int pending = 0;
+        for (int g = 0; g < 2 * MS && alive; ++g) {
+          const uint32_t bits = valid ? (__ldg(srow + (g >> 1)) >> (16 * (g & 1))) : 0xFFFFu;
           uint32_t hi[8], lo[8];
 #pragma unroll
           for (int pp = 0; pp < 8; ++pp) {
@@ -308,11 +320,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             hi[pp] = ghi2 ^ mask;
             lo[pp] = glo2 ^ mask;
           }
-          alive = emit(x0 + gc + 2 * u + set, hi, lo);
+          alive = put(x0 + gc + g, hi, lo);
+          if (alive && (++pending == 8 || g == 2 * MS - 1)) {
+            signal(x0 + gc + g + 1 - pending, pending);
+            pending = 0;
+          }
         }
       }
     }
-  } else if (warp == 8) {
+  } else if (warp == 4) {
     // ---------------------------------------------------------- B producer
     if (lane == 0) {
       int64_t issued = 0;
@@ -323,7 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int64_t x = ul * ngroups + g;
           const int st = (int)(x % kBStages);
           if (x >= kBStages &&
-              !tqtc::mbar_wait_or_abort(&b_empty[st], (uint32_t)((x / kBStages - 1) & 1), &s_abort)) {
+              !tqtc::mbar_wait_sleep_or_abort(&b_empty[st], (uint32_t)((x / kBStages - 1) & 1), &s_abort, 64)) {
             fail(tqtc::kErrCopyWait);
             break;
           }
@@ -338,7 +354,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!tqtc::mbar_wait_or_abort(&b_full[x % kBStages], (uint32_t)((x / kBStages) & 1), nullptr))
           atomicExch(p.err, tqtc::kErrCopyWait);
     }
-  } else if (warp == 9) {
+  } else if (warp == 5) {
     // ---------------------------------------------------------- MMA issue
     if (lane == 0) {
       const uint32_t idesc = tqtc::instr_desc(1, 0, 0, kRowsT, kQT);
@@ -359,12 +375,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tqtc::tc_fence_after();
-          const uint32_t acol = tbase + 256u + 32u * (uint32_t)slot;
+          const uint32_t acol = tbase + 256u + 16u * (uint32_t)slot;
           const uint32_t b0 = bbase + (uint32_t)st * kGroupBytes;
-#pragma unroll
-          for (int s = 0; s < 3; ++s)
-            tqtc::mma_f16_ts(tbase, acol + 8u * (uint32_t)s,
-                             tqtc::smem_desc(b0 + (uint32_t)s * kStepBytes, 4096u, 128u), idesc, g > 0 || s > 0);
+          const uint64_t bhi = tqtc::smem_desc(b0, 4096u, 128u), blo = tqtc::smem_desc(b0 + kStepBytes, 4096u, 128u);
+          tqtc::mma_f16_ts(tbase, acol, bhi, idesc, g > 0);       // A_hi B_hi
+          tqtc::mma_f16_ts(tbase, acol + 8u, bhi, idesc, true);   // A_lo B_hi
+          tqtc::mma_f16_ts(tbase, acol, blo, idesc, true);        // A_hi B_lo
           tqtc::mma_commit(&a_empty[slot]);
           tqtc::mma_commit(&b_empty[st]);
         }
@@ -376,15 +392,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------------------------------------------------- epilogue
-    // Per 32-column chunk of the accumulator: every thread (one index row)
-    // scales its 32 scores into the staging tile, then each warp owns 8 of
-    // the chunk's queries and updates their lists alone: few candidates are
-    // inserted one by one, many are merged by k rounds of a warp argmax.
+    // Eight warps: warp e reads TMEM lanes 32 (warp % 4) .. of accumulator
+    // columns [128 h, 128 h + 128), h = e / 4.  Per tile, a filter pass reads
+    // the warp's four 32-column chunks, compares every score with its
+    // query's current k-th best and appends the rare candidates to a shared
+    // buffer; the accumulator is released as soon as every chunk is read.
+    // The owner warp of each query (column j of a chunk -> warp j / 4) then
+    // inserts that query's candidates.  A tile with more candidates than the
+    // buffer holds (the first tile of every query tile, whose lists are
+    // still empty) takes the staging path: scores staged in shared memory a
+    // chunk per half at a time, owner warps (column j -> warp 4 h + j / 8)
+    // updating their queries (few candidates in order, many by k rounds of a
+    // warp argmax), the accumulator released after the last chunk.
     const uint32_t quarter = (uint32_t)(warp & 3);
-    const int ew = warp - 10;  // 0..3
+    const int e8 = warp - 6;  // 0..7
+    const int half = e8 >> 2;
     const int rloc = 32 * (int)quarter + lane;
     const float inv_sqrt_d = p.inv_sqrt_d;
-    // bounded barrier of the four epilogue warps (an mbarrier phase each)
+    // bounded barrier of the eight epilogue warps (an mbarrier phase each)
     uint32_t ephase = 0u;
     auto epi_sync = [&]() -> bool {
       tqtc::mbar_arrive(&epi_bar);
@@ -393,126 +418,192 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) fail(tqtc::kErrMmaWait);
       return ok;
     };
+    // insert (s, r) into query qi's list (one lane; the caller owns qi)
+    auto insert1 = [&](int qi, float sv, int rv) {
+      float* tq = tops + (size_t)qi * k;
+      int* ti = tidx + (size_t)qi * k;
+      if (!better(sv, rv, tq[k - 1], ti[k - 1])) return;
+      int pos = k - 1;
+      while (pos > 0 && better(sv, rv, tq[pos - 1], ti[pos - 1])) {
+        tq[pos] = tq[pos - 1];
+        ti[pos] = ti[pos - 1];
+        --pos;
+      }
+      tq[pos] = sv;
+      ti[pos] = rv;
+    };
+    auto load_chunk = [&](int c, uint32_t (&dv)[32]) {
+      tqtc::tmem_ld16(tqtc::tmem_addr(tbase, 32u * quarter, 32u * c), *reinterpret_cast<uint32_t(*)[16]>(dv));
+      tqtc::tmem_ld16(tqtc::tmem_addr(tbase, 32u * quarter, 32u * c + 16u),
+                      *reinterpret_cast<uint32_t(*)[16]>(dv + 16));
+      tqtc::tmem_wait_ld();
+    };
+    auto release_d = [&]() {
+      tqtc::tc_fence_before();
+      tqtc::mbar_arrive(&d_empty);
+    };
     bool alive = true;
     for (int64_t ul = 0; ul < nul && alive; ++ul) {
       const int64_t kt = (u0 + ul) / a.nqt, qt = (u0 + ul) % a.nqt;
       const int64_t row = kt * kRowsT + rloc;
       const bool valid = row < a.n;
       const float rs = valid ? __ldg(a.norms + row) * inv_sqrt_d : 0.f;
+      int* ncand = &s_ncand[ul & 1];
       if (!tqtc::mbar_wait_or_abort(&d_full, (uint32_t)(ul & 1), &s_abort)) {
         fail(tqtc::kErrMmaWait);
         break;
       }
       tqtc::tc_fence_after();
-      for (int c = 0; c < kQT / 32 && alive; ++c) {
+      // ---- filter pass over this warp's four chunks
+      for (int cc = 0; cc < 4; ++cc) {
+        const int c = 4 * half + cc;
         uint32_t dv[32];
-        tqtc::tmem_ld16(tqtc::tmem_addr(tbase, 32u * quarter, 32u * c), *reinterpret_cast<uint32_t(*)[16]>(dv));
-        tqtc::tmem_ld16(tqtc::tmem_addr(tbase, 32u * quarter, 32u * c + 16u),
-                        *reinterpret_cast<uint32_t(*)[16]>(dv + 16));
-        tqtc::tmem_wait_ld();
-        if (c == kQT / 32 - 1) {
-          tqtc::tc_fence_before();
-          tqtc::mbar_arrive(&d_empty);
-        }
+        load_chunk(c, dv);
         const int qbase = (int)qt * kQT + 32 * c;
+        // candidate mask first (loads only), then the rare writes
+        uint32_t cmask = 0u;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           const int qi = qbase + j;
-          const float sc = qi < nq ? s_qscale[qi] : 0.f;
-          stg[j * kRowsT + rloc] = valid ? __uint_as_float(dv[j]) * rs * sc : -INFINITY;
-        }
-        if (!(alive = epi_sync())) break;
-        for (int jj = 0; jj < 8; ++jj) {
-          const int j = ew * 8 + jj, qi = qbase + j;
-          if (qi >= nq) continue;
-          float* tq = tops + (size_t)qi * k;
-          int* ti = tidx + (size_t)qi * k;
-          const float ths = tq[k - 1];
-          const int thr = ti[k - 1];
-          float v[4];
-          int r[4];
-          unsigned cm = 0u;  // candidate bits of this lane
-          int cnt = 0;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            v[i] = stg[j * kRowsT + lane + 32 * i];
-            r[i] = (int)(kt * kRowsT) + lane + 32 * i;
-            const bool cand = r[i] < a.n && better(v[i], r[i], ths, thr);
-            cm |= (cand ? 1u : 0u) << i;
-            cnt += __popc(__ballot_sync(0xFFFFFFFFu, cand));
-          }
-          if (cnt == 0) continue;
-          if (cnt <= 4) {
-            // one by one, in lane order
-            for (int i = 0; i < 4; ++i) {
-              unsigned mask = __ballot_sync(0xFFFFFFFFu, (cm >> i) & 1u);
-              while (mask) {
-                const int leader = __ffs(mask) - 1;
-                if (lane == leader && better(v[i], r[i], tq[k - 1], ti[k - 1])) {
-                  int pos = k - 1;
-                  while (pos > 0 && better(v[i], r[i], tq[pos - 1], ti[pos - 1])) {
-                    tq[pos] = tq[pos - 1];
-                    ti[pos] = ti[pos - 1];
-                    --pos;
-                  }
-                  tq[pos] = v[i];
-                  ti[pos] = r[i];
-                }
-                mask &= mask - 1;
-                __syncwarp();
-              }
-            }
-          } else {
-            // merge: lanes < k hold the current list; k rounds of a warp argmax
-            float ls = lane < k ? tq[lane] : -INFINITY;
-            int lr = lane < k ? ti[lane] : 0x7FFFFFFF;
-            bool lused = lane >= k;
-            float outs = -INFINITY;
-            int outr = 0x7FFFFFFF;
-            for (int rnd = 0; rnd < k; ++rnd) {
-              float bs = -INFINITY;
-              int br = 0x7FFFFFFF;
-              if (!lused && better(ls, lr, bs, br)) {
-                bs = ls;
-                br = lr;
-              }
-#pragma unroll
-              for (int i = 0; i < 4; ++i)
-                if (((cm >> i) & 1u) && better(v[i], r[i], bs, br)) {
-                  bs = v[i];
-                  br = r[i];
-                }
-              float ws = bs;
-              int wr = br;
-#pragma unroll
-              for (int o = 16; o > 0; o >>= 1) {
-                const float os = __shfl_xor_sync(0xFFFFFFFFu, ws, o);
-                const int orr = __shfl_xor_sync(0xFFFFFFFFu, wr, o);
-                if (better(os, orr, ws, wr)) {
-                  ws = os;
-                  wr = orr;
-                }
-              }
-              if (lane == rnd) {
-                outs = ws;
-                outr = wr;
-              }
-              // the owner retires the winner (rows are distinct)
-              if (!lused && lr == wr) lused = true;
-#pragma unroll
-              for (int i = 0; i < 4; ++i)
-                if (((cm >> i) & 1u) && r[i] == wr) cm &= ~(1u << i);
-            }
-            __syncwarp();
-            if (lane < k) {
-              tq[lane] = outs;
-              ti[lane] = outr;
-            }
-            __syncwarp();
+          if (qi < nq) {
+            const float sv = __uint_as_float(dv[j]) * rs * s_qscale[qi];
+            dv[j] = __float_as_uint(sv);
+            const bool cnd = better(sv, (int)row, tops[(size_t)qi * k + k - 1], tidx[(size_t)qi * k + k - 1]);
+            cmask |= (cnd ? 1u : 0u) << j;
           }
         }
-        alive = epi_sync();
+        if (valid && cmask) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            if ((cmask >> j) & 1u) {
+              const int pos = atomicAdd(ncand, 1);
+              if (pos < kCandCap) {
+                cand_q[pos] = qbase + j;
+                cand_r[pos] = (int)row;
+                cand_s[pos] = __uint_as_float(dv[j]);
+              }
+            }
+          }
+        }
       }
+      if (!(alive = epi_sync())) break;
+      const int n_c = *reinterpret_cast<volatile int*>(ncand);
+      if (e8 == 0 && lane == 0) s_ncand[(ul + 1) & 1] = 0;  // next tile's counter
+      if (n_c <= kCandCap) {
+        release_d();
+        for (int base = 0; base < n_c; base += 32) {
+          const int e = base + lane;
+          const int qi = e < n_c ? cand_q[e] : -1;
+          const bool mine = qi >= 0 && (((qi - (int)qt * kQT) & 31) >> 2) == e8;
+          unsigned mask = __ballot_sync(0xFFFFFFFFu, mine);
+          while (mask) {
+            const int leader = __ffs(mask) - 1;
+            if (lane == leader) insert1(qi, cand_s[e], cand_r[e]);
+            mask &= mask - 1;
+            __syncwarp();
+          }
+        }
+      } else {
+        // ---- staging path: chunk 4 h + cc of each half per round
+        float* sbuf = stg + half * 32 * kRowsT;
+        for (int cc = 0; cc < 4 && alive; ++cc) {
+          const int c = 4 * half + cc;
+          uint32_t dv[32];
+          load_chunk(c, dv);
+          if (cc == 3) release_d();
+          const int qbase = (int)qt * kQT + 32 * c;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int qi = qbase + j;
+            const float sc = qi < nq ? s_qscale[qi] : 0.f;
+            sbuf[j * kRowsT + rloc] = valid ? __uint_as_float(dv[j]) * rs * sc : -INFINITY;
+          }
+          if (!(alive = epi_sync())) break;
+          for (int jj = 0; jj < 8; ++jj) {
+            const int j = (e8 & 3) * 8 + jj, qi = qbase + j;
+            if (qi >= nq) continue;
+            float* tq = tops + (size_t)qi * k;
+            int* ti = tidx + (size_t)qi * k;
+            const float ths = tq[k - 1];
+            const int thr = ti[k - 1];
+            float v[4];
+            int r[4];
+            unsigned cm = 0u;  // candidate bits of this lane
+            int cnt = 0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              v[i] = sbuf[j * kRowsT + lane + 32 * i];
+              r[i] = (int)(kt * kRowsT) + lane + 32 * i;
+              const bool cand = r[i] < a.n && better(v[i], r[i], ths, thr);
+              cm |= (cand ? 1u : 0u) << i;
+              cnt += __popc(__ballot_sync(0xFFFFFFFFu, cand));
+            }
+            if (cnt == 0) continue;
+            if (cnt <= 4) {
+              for (int i = 0; i < 4; ++i) {
+                unsigned mask = __ballot_sync(0xFFFFFFFFu, (cm >> i) & 1u);
+                while (mask) {
+                  const int leader = __ffs(mask) - 1;
+                  if (lane == leader) insert1(qi, v[i], r[i]);
+                  mask &= mask - 1;
+                  __syncwarp();
+                }
+              }
+            } else {
+              // merge: lanes < k hold the current list; k rounds of a warp argmax
+              float ls = lane < k ? tq[lane] : -INFINITY;
+              int lr = lane < k ? ti[lane] : 0x7FFFFFFF;
+              bool lused = lane >= k;
+              float outs = -INFINITY;
+              int outr = 0x7FFFFFFF;
+              for (int rnd = 0; rnd < k; ++rnd) {
+                float bs = -INFINITY;
+                int br = 0x7FFFFFFF;
+                if (!lused && better(ls, lr, bs, br)) {
+                  bs = ls;
+                  br = lr;
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                  if (((cm >> i) & 1u) && better(v[i], r[i], bs, br)) {
+                    bs = v[i];
+                    br = r[i];
+                  }
+                float ws = bs;
+                int wr = br;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                  const float os = __shfl_xor_sync(0xFFFFFFFFu, ws, o);
+                  const int orr = __shfl_xor_sync(0xFFFFFFFFu, wr, o);
+                  if (better(os, orr, ws, wr)) {
+                    ws = os;
+                    wr = orr;
+                  }
+                }
+                if (lane == rnd) {
+                  outs = ws;
+                  outr = wr;
+                }
+                // the owner retires the winner (rows are distinct)
+                if (!lused && lr == wr) lused = true;
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                  if (((cm >> i) & 1u) && r[i] == wr) cm &= ~(1u << i);
+              }
+              __syncwarp();
+              if (lane < k) {
+                tq[lane] = outs;
+                ti[lane] = outr;
+              }
+              __syncwarp();
+            }
+          }
+          // this round's staging tile is read before the next round writes it
+          if (!(alive = epi_sync())) break;
+        }
+      }
+      // every list update of this tile is done before the next filter pass
+      if (alive) alive = epi_sync();
     }
   }
   tqtc::tc_fence_before();
@@ -581,10 +672,10 @@ int sms() {
 
 }  // namespace
 
-// query batch: the largest multiple of 256 (or nq) whose lists fit 104 KB
+// query batch: the largest multiple of 256 (or nq) whose lists fit 96 KB
 int tq_search_batch(int nq, int k) {
   const int per = 8 * k + 4;
-  int nb = (104 * 1024 / per) / kQT * kQT;
+  int nb = (96 * 1024 / per) / kQT * kQT;
   if (nb < kQT) nb = kQT;
   return nq < nb ? nq : nb;
 }
@@ -641,7 +732,8 @@ cudaError_t tq_launch_search(const tq_params& p, const float* qprep, int nq, int
   a.qscale = qscale;
   a.part_s = part_s;
   a.part_i = part_i;
-  size_t smem = (size_t)kBStages * kGroupBytes + 32 * kRowsT * 4 + (size_t)nb * 4 + (size_t)nb * k * 8;
+  size_t smem = (size_t)kBStages * kGroupBytes + 2 * 32 * kRowsT * 4 + (size_t)kCandCap * 12 + (size_t)nb * 4 +
+                (size_t)nb * k * 8;
   // the block takes all 512 TMEM columns: ask for more than half of the SM's
   // shared memory so that a second block never waits on the allocation
   {

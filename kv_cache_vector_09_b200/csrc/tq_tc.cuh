@@ -60,6 +60,19 @@ __device__ __forceinline__ bool mbar_wait_or_abort(uint64_t* bar, uint32_t parit
   return true;
 }
 
+// As mbar_wait_or_abort, sleeping `ns` nanoseconds between polls: for
+// waiters that may wait long and would otherwise take issue slots from the
+// warps they wait for.
+__device__ __forceinline__ bool mbar_wait_sleep_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                                         unsigned ns) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if ((abort && *abort) || clock64() - t0 > kWaitCycles) return false;
+    __nanosleep(ns);
+  }
+  return true;
+}
+
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
