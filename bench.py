@@ -189,8 +189,9 @@ class Layer:
         ]
 
     # launches of libtq kernels per stage (quantize: 1; scores: query prep +
-    # scoring; attend: query prep + split-context attention + combine)
-    LAUNCHES = {"tq_quantize_K": 1, "tq_quantize_V": 1, "tq_scores": 2, "tq_attend": 3}
+    # query-limb image + scoring; attend: query prep + fused attention +
+    # combine)
+    LAUNCHES = {"tq_quantize_K": 1, "tq_quantize_V": 1, "tq_scores": 3, "tq_attend": 3}
 
     def algorithmic_bytes(self):
         w, d = self.w, self.w.d

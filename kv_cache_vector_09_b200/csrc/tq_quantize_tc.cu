@@ -88,13 +88,14 @@ __device__ __forceinline__ float2 unpack_half2(uint32_t v) {
 
 // Shared-memory layout of one block (all offsets 16-byte aligned).
 struct QLayout {
-  uint32_t a_hi, a_lo, bimg, codes, signs, nu, gam, err, flag, fmask, scratch, total;
+  uint32_t a_hi, a_lo, bimg, sl2n, codes, signs, nu, gam, err, flag, fmask, scratch, total;
   __host__ __device__ QLayout(int D, int m, int W, int nwarps) {
     uint32_t o = 0;
     const uint32_t atile = m > 0 ? (uint32_t)kRows * D * 2 : 0;
     a_hi = o; o += atile;
     a_lo = o; o += atile;
     bimg = o; o += (uint32_t)m * D * 4;
+    sl2n = o; o += (uint32_t)((m * 4 + 15) / 16 * 16);
     codes = o; o += (uint32_t)kRows * W * 4;
     signs = o; o += (uint32_t)kRows * 8 * 4;
     nu = o; o += kRows * 4;
@@ -111,7 +112,7 @@ struct QLayout {
 // Warp-cooperative fp64 evaluation of one row, written straight to the
 // outputs.  full: every code, sign, nu and gamma is rewritten; otherwise the
 // codes are certified and only the sign bits in fmask (plus nu and gamma) are.
-template <int D, typename TIn>
+template <int D, typename TIn, bool SK>
 __device__ void exact_row(const tq_params& p, const QBook& qb, const TIn* __restrict__ xr, int64_t row, bool full,
                           const uint32_t* fmask, const tq_compressed& out, double* scratch) {
   constexpr int VPL = D / 32;
@@ -148,9 +149,30 @@ __device__ void exact_row(const tq_params& p, const QBook& qb, const TIn* __rest
   }
   g2 = tq_warp_sum(g2);
   __syncwarp();
-  // sketch rows t_j = sum_i S_ji r_i: lanes split i, warp reduction
-  const int MS = p.MS;
-  for (int w = 0; w < MS; ++w) {
+  const int MS = SK ? p.MS : 0;
+  if (SK && full) {
+    // every sketch row: lane owns rows lane + 32 q, reading S^T (columns
+    // permuted so that lane l's q-th column is row l + 32 q) coalesced
+    double t[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) t[q] = 0.0;
+    for (int i = 0; i < D; ++i) {
+      const double ri = scratch[i];
+      const float* sti = p.St + (size_t)i * p.m + lane * MS;
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (q < MS) t[q] = fma((double)__ldg(sti + q), ri, t[q]);
+    }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      if (q < MS) {
+        const uint32_t word = __ballot_sync(TQ_FULL_MASK, t[q] >= 0.0);
+        if (lane == 0) out.signs[row * MS + q] = word;
+      }
+    }
+  }
+  // flagged sketch rows only: t_j = sum_i S_ji r_i, lanes split i, warp reduction
+  for (int w = 0; SK && w < MS && !full; ++w) {
     uint32_t todo = full ? 0xffffffffu : fmask[w];
     if (!todo) continue;
     uint32_t word = full ? 0u : out.signs[row * MS + w];
@@ -245,7 +267,17 @@ __global__ void __launch_bounds__(kRows * (D / 32), SK ? 1 : 2)
   if constexpr (SK) {
     const uint4* src = reinterpret_cast<const uint4*>(p.bimg);
     uint4* dst = reinterpret_cast<uint4*>(smem + ly.bimg);
-    for (int i = tid; i < m * D * 4 / 16; i += NT) dst[i] = __ldg(src + i);
+    if (m <= 128) {
+      // one B operand of N = 2m rows, [S_hi; S_lo]: 16-byte chunk `rest` of
+      // K chunk i8 of half h goes to i8 * 2m + h * m + rest
+      for (int i = tid; i < m * D * 4 / 16; i += NT) {
+        const int h = i / (m * D / 8), c = i % (m * D / 8);
+        dst[(c / m) * 2 * m + h * m + c % m] = __ldg(src + i);
+      }
+    } else {
+      for (int i = tid; i < m * D * 4 / 16; i += NT) dst[i] = __ldg(src + i);
+    }
+    for (int i = tid; i < m; i += NT) reinterpret_cast<float*>(smem + ly.sl2n)[i] = __ldg(p.sl2n + i);
     if (tid == 0) {
       tqtc::mbar_init(&s_bar, 1);
       tqtc::fence_mbar_init();
@@ -270,7 +302,7 @@ __global__ void __launch_bounds__(kRows * (D / 32), SK ? 1 : 2)
     if (tid == 0 && cnt > 0) atomicAdd(p.exact_rows, (unsigned long long)cnt);
     for (int e = warp; e < cnt; e += NW) {
       const FixEntry& f = s_fix[e];
-      exact_row<D, TIn>(p, qb, x + f.row * ld, f.row, f.full != 0, f.fmask, out, scr);
+      exact_row<D, TIn, SK>(p, qb, x + f.row * ld, f.row, f.full != 0, f.fmask, out, scr);
     }
     __syncthreads();
     if (tid == 0) s_nfix = 0;
@@ -461,20 +493,36 @@ __global__ void __launch_bounds__(kRows * (D / 32), SK ? 1 : 2)
       __syncthreads();
       if (tid == 0) {
         tqtc::tc_fence_after();
-        const uint32_t idesc = tqtc::instr_desc(1, 0, 0, kRows, (uint32_t)m);
-        const uint32_t lbo_b = 16u * (uint32_t)m;
         const uint32_t ahi = tqtc::smem_u32(smem + ly.a_hi), alo = tqtc::smem_u32(smem + ly.a_lo);
-        const uint32_t bhi = tqtc::smem_u32(smem + ly.bimg), blo = bhi + 2u * (uint32_t)m * D;
-        bool accum = false;
+        if (m <= 128) {
+          // two products: A_hi [S_hi; S_lo] (N = 2m: columns [0, m) hi*hi,
+          // [m, 2m) hi*lo) and A_lo S_hi accumulated onto columns [0, m)
+          const uint32_t b2 = tqtc::smem_u32(smem + ly.bimg), lbo2 = 32u * (uint32_t)m;
+          const uint32_t id2 = tqtc::instr_desc(1, 0, 0, kRows, 2u * (uint32_t)m);
+          const uint32_t id1 = tqtc::instr_desc(1, 0, 0, kRows, (uint32_t)m);
 #pragma unroll
-        for (int pass = 0; pass < 3; ++pass) {
-          const uint32_t aa = pass == 1 ? alo : ahi;
-          const uint32_t bb = pass == 2 ? blo : bhi;
+          for (int s = 0; s < D / 16; ++s)
+            tqtc::mma_f16_ss(tbase, tqtc::smem_desc(ahi + 2u * s * LBO_A, LBO_A, 128),
+                             tqtc::smem_desc(b2 + 2u * s * lbo2, lbo2, 128), id2, s > 0);
 #pragma unroll
-          for (int s = 0; s < D / 16; ++s) {
-            tqtc::mma_f16_ss(tbase, tqtc::smem_desc(aa + 2u * s * LBO_A, LBO_A, 128),
-                             tqtc::smem_desc(bb + 2u * s * lbo_b, lbo_b, 128), idesc, accum);
-            accum = true;
+          for (int s = 0; s < D / 16; ++s)
+            tqtc::mma_f16_ss(tbase, tqtc::smem_desc(alo + 2u * s * LBO_A, LBO_A, 128),
+                             tqtc::smem_desc(b2 + 2u * s * lbo2, lbo2, 128), id1, true);
+        } else {
+          const uint32_t idesc = tqtc::instr_desc(1, 0, 0, kRows, (uint32_t)m);
+          const uint32_t lbo_b = 16u * (uint32_t)m;
+          const uint32_t bhi = tqtc::smem_u32(smem + ly.bimg), blo = bhi + 2u * (uint32_t)m * D;
+          bool accum = false;
+#pragma unroll
+          for (int pass = 0; pass < 3; ++pass) {
+            const uint32_t aa = pass == 1 ? alo : ahi;
+            const uint32_t bb = pass == 2 ? blo : bhi;
+#pragma unroll
+            for (int s = 0; s < D / 16; ++s) {
+              tqtc::mma_f16_ss(tbase, tqtc::smem_desc(aa + 2u * s * LBO_A, LBO_A, 128),
+                               tqtc::smem_desc(bb + 2u * s * lbo_b, lbo_b, 128), idesc, accum);
+              accum = true;
+            }
           }
         }
         tqtc::mma_commit(&s_bar);
@@ -491,15 +539,20 @@ __global__ void __launch_bounds__(kRows * (D / 32), SK ? 1 : 2)
       const int rr = 32 * lq + lane;
       const float2 eg = st_err[rr];
       for (int c = warp >> 2; c < m / 32; c += NW / 4) {
-        uint32_t t16[2][16];
+        uint32_t t16[2][16], u16[2][16];
         tqtc::tmem_ld16(tqtc::tmem_addr(tbase, 32u * lq, 32u * c), t16[0]);
         tqtc::tmem_ld16(tqtc::tmem_addr(tbase, 32u * lq, 32u * c + 16u), t16[1]);
+        if (m <= 128) {
+          tqtc::tmem_ld16(tqtc::tmem_addr(tbase, 32u * lq, (uint32_t)m + 32u * c), u16[0]);
+          tqtc::tmem_ld16(tqtc::tmem_addr(tbase, 32u * lq, (uint32_t)m + 32u * c + 16u), u16[1]);
+        }
         tqtc::tmem_wait_ld();
         uint32_t word = 0, unsure = 0;
 #pragma unroll
         for (int jj = 0; jj < 32; ++jj) {
-          const float t = __uint_as_float(t16[jj >> 4][jj & 15]);
-          const float tau = fmaf(__ldg(p.sl2n + 32 * c + jj), eg.x, eg.y);
+          float t = __uint_as_float(t16[jj >> 4][jj & 15]);
+          if (m <= 128) t += __uint_as_float(u16[jj >> 4][jj & 15]);
+          const float tau = fmaf(reinterpret_cast<const float*>(smem + ly.sl2n)[32 * c + jj], eg.x, eg.y);
           unsure |= (fabsf(t) > tau ? 0u : 1u) << jj;
           word |= (t >= 0.f ? 1u : 0u) << jj;
         }
@@ -574,8 +627,8 @@ cudaError_t launch_quad(const tq_params& p, const void* x, int64_t n, int64_t ld
   auto fn = tq_quantize_quad_kernel<D, B0, B1, SK, TIn>;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ly.total);
   if (e != cudaSuccess) return e;
-  uint32_t cols = 32;
-  while (cols < (uint32_t)m) cols <<= 1;
+  uint32_t cols = 32;  // accumulator: 2m columns when the sketch uses the merged N = 2m product
+  while (cols < (uint32_t)(m <= 128 ? 2 * m : m)) cols <<= 1;
   int per_sm = 0;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, NT, ly.total);
   if (e != cudaSuccess) return e;

@@ -16,7 +16,7 @@
 // into TMEM (codes -> centroid hi/lo pairs), B is a per-query image built
 // once per call and streamed from L2 by bulk copies.  One block per SM:
 //   warps 0-3   A builders (warp w writes TMEM lanes 32 w ..)
-//   warp 4      B producer (bulk copies into a 4-stage ring)
+//   warp 4      B producer (bulk copies into a 5-stage ring)
 //   warp 5      MMA issue: 3 MMAs (M = 128, N = 256, K = 16) per group
 //   warps 6-13  epilogue: scores of the tile -> per-query top-k lists in
 //               shared memory (each query's list updated by one warp)
@@ -35,7 +35,7 @@ constexpr int kRowsT = 128;                // index rows per tile (MMA M)
 constexpr int kQT = 256;                   // queries per tile (MMA N)
 constexpr int kStepBytes = kQT * 16 * 2;   // one K = 16 step of B: 8 KB
 constexpr int kGroupBytes = 2 * kStepBytes;  // [hi | lo]
-constexpr int kBStages = 4;
+constexpr int kBStages = 5;
 constexpr int kCandCap = 2048;             // candidate buffer of the epilogue (entries)
 constexpr int kASlots = 16;                // TMEM A ring, 16 columns per slot ([hi | lo])
 constexpr int kThreads = 448;
@@ -156,10 +156,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   unsigned char* bring = smem;                                        // [kBStages][kGroupBytes]
   float* stg = reinterpret_cast<float*>(smem + kBStages * kGroupBytes);   // [2][32][kRowsT] score staging
-  int* cand_q = reinterpret_cast<int*>(stg + 2 * 32 * kRowsT);           // [kCandCap] candidates: query,
+  // the candidate buffer shares the staging tile's memory: a tile uses one
+  // or the other
+  int* cand_q = reinterpret_cast<int*>(stg);                              // [kCandCap] candidates: query,
   int* cand_r = cand_q + kCandCap;                                        //   row,
   float* cand_s = reinterpret_cast<float*>(cand_r + kCandCap);            //   score
-  float* s_qscale = cand_s + kCandCap;                                    // [nq]
+  float* s_qscale = stg + 2 * 32 * kRowsT;                                // [nq]
   float* tops = s_qscale + nq;                                            // [nq][k]
   int* tidx = reinterpret_cast<int*>(tops + (size_t)nq * k);              // [nq][k]
 
@@ -732,8 +734,7 @@ cudaError_t tq_launch_search(const tq_params& p, const float* qprep, int nq, int
   a.qscale = qscale;
   a.part_s = part_s;
   a.part_i = part_i;
-  size_t smem = (size_t)kBStages * kGroupBytes + 2 * 32 * kRowsT * 4 + (size_t)kCandCap * 12 + (size_t)nb * 4 +
-                (size_t)nb * k * 8;
+  size_t smem = (size_t)kBStages * kGroupBytes + 2 * 32 * kRowsT * 4 + (size_t)nb * 4 + (size_t)nb * k * 8;
   // the block takes all 512 TMEM columns: ask for more than half of the SM's
   // shared memory so that a second block never waits on the allocation
   {
