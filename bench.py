@@ -42,6 +42,39 @@ FALLBACK_HBM_GBS = 6650.0
 
 
 # ------------------------------------------------------------------ helpers
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of
+# each stage's main kernel, from the ncu capture summarised in
+# profiles/kernels_llama8b_decode_step.md.  It is reported only while the
+# kernel sources are the ones that capture measured (same source digest);
+# after any change to them the field is null until the capture is redone.
+TRAFFIC_SOURCES = "032341217d9c980844c51180000e367347d62b53fdfceea3bee0b467773d6a6b"
+TRAFFIC = {
+    "tq_quantize_K": 548_347_648 + 137_637_376,
+    "tq_quantize_V": 539_320_064 + 130_152_960,
+    "tq_scores": 152_045_824 + 20_649_728,
+    "tq_attend": 294_062_592 + 5_153_792,
+}
+
+
+def kernel_sources_digest() -> str:
+    """sha256 over the library's kernel and header sources (names + bytes)."""
+    import hashlib
+    csrc = os.path.join(ROOT, "kv_cache_vector_09_b200", "csrc")
+    h = hashlib.sha256()
+    for n in sorted(os.listdir(csrc)):
+        if n.endswith((".cu", ".cuh", ".h", ".cpp")):
+            h.update(n.encode())
+            with open(os.path.join(csrc, n), "rb") as f:
+                h.update(f.read())
+    with open(os.path.join(ROOT, "include", "tq.h"), "rb") as f:
+        h.update(f.read())
+    return h.hexdigest()
+
+
+def measured_traffic(stage: str):
+    return TRAFFIC.get(stage) if kernel_sources_digest() == TRAFFIC_SOURCES else None
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -543,7 +576,7 @@ def main():
     def roof(name):
         s = stages[name]
         return {"kernel": name, "bound": "hbm", "achieved": s["GB_s"], "peak": hbm, "unit": "GB/s",
-                "frac": s["frac_hbm"], "traffic": None, "peak_source": f"{peak_src} hbm_gbs",
+                "frac": s["frac_hbm"], "traffic": measured_traffic(name), "peak_source": f"{peak_src} hbm_gbs",
                 "bytes_per_launch": s["algorithmic_bytes"]}
 
     line = {

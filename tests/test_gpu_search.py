@@ -126,3 +126,47 @@ def test_search_rejects_bad_arguments():
     with pytest.raises(tq.TQError) as e:
         tq.tq_search_workspace_size(c2, 4, 10)
     assert e.value.status == 2
+
+
+def test_search_full_size_sampled():
+    """The bench's launch: 1M-row index (d = 1536, b = 3, m = 256), all 1024
+    queries, top-10.  Two sampled queries are checked against the oracle's
+    scores of every index row (evaluated in blocks on the GPU's compressed
+    index)."""
+    w = synth.VSEARCH
+    codec = tq.Codec(w.d, w.bits, w.m, w.codec_seed)
+    X = tq.Compressed.empty(codec, w.n)
+    for r0 in range(0, w.n, w.row_block):
+        r1 = min(w.n, r0 + w.row_block)
+        tq.tq_quantize(codec, synth.search_rows(w, r0, r1).to(DEV), X.rows(r0, r1))
+    torch.cuda.synchronize()
+    q = synth.search_queries(w)
+    gi, gs = _gpu_search(codec, q, X, w.n, w.k)
+    oc = O.make_codec(w.d, w.bits, w.m, w.codec_seed)
+    Xo = _to_oracle(X, w.m)
+    picks = synth.sample_indices(91, w.nq, 2)
+    q64 = q[picks].to(torch.float64).numpy()
+    # oracle top-k over all rows, block by block, then merged by a full sort
+    blk = 32768
+    cand_i, cand_s = [], []
+    for r0 in range(0, w.n, blk):
+        r1 = min(w.n, r0 + blk)
+        sub = O.Compressed(codes=Xo.codes[r0:r1], signs=Xo.signs[r0:r1], norms=Xo.norms[r0:r1],
+                           rnorms=Xo.rnorms[r0:r1])
+        ii, ss = O.search_topk(q64, sub, oc, w.k, row_offset=r0)
+        cand_i.append(ii)
+        cand_s.append(ss)
+    ci, cs = np.concatenate(cand_i, axis=1), np.concatenate(cand_s, axis=1)
+    oi = np.empty((len(picks), w.k), np.int64)
+    os_ = np.empty((len(picks), w.k))
+    for t in range(len(picks)):
+        order = np.lexsort((ci[t], -cs[t]))[:w.k]
+        oi[t], os_[t] = ci[t, order], cs[t, order]
+    tol = TIE * float(Xo.norms.max()) * np.linalg.norm(q64, axis=1)
+
+    def full_scores(t, rows):
+        sub = O.Compressed(codes=Xo.codes[rows], signs=Xo.signs[rows], norms=Xo.norms[rows], rnorms=Xo.rnorms[rows])
+        return O.estimate_scores(q64[t:t + 1], sub, oc, 1, 1, 1, len(rows))[0, 0]
+
+    check_topk(gi[picks], gs[picks], oi, os_, full_scores, tol)
+    print("full-size search, queries", picks.tolist(), "kth", os_[:, -1])
