@@ -86,6 +86,33 @@ __device__ __forceinline__ float2 unpack_half2(uint32_t v) {
   return __half22float2(*reinterpret_cast<const __half2*>(&v));
 }
 
+// packed f32x2 arithmetic (two fp32 lanes in one 64-bit register)
+__device__ __forceinline__ uint64_t pk2(float a, float b) {
+  return (uint64_t)__float_as_uint(a) | ((uint64_t)__float_as_uint(b) << 32);
+}
+__device__ __forceinline__ float lo2(uint64_t v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float hi2(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+// acc += a * b
+__device__ __forceinline__ void fma2(uint64_t& acc, uint64_t a, uint64_t b) {
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(a), "l"(b));
+}
+// a * b + c
+__device__ __forceinline__ uint64_t fma2r(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
 // Shared-memory layout of one block (all offsets 16-byte aligned).
 struct QLayout {
   uint32_t a_hi, a_lo, bimg, sl2n, codes, signs, nu, gam, err, flag, fmask, scratch, total;
@@ -368,32 +395,97 @@ __global__ void __launch_bounds__(kRows * (D / 32), SK ? 1 : 2)
         }
       }
     }
-    // ---------------------------------------------------------------- norm
-    float a4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int i = 0; i < 32; ++i) a4[i & 3] = fmaf(v[i], v[i], a4[i & 3]);
-    float ss = (a4[0] + a4[1]) + (a4[2] + a4[3]);
-    ss += __shfl_xor_sync(TQ_FULL_MASK, ss, 1);
-    if constexpr (TPR == 4) ss += __shfl_xor_sync(TQ_FULL_MASK, ss, 2);
-    bool codeflag = !(ss >= 1e-30f && ss <= 1e30f);
-    const float nu = sqrtf(ss);
-    // ---------------------------------------------------------------- FWHT
-#pragma unroll
-    for (int h = 1; h < 32; h <<= 1) {
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        if ((i & h) == 0) {
-          const float a = v[i], b = v[i + h];
-          v[i] = a + b;
-          v[i + h] = a - b;
+    // ---------------------------------------------------------------- norm, FWHT
+    // Two spellings of the same arithmetic: packed f32x2 pairs (fewer
+    // instructions) for the kernels without a sketch, scalar for the sketch
+    // kernels, whose register budget the pairs would overrun.
+    float nu;
+    bool codeflag;
+    if constexpr (!SK) {
+      // values in packed pairs (v[2k], v[2k+1]) for f32x2 arithmetic; every
+      // lane of a packed op rounds like the scalar op, so results are the same
+      uint64_t P[16];
+  #pragma unroll
+      for (int k = 0; k < 16; ++k) P[k] = pk2(v[2 * k], v[2 * k + 1]);
+      uint64_t s01 = 0ull, s23 = 0ull;  // partial sums of v_i^2 over i mod 4
+  #pragma unroll
+      for (int k = 0; k < 16; k += 2) {
+        fma2(s01, P[k], P[k]);
+        fma2(s23, P[k + 1], P[k + 1]);
+      }
+      float ss = (lo2(s01) + hi2(s01)) + (lo2(s23) + hi2(s23));
+      ss += __shfl_xor_sync(TQ_FULL_MASK, ss, 1);
+      if constexpr (TPR == 4) ss += __shfl_xor_sync(TQ_FULL_MASK, ss, 2);
+      codeflag = !(ss >= 1e-30f && ss <= 1e30f);
+      nu = sqrtf(ss);
+      // ---------------------------------------------------------------- FWHT
+      // stage h = 1 inside each pair, stages h = 2..16 between pairs, then the
+      // thread-bit stages across the row's threads
+  #pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        const float a = lo2(P[k]), b = hi2(P[k]);
+        P[k] = pk2(a + b, a - b);
+      }
+  #pragma unroll
+      for (int hp = 1; hp < 16; hp <<= 1) {
+  #pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          if ((k & hp) == 0) {
+            const uint64_t a = P[k], b = P[k + hp];
+            P[k] = add2(a, b);
+            P[k + hp] = sub2(a, b);
+          }
         }
       }
-    }
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = fmaf(sgn1, v[i], __shfl_xor_sync(TQ_FULL_MASK, v[i], 1));
-    if constexpr (TPR == 4) {
-#pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = fmaf(sgn2, v[i], __shfl_xor_sync(TQ_FULL_MASK, v[i], 2));
+      {
+        const uint64_t g1 = pk2(sgn1, sgn1);
+  #pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const uint64_t o = pk2(__shfl_xor_sync(TQ_FULL_MASK, lo2(P[k]), 1), __shfl_xor_sync(TQ_FULL_MASK, hi2(P[k]), 1));
+          P[k] = fma2r(g1, P[k], o);
+        }
+        if constexpr (TPR == 4) {
+          const uint64_t g2 = pk2(sgn2, sgn2);
+  #pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            const uint64_t o =
+                pk2(__shfl_xor_sync(TQ_FULL_MASK, lo2(P[k]), 2), __shfl_xor_sync(TQ_FULL_MASK, hi2(P[k]), 2));
+            P[k] = fma2r(g2, P[k], o);
+          }
+        }
+      }
+  #pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        v[2 * k] = lo2(P[k]);
+        v[2 * k + 1] = hi2(P[k]);
+      }
+    } else {
+      float a4[4] = {0.f, 0.f, 0.f, 0.f};
+  #pragma unroll
+      for (int i = 0; i < 32; ++i) a4[i & 3] = fmaf(v[i], v[i], a4[i & 3]);
+      float ss = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+      ss += __shfl_xor_sync(TQ_FULL_MASK, ss, 1);
+      if constexpr (TPR == 4) ss += __shfl_xor_sync(TQ_FULL_MASK, ss, 2);
+      codeflag = !(ss >= 1e-30f && ss <= 1e30f);
+      nu = sqrtf(ss);
+      // ---------------------------------------------------------------- FWHT
+  #pragma unroll
+      for (int h = 1; h < 32; h <<= 1) {
+  #pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          if ((i & h) == 0) {
+            const float a = v[i], b = v[i + h];
+            v[i] = a + b;
+            v[i + h] = a - b;
+          }
+        }
+      }
+  #pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = fmaf(sgn1, v[i], __shfl_xor_sync(TQ_FULL_MASK, v[i], 1));
+      if constexpr (TPR == 4) {
+  #pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = fmaf(sgn2, v[i], __shfl_xor_sync(TQ_FULL_MASK, v[i], 2));
+      }
     }
     // ---------------------------------------------------------------- codes
     float mt0[H0], mt1[H1];

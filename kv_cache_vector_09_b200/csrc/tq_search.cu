@@ -13,10 +13,12 @@
 // and the three MMAs of a group pair (A_hi, B_hi), (A_lo, B_hi), (A_hi, B_lo)
 // with B scaled per query by 2^e (w by 2^(e-6), g by 2^6) to keep the fp16
 // parts normal.  A is built per 128-row tile by CUDA-core warps straight
-// into TMEM (codes -> centroid hi/lo pairs), B is a per-query image built
-// once per call and streamed from L2 by bulk copies.  One block per SM:
-//   warps 0-3   A builders (warp w writes TMEM lanes 32 w ..)
-//   warp 4      B producer (bulk copies into a 5-stage ring)
+// into a shared-memory ring (codes -> centroid hi/lo pairs), B is a
+// per-query image built once per call and streamed from L2 by bulk copies;
+// the fp32 accumulator is double-buffered in TMEM so that the epilogue of one
+// tile overlaps the MMAs of the next.  One block per SM:
+//   warps 0-3   A builders (warp w builds rows 32 w ..)
+//   warp 4      B producer (bulk copies into a 4-stage ring)
 //   warp 5      MMA issue: 3 MMAs (M = 128, N = 256, K = 16) per group
 //   warps 6-13  epilogue: scores of the tile -> per-query top-k lists in
 //               shared memory (each query's list updated by one warp)
@@ -35,9 +37,12 @@ constexpr int kRowsT = 128;                // index rows per tile (MMA M)
 constexpr int kQT = 256;                   // queries per tile (MMA N)
 constexpr int kStepBytes = kQT * 16 * 2;   // one K = 16 step of B: 8 KB
 constexpr int kGroupBytes = 2 * kStepBytes;  // [hi | lo]
-constexpr int kBStages = 5;
+constexpr int kBStages = 4;
 constexpr int kCandCap = 2048;             // candidate buffer of the epilogue (entries)
-constexpr int kASlots = 16;                // TMEM A ring, 16 columns per slot ([hi | lo])
+constexpr int kASlots = 8;                 // A ring in shared memory, [hi | lo] per slot
+constexpr int kABatch = 4;                 // groups signalled together; at most kASlots / 2, so that a
+                                           // batch never waits on a slot of its own
+constexpr int kASlotBytes = 2 * kRowsT * 16 * 2;  // two K = 16 steps of 128 rows: 8 KB
 constexpr int kThreads = 448;
 constexpr float kQjlGain = 64.f;           // 2^6 on the A side of the sketch groups
 
@@ -143,7 +148,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     search_kernel(const tq_params p, const SearchArgs a) {
   extern __shared__ __align__(1024) unsigned char smem[];
   __shared__ uint64_t a_full[kASlots], a_empty[kASlots], b_full[kBStages], b_empty[kBStages];
-  __shared__ uint64_t d_full, d_empty, drained, epi_bar;
+  __shared__ uint64_t d_full[2], d_empty[2], drained, epi_bar;
   __shared__ int s_ncand[2];
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_abort;
@@ -155,7 +160,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nq = a.nq, k = a.k;
 
   unsigned char* bring = smem;                                        // [kBStages][kGroupBytes]
-  float* stg = reinterpret_cast<float*>(smem + kBStages * kGroupBytes);   // [2][32][kRowsT] score staging
+  unsigned char* aring = smem + kBStages * kGroupBytes;               // [kASlots][kASlotBytes]
+  float* stg = reinterpret_cast<float*>(aring + kASlots * kASlotBytes);  // [2][32][kRowsT] score staging
   // the candidate buffer shares the staging tile's memory: a tile uses one
   // or the other
   int* cand_q = reinterpret_cast<int*>(stg);                              // [kCandCap] candidates: query,
@@ -189,8 +195,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tqtc::mbar_init(&b_full[i], 1);
       tqtc::mbar_init(&b_empty[i], 1);
     }
-    tqtc::mbar_init(&d_full, 1);
-    tqtc::mbar_init(&d_empty, 256);
+    for (int i = 0; i < 2; ++i) {
+      tqtc::mbar_init(&d_full[i], 1);
+      tqtc::mbar_init(&d_empty[i], 256);
+    }
     tqtc::mbar_init(&drained, 1);
     tqtc::mbar_init(&epi_bar, 256);
     tqtc::fence_mbar_init();
@@ -201,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tqtc::tc_fence_before();
   __syncthreads();
   tqtc::tc_fence_after();
-  const uint32_t tbase = s_tmem;  // D: columns [0, 256); A ring: [256, 512)
+  const uint32_t tbase = s_tmem;  // accumulators: columns [0, 256) and [256, 512)
   auto fail = [&](uint32_t code) {
     atomicExch(p.err, code);
     s_abort = 1;
@@ -209,12 +217,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < 4) {
     // ---------------------------------------------------------- A builders
-    const uint32_t lane_base = 32u * (uint32_t)warp;
     const int rloc = 32 * warp + lane;
     const float gk = p.qjl_coef * sqrtf((float)d) * kQjlGain;
     // put one group into its ring slot (after the slot's previous MMAs are
-    // done); groups are signalled in batches: one wait for the stores, then
-    // an arrival per slot
+    // done); groups are signalled in batches of kABatch: one proxy fence,
+    // then an arrival per slot
     auto put = [&](int64_t x, const uint32_t (&hi)[8], const uint32_t (&lo)[8]) -> bool {
       const int slot = (int)(x % kASlots);
       if (x >= kASlots &&
@@ -222,16 +229,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         fail(tqtc::kErrMmaWait);
         return false;
       }
-      tqtc::tc_fence_after();
-      const uint32_t col = 256u + 16u * (uint32_t)slot;
-      tqtc::tmem_st8(tqtc::tmem_addr(tbase, lane_base, col), hi);
-      tqtc::tmem_st8(tqtc::tmem_addr(tbase, lane_base, col + 8u), lo);
+      // K-major core matrices: (row, k) at (k / 8) * 2048 + (row / 8) * 128 + (row % 8) * 16 + (k % 8) * 2
+      unsigned char* sl = aring + (size_t)slot * kASlotBytes + (rloc / 8) * 128 + (rloc % 8) * 16;
+      *reinterpret_cast<uint4*>(sl) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      *reinterpret_cast<uint4*>(sl + 2048) = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+      *reinterpret_cast<uint4*>(sl + 4096) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      *reinterpret_cast<uint4*>(sl + 6144) = make_uint4(lo[4], lo[5], lo[6], lo[7]);
       return true;
     };
     // signal groups x0 .. x0 + cnt - 1
     auto signal = [&](int64_t x0, int cnt) {
-      tqtc::tmem_wait_st();
-      tqtc::tc_fence_before();
+      tqtc::fence_proxy_async_smem();  // the MMAs read these stores through the async proxy
       for (int i = 0; i < cnt; ++i) tqtc::mbar_arrive(&a_full[(int)((x0 + i) % kASlots)]);
     };
     // 16 codes (one 16-bit half of each plane word) -> centroid hi / lo pairs
@@ -288,9 +296,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               decode16(pl, hi, lo);
               if (alive && !put(x0 + 2 * (4 * blk + ww) + hh, hi, lo)) alive = false;
             }
+            if (alive && (ww & 1)) signal(x0 + 8 * blk + 2 * (ww - 1), kABatch);
           }
           if (!alive) break;
-          signal(x0 + 8 * blk, 8);
 #pragma unroll
           for (int b = 0; b < BITS; ++b) cur[b] = nxt[b];
         }
@@ -323,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             lo[pp] = glo2 ^ mask;
           }
           alive = put(x0 + gc + g, hi, lo);
-          if (alive && (++pending == 8 || g == 2 * MS - 1)) {
+          if (alive && (++pending == kABatch || g == 2 * MS - 1)) {
             signal(x0 + gc + g + 1 - pending, pending);
             pending = 0;
           }
@@ -360,9 +368,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------- MMA issue
     if (lane == 0) {
       const uint32_t idesc = tqtc::instr_desc(1, 0, 0, kRowsT, kQT);
-      const uint32_t bbase = tqtc::smem_u32(bring);
+      const uint32_t bbase = tqtc::smem_u32(bring), abase = tqtc::smem_u32(aring);
       for (int64_t ul = 0; ul < nul && !s_abort; ++ul) {
-        if (ul >= 1 && !tqtc::mbar_wait_or_abort(&d_empty, (uint32_t)((ul - 1) & 1), &s_abort)) {
+        const int db = (int)(ul & 1);
+        if (ul >= 2 && !tqtc::mbar_wait_or_abort(&d_empty[db], (uint32_t)((ul / 2 - 1) & 1), &s_abort)) {
           fail(tqtc::kErrMmaWait);
           break;
         }
@@ -377,17 +386,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tqtc::tc_fence_after();
-          const uint32_t acol = tbase + 256u + 16u * (uint32_t)slot;
+          const uint32_t a0 = abase + (uint32_t)slot * kASlotBytes;
           const uint32_t b0 = bbase + (uint32_t)st * kGroupBytes;
+          const uint64_t ahi = tqtc::smem_desc(a0, 2048u, 128u), alo = tqtc::smem_desc(a0 + 4096u, 2048u, 128u);
           const uint64_t bhi = tqtc::smem_desc(b0, 4096u, 128u), blo = tqtc::smem_desc(b0 + kStepBytes, 4096u, 128u);
-          tqtc::mma_f16_ts(tbase, acol, bhi, idesc, g > 0);       // A_hi B_hi
-          tqtc::mma_f16_ts(tbase, acol + 8u, bhi, idesc, true);   // A_lo B_hi
-          tqtc::mma_f16_ts(tbase, acol, blo, idesc, true);        // A_hi B_lo
+          const uint32_t dcol = tbase + 256u * (uint32_t)db;
+          tqtc::mma_f16_ss(dcol, ahi, bhi, idesc, g > 0);  // A_hi B_hi
+          tqtc::mma_f16_ss(dcol, alo, bhi, idesc, true);   // A_lo B_hi
+          tqtc::mma_f16_ss(dcol, ahi, blo, idesc, true);   // A_hi B_lo
           tqtc::mma_commit(&a_empty[slot]);
           tqtc::mma_commit(&b_empty[st]);
         }
         if (!ok) break;
-        tqtc::mma_commit(&d_full);
+        tqtc::mma_commit(&d_full[db]);
       }
       tqtc::mma_commit(&drained);
       if (!tqtc::mbar_wait_or_abort(&drained, 0, nullptr)) atomicExch(p.err, tqtc::kErrMmaWait);
@@ -434,15 +445,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       tq[pos] = sv;
       ti[pos] = rv;
     };
+    int db = 0;          // accumulator buffer of the current tile
+    uint32_t dcol = 0u;  // its first TMEM column
     auto load_chunk = [&](int c, uint32_t (&dv)[32]) {
-      tqtc::tmem_ld16(tqtc::tmem_addr(tbase, 32u * quarter, 32u * c), *reinterpret_cast<uint32_t(*)[16]>(dv));
-      tqtc::tmem_ld16(tqtc::tmem_addr(tbase, 32u * quarter, 32u * c + 16u),
+      tqtc::tmem_ld16(tqtc::tmem_addr(tbase, 32u * quarter, dcol + 32u * c), *reinterpret_cast<uint32_t(*)[16]>(dv));
+      tqtc::tmem_ld16(tqtc::tmem_addr(tbase, 32u * quarter, dcol + 32u * c + 16u),
                       *reinterpret_cast<uint32_t(*)[16]>(dv + 16));
       tqtc::tmem_wait_ld();
     };
     auto release_d = [&]() {
       tqtc::tc_fence_before();
-      tqtc::mbar_arrive(&d_empty);
+      tqtc::mbar_arrive(&d_empty[db]);
     };
     bool alive = true;
     for (int64_t ul = 0; ul < nul && alive; ++ul) {
@@ -451,7 +464,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool valid = row < a.n;
       const float rs = valid ? __ldg(a.norms + row) * inv_sqrt_d : 0.f;
       int* ncand = &s_ncand[ul & 1];
-      if (!tqtc::mbar_wait_or_abort(&d_full, (uint32_t)(ul & 1), &s_abort)) {
+      db = (int)(ul & 1);
+      dcol = 256u * (uint32_t)db;
+      if (!tqtc::mbar_wait_or_abort(&d_full[db], (uint32_t)((ul / 2) & 1), &s_abort)) {
         fail(tqtc::kErrMmaWait);
         break;
       }
@@ -674,10 +689,10 @@ int sms() {
 
 }  // namespace
 
-// query batch: the largest multiple of 256 (or nq) whose lists fit 96 KB
+// query batch: the largest multiple of 256 (or nq) whose lists fit 64 KB
 int tq_search_batch(int nq, int k) {
   const int per = 8 * k + 4;
-  int nb = (96 * 1024 / per) / kQT * kQT;
+  int nb = (64 * 1024 / per) / kQT * kQT;
   if (nb < kQT) nb = kQT;
   return nq < nb ? nq : nb;
 }
@@ -734,7 +749,8 @@ cudaError_t tq_launch_search(const tq_params& p, const float* qprep, int nq, int
   a.qscale = qscale;
   a.part_s = part_s;
   a.part_i = part_i;
-  size_t smem = (size_t)kBStages * kGroupBytes + 2 * 32 * kRowsT * 4 + (size_t)nb * 4 + (size_t)nb * k * 8;
+  size_t smem = (size_t)kBStages * kGroupBytes + (size_t)kASlots * kASlotBytes + 2 * 32 * kRowsT * 4 + (size_t)nb * 4 +
+                (size_t)nb * k * 8;
   // the block takes all 512 TMEM columns: ask for more than half of the SM's
   // shared memory so that a second block never waits on the allocation
   {
