@@ -18,7 +18,7 @@
 // the fp32 accumulator is double-buffered in TMEM so that the epilogue of one
 // tile overlaps the MMAs of the next.  One block per SM:
 //   warps 0-3   A builders (warp w builds rows 32 w ..)
-//   warp 4      B producer (bulk copies into a 4-stage ring)
+//   warp 4      B producer (bulk copies into a ring of 4..8 stages)
 //   warp 5      MMA issue: 3 MMAs (M = 128, N = 256, K = 16) per group
 //   warps 6-13  epilogue: scores of the tile -> per-query top-k lists in
 //               shared memory (each query's list updated by one warp)
@@ -37,7 +37,7 @@ constexpr int kRowsT = 128;                // index rows per tile (MMA M)
 constexpr int kQT = 256;                   // queries per tile (MMA N)
 constexpr int kStepBytes = kQT * 16 * 2;   // one K = 16 step of B: 8 KB
 constexpr int kGroupBytes = 2 * kStepBytes;  // [hi | lo]
-constexpr int kBStages = 4;
+constexpr int kBStagesMax = 8;               // B ring depth: as many as shared memory allows
 constexpr int kCandCap = 2048;             // candidate buffer of the epilogue (entries)
 constexpr int kASlots = 8;                 // A ring in shared memory, [hi | lo] per slot
 constexpr int kABatch = 4;                 // groups signalled together; at most kASlots / 2, so that a
@@ -137,6 +137,7 @@ struct SearchArgs {
   int k;
   const uint8_t* img;
   const float* qscale;
+  int bstages;     // B ring depth (<= kBStagesMax)
   float* part_s;   // [grid][nq][k]
   int* part_i;
 };
@@ -147,7 +148,7 @@ template <int BITS>
 __global__ void __launch_bounds__(kThreads, 1)
     search_kernel(const tq_params p, const SearchArgs a) {
   extern __shared__ __align__(1024) unsigned char smem[];
-  __shared__ uint64_t a_full[kASlots], a_empty[kASlots], b_full[kBStages], b_empty[kBStages];
+  __shared__ uint64_t a_full[kASlots], a_empty[kASlots], b_full[kBStagesMax], b_empty[kBStagesMax];
   __shared__ uint64_t d_full[2], d_empty[2], drained, epi_bar;
   __shared__ int s_ncand[2];
   __shared__ uint32_t s_tmem;
@@ -159,6 +160,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nq = a.nq, k = a.k;
 
+  const int kBStages = a.bstages;
   unsigned char* bring = smem;                                        // [kBStages][kGroupBytes]
   unsigned char* aring = smem + kBStages * kGroupBytes;               // [kASlots][kASlotBytes]
   float* stg = reinterpret_cast<float*>(aring + kASlots * kASlotBytes);  // [2][32][kRowsT] score staging
@@ -689,7 +691,8 @@ int sms() {
 
 }  // namespace
 
-// query batch: the largest multiple of 256 (or nq) whose lists fit 64 KB
+// query batch: the largest multiple of 256 (or nq) whose lists fit 64 KB (512
+// queries at k = 10; each batch re-reads the index, so batches stay large)
 int tq_search_batch(int nq, int k) {
   const int per = 8 * k + 4;
   int nb = (64 * 1024 / per) / kQT * kQT;
@@ -749,8 +752,12 @@ cudaError_t tq_launch_search(const tq_params& p, const float* qprep, int nq, int
   a.qscale = qscale;
   a.part_s = part_s;
   a.part_i = part_i;
-  size_t smem = (size_t)kBStages * kGroupBytes + (size_t)kASlots * kASlotBytes + 2 * 32 * kRowsT * 4 + (size_t)nb * 4 +
-                (size_t)nb * k * 8;
+  // the B ring takes what shared memory the rest leaves (227 KB per block,
+  // 2 KB kept for the static part)
+  const size_t fixed = (size_t)kASlots * kASlotBytes + 2 * 32 * kRowsT * 4 + (size_t)nb * 4 + (size_t)nb * k * 8;
+  a.bstages = (int)std::min<size_t>(kBStagesMax, (227 * 1024 - 2048 - fixed) / kGroupBytes);
+  if (a.bstages < 2) return cudaErrorNotSupported;
+  size_t smem = (size_t)a.bstages * kGroupBytes + fixed;
   // the block takes all 512 TMEM columns: ask for more than half of the SM's
   // shared memory so that a second block never waits on the allocation
   {
