@@ -366,6 +366,16 @@ def load_tensor_peak():
         return 1590.0, "fallback 1.59 PFLOP/s"
 
 
+def search_batches(nq: int, k: int) -> int:
+    """Query batches of one tq_search_topk call: the library takes the largest
+    multiple of 256 queries whose top-k lists (8k + 4 bytes per query) fit
+    64 KB of shared memory, at least 256; each batch launches query prep,
+    exponents, query image, search and merge (5 kernels)."""
+    per = 8 * k + 4
+    nb = max(256, (64 * 1024 // per) // 256 * 256)
+    return -(-nq // nb)
+
+
 def cpu_search_sample(w, budget_s: float):
     """The oracle's top-k on a bounded sample: a few queries against the first
     rows of the index (quantised by the oracle).  Returns (pairs/s, seconds,
@@ -459,7 +469,7 @@ def run_search(args, tq, dev, rank, world, pg):
         "roofline": {"kernel": "tq_search_topk", "bound": "tensor", "achieved": round(ach, 1), "peak": peak,
                      "unit": "TFLOP/s", "frac": round(ach / peak, 4), "traffic": None, "peak_source": peak_src,
                      "flops_per_launch": alg_flops, "executed_tensor_flops_per_launch": exec_flops},
-        "gpu_launches": args.steps * 5,
+        "gpu_launches": args.steps * 5 * search_batches(w.nq, w.k),
         "e2e": {"value": whole_job_value(pairs, world, e2e_ms), "unit": "pairs/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": qh.numel() * 4, "d2h_bytes_per_step": ih.numel() * 4 + sh.numel() * 4},
         "clocks": clocks.summary(t_wall0, t_wall1),

@@ -210,32 +210,48 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
 template <int VPL, typename TIn>
 __global__ void __launch_bounds__(256)
     tq_qprep_kernel(const tq_params p, const TIn* __restrict__ q, const int nq, float* __restrict__ qprep) {
+  // one query per block: warp 0 rotates it (q' = Pi q), then every thread
+  // takes sketch rows j = tid, tid + blockDim.x, .. of w = S q', reading the
+  // rows of S (row-major [m][d]) with 16-byte loads
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int d = p.d, Q = p.MS;
-  float* buf = reinterpret_cast<float*>(smem_raw) + (size_t)warp * d;
-  const int row = blockIdx.x * (blockDim.x >> 5) + warp;
+  const int d = p.d, m = p.m;
+  float* buf = reinterpret_cast<float*>(smem_raw);
+  const int row = blockIdx.x;
   if (row >= nq) return;
-  float v[VPL];
+  float* o = qprep + (size_t)row * (d + m);
+  if (warp == 0) {
+    float v[VPL];
 #pragma unroll
-  for (int k = 0; k < VPL; ++k) {
-    const float a = tq_to_f32(q[(size_t)row * d + lane + 32 * k]);
-    v[k] = tq_dneg(p.dbits, k, lane) ? -a : a;
-  }
-  tq_fwht_warp<VPL>(v, lane);
-  float* o = qprep + (size_t)row * (d + p.m);
+    for (int k = 0; k < VPL; ++k) {
+      const float a = tq_to_f32(q[(size_t)row * d + lane + 32 * k]);
+      v[k] = tq_dneg(p.dbits, k, lane) ? -a : a;
+    }
+    tq_fwht_warp<VPL>(v, lane);
 #pragma unroll
-  for (int k = 0; k < VPL; ++k) {
-    v[k] *= p.inv_sqrt_p;
-    o[lane + 32 * k] = v[k];
-    buf[lane + 32 * k] = v[k];
+    for (int k = 0; k < VPL; ++k) {
+      v[k] *= p.inv_sqrt_p;
+      o[lane + 32 * k] = v[k];
+      buf[lane + 32 * k] = v[k];
+    }
   }
-  __syncwarp();
-  for (int qq = 0; qq < Q; ++qq) {
-    const float* sc = p.St + lane * Q + qq;
-    float t = 0.f;
-    for (int i = 0; i < d; ++i) t = fmaf(__ldg(sc + (size_t)i * p.m), buf[i], t);
-    o[d + lane + 32 * qq] = t;
+  __syncthreads();
+  for (int j = threadIdx.x; j < m; j += blockDim.x) {
+    const float4* sr = reinterpret_cast<const float4*>(p.S + (size_t)j * d);
+    float t0 = 0.f, t1 = 0.f;
+    for (int i = 0; i < d / 4; i += 2) {
+      const float4 a = __ldg(sr + i);
+      const float4 b = __ldg(sr + i + 1);
+      t0 = fmaf(a.x, buf[4 * i], t0);
+      t0 = fmaf(a.y, buf[4 * i + 1], t0);
+      t0 = fmaf(a.z, buf[4 * i + 2], t0);
+      t0 = fmaf(a.w, buf[4 * i + 3], t0);
+      t1 = fmaf(b.x, buf[4 * i + 4], t1);
+      t1 = fmaf(b.y, buf[4 * i + 5], t1);
+      t1 = fmaf(b.z, buf[4 * i + 6], t1);
+      t1 = fmaf(b.w, buf[4 * i + 7], t1);
+    }
+    o[d + j] = t0 + t1;
   }
 }
 
@@ -542,12 +558,13 @@ cudaError_t launch_quantize_v(const tq_params& p, const void* x, tq_dtype dt, in
 
 template <int VPL, typename TIn>
 cudaError_t launch_qprep_t(const tq_params& p, const void* q, int nq, float* qprep, cudaStream_t st) {
-  const int warps = 8;
-  const size_t smem = sizeof(float) * (size_t)warps * p.d;
+  const size_t smem = sizeof(float) * (size_t)p.d;
+  const int threads = p.m > 128 ? 256 : 128;
   auto fn = tq_qprep_kernel<VPL, TIn>;
   cudaError_t e = set_smem(fn, smem);
   if (e != cudaSuccess) return e;
-  fn<<<(nq + warps - 1) / warps, warps * 32, smem, st>>>(p, (const TIn*)q, nq, qprep);
+  if (nq == 0) return cudaSuccess;
+  fn<<<nq, threads, smem, st>>>(p, (const TIn*)q, nq, qprep);
   return cudaGetLastError();
 }
 

@@ -53,7 +53,9 @@ struct Geom {
 };
 
 // ------------------------------------------------------------ B operand
-// One block per (batch, KV head) group.  qprep rows are [q' (d) | w (m)].
+// Blocks (group, part): every block of a (batch, KV head) group computes the
+// group's per-query exponents, then writes part `blockIdx.y` of its image
+// (part 0 also the per-query constants).  qprep rows are [q' (d) | w (m)].
 __global__ void __launch_bounds__(256) tq_scores_bbuild_kernel(const tq_params p, const float* __restrict__ qprep,
                                                                const int Hq, const int Hkv, uint8_t* __restrict__ ws) {
   const Geom g(p, Hq / Hkv);
@@ -97,15 +99,19 @@ __global__ void __launch_bounds__(256) tq_scores_bbuild_kernel(const tq_params p
       const int eq = 30 - ex;
       s_xmse[gq] = em;
       s_xqjl[gq] = eq;
-      consts[4 * gq + 0] = ldexpf(1.f, -em);
-      consts[4 * gq + 1] = corr;
-      consts[4 * gq + 2] = ldexpf(1.f, -eq);
-      consts[4 * gq + 3] = wsum;
+      if (blockIdx.y == 0) {
+        consts[4 * gq + 0] = ldexpf(1.f, -em);
+        consts[4 * gq + 1] = corr;
+        consts[4 * gq + 2] = ldexpf(1.f, -eq);
+        consts[4 * gq + 3] = wsum;
+      }
     }
   }
   __syncthreads();
   const int u0 = p.nterms[0] * p.pw;
-  for (int idx = threadIdx.x; idx < g.Kt * g.N; idx += blockDim.x) {
+  const int total = g.Kt * g.N, per = (total + gridDim.y - 1) / gridDim.y;
+  const int i0 = blockIdx.y * per, i1 = min(total, i0 + per);
+  for (int idx = i0 + threadIdx.x; idx < i1; idx += blockDim.x) {
     const int n = idx / g.Kt, k = idx % g.Kt;
     const int gq = n / 4, l = n % 4;
     int8_t limb = 0;
@@ -536,7 +542,7 @@ cudaError_t tq_launch_scores_tc(const tq_params& p, const float* qprep, int B, i
   uint32_t cols = 0;
   if (!supported(p, Hq / Hkv, &cols)) return cudaErrorNotSupported;
   uint8_t* ws = reinterpret_cast<uint8_t*>(ws_tc);
-  tq_scores_bbuild_kernel<<<B * Hkv, 256, 0, st>>>(p, qprep, Hq, Hkv, ws);
+  tq_scores_bbuild_kernel<<<dim3((unsigned)(B * Hkv), 8), 256, 0, st>>>(p, qprep, Hq, Hkv, ws);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   switch (p.d * 100 + p.bits[0] * 10 + (p.nseg == 2 ? p.bits[1] : 0)) {

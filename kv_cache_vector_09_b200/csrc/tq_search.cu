@@ -344,21 +344,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------- B producer
     if (lane == 0) {
       int64_t issued = 0;
+      int st = 0, wrap = 0;  // ring stage and completed passes over the ring
       for (int64_t ul = 0; ul < nul && !s_abort; ++ul) {
         const int64_t qt = (u0 + ul) % a.nqt;
         const uint8_t* src = a.img + (size_t)qt * ngroups * kGroupBytes;
         for (int g = 0; g < ngroups; ++g) {
-          const int64_t x = ul * ngroups + g;
-          const int st = (int)(x % kBStages);
-          if (x >= kBStages &&
-              !tqtc::mbar_wait_sleep_or_abort(&b_empty[st], (uint32_t)((x / kBStages - 1) & 1), &s_abort, 64)) {
+          if (wrap > 0 && !tqtc::mbar_wait_sleep_or_abort(&b_empty[st], (uint32_t)((wrap - 1) & 1), &s_abort, 64)) {
             fail(tqtc::kErrCopyWait);
             break;
           }
           tqtc::mbar_arrive_expect_tx(&b_full[st], (uint32_t)kGroupBytes);
           tqtc::bulk_g2s(bring + (size_t)st * kGroupBytes, src + (size_t)g * kGroupBytes, (uint32_t)kGroupBytes,
                          &b_full[st]);
-          issued = x + 1;
+          ++issued;
+          if (++st == kBStages) {
+            st = 0;
+            ++wrap;
+          }
         }
       }
       // let every copy still in flight land before the block exits (bounded)
@@ -371,6 +373,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t idesc = tqtc::instr_desc(1, 0, 0, kRowsT, kQT);
       const uint32_t bbase = tqtc::smem_u32(bring), abase = tqtc::smem_u32(aring);
+      int st = 0, wrap = 0;  // B ring stage and completed passes over the ring
       for (int64_t ul = 0; ul < nul && !s_abort; ++ul) {
         const int db = (int)(ul & 1);
         if (ul >= 2 && !tqtc::mbar_wait_or_abort(&d_empty[db], (uint32_t)((ul / 2 - 1) & 1), &s_abort)) {
@@ -380,9 +383,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         for (int g = 0; g < ngroups; ++g) {
           const int64_t x = ul * ngroups + g;
-          const int slot = (int)(x % kASlots), st = (int)(x % kBStages);
+          const int slot = (int)(x % kASlots);
           if (!tqtc::mbar_wait_or_abort(&a_full[slot], (uint32_t)((x / kASlots) & 1), &s_abort) ||
-              !tqtc::mbar_wait_or_abort(&b_full[st], (uint32_t)((x / kBStages) & 1), &s_abort)) {
+              !tqtc::mbar_wait_or_abort(&b_full[st], (uint32_t)(wrap & 1), &s_abort)) {
             fail(tqtc::kErrMmaWait);
             ok = false;
             break;
@@ -398,6 +401,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tqtc::mma_f16_ss(dcol, ahi, blo, idesc, true);   // A_hi B_lo
           tqtc::mma_commit(&a_empty[slot]);
           tqtc::mma_commit(&b_empty[st]);
+          if (++st == kBStages) {
+            st = 0;
+            ++wrap;
+          }
         }
         if (!ok) break;
         tqtc::mma_commit(&d_full[db]);
