@@ -372,7 +372,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------- MMA issue
     if (lane == 0) {
       const uint32_t idesc = tqtc::instr_desc(1, 0, 0, kRowsT, kQT);
-      const uint32_t bbase = tqtc::smem_u32(bring), abase = tqtc::smem_u32(aring);
+      // descriptors of slot 0 / stage 0; other slots and stages, and the lo
+      // halves, are offsets of the 16-byte-unit address field
+      const uint64_t adesc0 = tqtc::smem_desc(tqtc::smem_u32(aring), 2048u, 128u);
+      const uint64_t bdesc0 = tqtc::smem_desc(tqtc::smem_u32(bring), 4096u, 128u);
+      // fast path: the barrier is usually complete already
+      auto wait_full = [&](uint64_t* bar, uint32_t parity) -> bool {
+        return tqtc::mbar_try_wait(bar, parity) || tqtc::mbar_wait_or_abort(bar, parity, &s_abort);
+      };
       int st = 0, wrap = 0;  // B ring stage and completed passes over the ring
       for (int64_t ul = 0; ul < nul && !s_abort; ++ul) {
         const int db = (int)(ul & 1);
@@ -384,17 +391,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int g = 0; g < ngroups; ++g) {
           const int64_t x = ul * ngroups + g;
           const int slot = (int)(x % kASlots);
-          if (!tqtc::mbar_wait_or_abort(&a_full[slot], (uint32_t)((x / kASlots) & 1), &s_abort) ||
-              !tqtc::mbar_wait_or_abort(&b_full[st], (uint32_t)(wrap & 1), &s_abort)) {
+          if (!wait_full(&a_full[slot], (uint32_t)((x / kASlots) & 1)) || !wait_full(&b_full[st], (uint32_t)(wrap & 1))) {
             fail(tqtc::kErrMmaWait);
             ok = false;
             break;
           }
           tqtc::tc_fence_after();
-          const uint32_t a0 = abase + (uint32_t)slot * kASlotBytes;
-          const uint32_t b0 = bbase + (uint32_t)st * kGroupBytes;
-          const uint64_t ahi = tqtc::smem_desc(a0, 2048u, 128u), alo = tqtc::smem_desc(a0 + 4096u, 2048u, 128u);
-          const uint64_t bhi = tqtc::smem_desc(b0, 4096u, 128u), blo = tqtc::smem_desc(b0 + kStepBytes, 4096u, 128u);
+          const uint64_t ahi = adesc0 + (uint64_t)(slot * (kASlotBytes >> 4)), alo = ahi + (4096u >> 4);
+          const uint64_t bhi = bdesc0 + (uint64_t)(st * (kGroupBytes >> 4)), blo = bhi + (uint64_t)(kStepBytes >> 4);
           const uint32_t dcol = tbase + 256u * (uint32_t)db;
           tqtc::mma_f16_ss(dcol, ahi, bhi, idesc, g > 0);  // A_hi B_hi
           tqtc::mma_f16_ss(dcol, alo, bhi, idesc, true);   // A_lo B_hi
