@@ -97,3 +97,33 @@ def test_not_converged_is_reported():
     lib = tq.c_api()
     st = lib.tq_make_codebook(3, 128, 1e-15, 3, cen.ctypes.data, bnd.ctypes.data)
     assert st == 6 and np.all(cen == 0)
+
+
+def test_search_arguments_are_checked_on_the_host():
+    lib = tq.c_api()
+    c = tq.Codec(1536, (3,), 256, 0, device=-1)
+    assert tq.tq_search_workspace_size(c, 1024, 10) > 0
+    for nq, k in [(4, 0), (4, 33), (-1, 10)]:
+        with pytest.raises(tq.TQError) as e:
+            tq.tq_search_workspace_size(c, nq, k)
+        assert e.value.status == 1
+    seg = tq.Codec(128, (2, 3), 64, 0, device=-1)
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_search_workspace_size(seg, 4, 10)
+    assert e.value.status == 2
+    # a compute call on a host-only codec fails before touching a GPU
+    xs = tq.tq_compressed()
+    st = lib.tq_search_topk(c.handle, None, 0, 4, ctypes.byref(xs), 100, 10, None, None, None, 0, None)
+    assert st == 1 and "host-only" in tq.tq_last_error_string()
+
+
+def test_bench_search_batches_follow_the_library_rule():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
+    b = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(b)
+    # 64 KB of top-k lists (8k + 4 bytes per query), multiples of 256, at least 256
+    assert b.search_batches(1024, 10) == 2
+    assert b.search_batches(768, 10) == 1
+    assert b.search_batches(300, 32) == 2
+    assert b.search_batches(1, 1) == 1
