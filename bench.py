@@ -47,12 +47,12 @@ FALLBACK_HBM_GBS = 6650.0
 # profiles/kernels_llama8b_decode_step.md.  It is reported only while the
 # kernel sources are the ones that capture measured (same source digest);
 # after any change to them the field is null until the capture is redone.
-TRAFFIC_SOURCES = "032341217d9c980844c51180000e367347d62b53fdfceea3bee0b467773d6a6b"
+TRAFFIC_SOURCES = "15d0fe6504f2ec3a3f451d976c02cd9a270d26aa06d667b4dc990a2f0561fedc"
 TRAFFIC = {
-    "tq_quantize_K": 548_347_648 + 137_637_376,
-    "tq_quantize_V": 539_320_064 + 130_152_960,
-    "tq_scores": 152_045_824 + 20_649_728,
-    "tq_attend": 294_062_592 + 5_153_792,
+    "tq_quantize_K": 547_984_384 + 137_492_480,
+    "tq_quantize_V": 539_168_256 + 131_811_584,
+    "tq_scores": 152_022_016 + 19_559_168,
+    "tq_attend": 293_933_056 + 6_545_152,
 }
 
 
