@@ -388,27 +388,38 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         bool ok = true;
-        for (int g = 0; g < ngroups; ++g) {
+        const uint32_t dcol = tbase + 256u * (uint32_t)db;
+        // two K groups per iteration (ngroups is even): both groups' operands
+        // are checked, then their six MMAs go out back to back
+        for (int g = 0; g < ngroups; g += 2) {
           const int64_t x = ul * ngroups + g;
-          const int slot = (int)(x % kASlots);
-          if (!wait_full(&a_full[slot], (uint32_t)((x / kASlots) & 1)) || !wait_full(&b_full[st], (uint32_t)(wrap & 1))) {
+          const int slot = (int)(x % kASlots);  // x even: slot + 1 < kASlots
+          const uint32_t apar = (uint32_t)((x / kASlots) & 1);
+          const int st2 = st + 1 == kBStages ? 0 : st + 1;
+          const uint32_t bpar2 = (uint32_t)((st2 == 0 ? wrap + 1 : wrap) & 1);
+          if (!wait_full(&a_full[slot], apar) || !wait_full(&a_full[slot + 1], apar) ||
+              !wait_full(&b_full[st], (uint32_t)(wrap & 1)) || !wait_full(&b_full[st2], bpar2)) {
             fail(tqtc::kErrMmaWait);
             ok = false;
             break;
           }
           tqtc::tc_fence_after();
-          const uint64_t ahi = adesc0 + (uint64_t)(slot * (kASlotBytes >> 4)), alo = ahi + (4096u >> 4);
-          const uint64_t bhi = bdesc0 + (uint64_t)(st * (kGroupBytes >> 4)), blo = bhi + (uint64_t)(kStepBytes >> 4);
-          const uint32_t dcol = tbase + 256u * (uint32_t)db;
-          tqtc::mma_f16_ss(dcol, ahi, bhi, idesc, g > 0);  // A_hi B_hi
-          tqtc::mma_f16_ss(dcol, alo, bhi, idesc, true);   // A_lo B_hi
-          tqtc::mma_f16_ss(dcol, ahi, blo, idesc, true);   // A_hi B_lo
-          tqtc::mma_commit(&a_empty[slot]);
-          tqtc::mma_commit(&b_empty[st]);
-          if (++st == kBStages) {
-            st = 0;
-            ++wrap;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int sl = slot + h, sb = h ? st2 : st;
+            const uint64_t ahi = adesc0 + (uint64_t)(sl * (kASlotBytes >> 4)), alo = ahi + (4096u >> 4);
+            const uint64_t bhi = bdesc0 + (uint64_t)(sb * (kGroupBytes >> 4)), blo = bhi + (uint64_t)(kStepBytes >> 4);
+            tqtc::mma_f16_ss(dcol, ahi, bhi, idesc, g > 0 || h > 0);  // A_hi B_hi
+            tqtc::mma_f16_ss(dcol, alo, bhi, idesc, true);            // A_lo B_hi
+            tqtc::mma_f16_ss(dcol, ahi, blo, idesc, true);            // A_hi B_lo
           }
+          tqtc::mma_commit(&a_empty[slot]);
+          tqtc::mma_commit(&a_empty[slot + 1]);
+          tqtc::mma_commit(&b_empty[st]);
+          tqtc::mma_commit(&b_empty[st2]);
+          if (st2 == 0) ++wrap;
+          st = st2 + 1 == kBStages ? 0 : st2 + 1;
+          if (st == 0 && st2 != 0) ++wrap;
         }
         if (!ok) break;
         tqtc::mma_commit(&d_full[db]);
