@@ -77,6 +77,51 @@ __device__ __forceinline__ void mag_search(float a, const float* mt, int& m, flo
   }
 }
 
+// The same search, returning for each magnitude bit p the difference
+// dd[p] = a - (boundary compared for bit p) and the bit itself, mb[p] =
+// (dd[p] >= 0), i.e. a >= that boundary.  For finite a the sign bit of dd[p]
+// is the complement of mb[p]: a - t rounds to zero only when a == t, and then
+// to +0.
+template <int BITS>
+__device__ __forceinline__ void mag_diff(float a, const float* mt, float* dd, bool* mb, float& margin) {
+  if constexpr (BITS == 1) {
+    margin = a;
+  } else if constexpr (BITS == 2) {
+    dd[0] = a - mt[1];
+    mb[0] = dd[0] >= 0.f;
+    margin = fminf(a, fabsf(dd[0]));
+  } else if constexpr (BITS == 3) {
+    dd[1] = a - mt[2];
+    mb[1] = dd[1] >= 0.f;
+    dd[0] = a - (mb[1] ? mt[3] : mt[1]);
+    mb[0] = dd[0] >= 0.f;
+    margin = fminf(a, fminf(fabsf(dd[1]), fabsf(dd[0])));
+  } else {
+    dd[2] = a - mt[4];
+    mb[2] = dd[2] >= 0.f;
+    dd[1] = a - (mb[2] ? mt[6] : mt[2]);
+    mb[1] = dd[1] >= 0.f;
+    dd[0] = a - (mb[2] ? (mb[1] ? mt[7] : mt[5]) : (mb[1] ? mt[3] : mt[1]));
+    mb[0] = dd[0] >= 0.f;
+    margin = fminf(fminf(a, fabsf(dd[2])), fminf(fabsf(dd[1]), fabsf(dd[0])));
+  }
+}
+
+// Magnitude of the centroid of cell (mb) from ct[k] = nu * (k-th positive
+// centroid), by selects (BITS <= 3).
+template <int BITS>
+__device__ __forceinline__ float sel_cen(const bool* mb, const float* ct) {
+  if constexpr (BITS == 1) {
+    return ct[0];
+  } else if constexpr (BITS == 2) {
+    return mb[0] ? ct[1] : ct[0];
+  } else {
+    const float hi = mb[0] ? ct[3] : ct[2];
+    const float lo = mb[0] ? ct[1] : ct[0];
+    return mb[1] ? hi : lo;
+  }
+}
+
 __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
   const __half2 h = __floats2half2_rn(a, b);
   return *reinterpret_cast<const uint32_t*>(&h);
@@ -500,43 +545,81 @@ __global__ void __launch_bounds__(kRows * (D / 32), SK ? 1 : 2)
     frexp_e = max(-125, min(125, frexp_e));
     const float rscale = ldexpf(1.f, -frexp_e);
     float runmin = INFINITY, g2 = 0.f, cv2 = 0.f;
+    // centroid magnitudes nu * cen for the sketch's residual, picked by
+    // selects where the codebook has at most 4 positive cells
+    constexpr bool kSel0 = B0 <= 3, kSel1 = B1 <= 3;
+    float ct0[SK && kSel0 ? H0 : 1], ct1[SK && kSel1 ? H1 : 1];
+    if constexpr (SK && kSel0) {
+#pragma unroll
+      for (int k = 0; k < H0; ++k) ct0[k] = nu * qb.cen[0][H0 + k];
+    }
+    if constexpr (SK && kSel1 && B1 > 0) {
+#pragma unroll
+      for (int k = 0; k < H1; ++k) ct1[k] = nu * qb.cen[1][H1 + k];
+    }
     unsigned char* crow = reinterpret_cast<unsigned char*>(st_codes + r * W);
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const int c = q + TPR * k;
       const bool seg1 = NSEG == 2 && c >= CHSEG;
       const int cs = seg1 ? c - CHSEG : c;
+      // Plane bits are gathered most recent first with funnel shifts of sign
+      // bits (value e ends at bit 7 - e, reversed below): plane p below the
+      // top is (mag bit p) xor (w < 0), the sign bit of dd[p] ^ w inverted;
+      // the top plane is w >= 0, the sign bit of w inverted.  A coordinate
+      // with w == -0 has a == 0, so its row fails the margin test and is
+      // recomputed exactly; the sign bit stands for w < 0 everywhere else.
       uint32_t pb[4] = {0u, 0u, 0u, 0u};
       float rr[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         const float w = v[8 * k + e];
         const float a = fabsf(w);
-        const bool pos = w >= 0.f;
-        int mc;
+        const uint32_t wu = __float_as_uint(w);
+        float dd[3];
+        bool mb[3];
         float margin;
         if (seg1) {
-          mag_search<(B1 > 0 ? B1 : 1)>(a, mt1, mc, margin);
+          mag_diff<(B1 > 0 ? B1 : 1)>(a, mt1, dd, mb, margin);
         } else {
-          mag_search<B0>(a, mt0, mc, margin);
+          mag_diff<B0>(a, mt0, dd, mb, margin);
         }
         runmin = fminf(runmin, fmaf(-Bc, a, margin));
         const int bits = seg1 ? B1 : B0;
 #pragma unroll
         for (int pl = 0; pl < 4; ++pl) {
-          if (pl < bits) {
-            const bool b = (pl == bits - 1) ? pos : ((((mc >> pl) & 1) != 0) != !pos);
-            pb[pl] |= (b ? 1u : 0u) << e;
-          }
+          if (pl < bits - 1) pb[pl] = __funnelshift_l(__float_as_uint(dd[pl]) ^ wu, pb[pl], 1);
+          if (pl == bits - 1) pb[pl] = __funnelshift_l(wu, pb[pl], 1);
         }
         if constexpr (SK) {
-          const float cvv = nu * (seg1 ? qb.cen[1][H1 + mc] : qb.cen[0][H0 + mc]);
+          float cvv;
+          if (seg1) {
+            if constexpr (kSel1) {
+              cvv = sel_cen<(B1 > 0 ? B1 : 1)>(mb, ct1);
+            } else {
+              int mc = 0;
+#pragma unroll
+              for (int b = 0; b < (B1 > 0 ? B1 : 1) - 1; ++b) mc |= (mb[b] ? 1 : 0) << b;
+              cvv = nu * qb.cen[1][H1 + mc];
+            }
+          } else {
+            if constexpr (kSel0) {
+              cvv = sel_cen<B0>(mb, ct0);
+            } else {
+              int mc = 0;
+#pragma unroll
+              for (int b = 0; b < B0 - 1; ++b) mc |= (mb[b] ? 1 : 0) << b;
+              cvv = nu * qb.cen[0][H0 + mc];
+            }
+          }
           const float rv = w - copysignf(cvv, w);
           g2 = fmaf(rv, rv, g2);
           cv2 = fmaf(cvv, cvv, cv2);
           rr[e] = rv * rscale;
         }
       }
+#pragma unroll
+      for (int pl = 0; pl < 4; ++pl) pb[pl] = (__brev(pb[pl]) >> 24) ^ 0xFFu;
       const int bits = seg1 ? B1 : B0;
       const int wbase = seg1 ? B0 * PW : 0;
 #pragma unroll
@@ -639,15 +722,27 @@ __global__ void __launch_bounds__(kRows * (D / 32), SK ? 1 : 2)
           tqtc::tmem_ld16(tqtc::tmem_addr(tbase, 32u * lq, (uint32_t)m + 32u * c + 16u), u16[1]);
         }
         tqtc::tmem_wait_ld();
-        uint32_t word = 0, unsure = 0;
+        // sign bits gathered most recent first (bit jj ends at 31 - jj):
+        // neg: t < 0; sure: |t| > tau, i.e. tau - |t| < 0.  A bit with
+        // |t| <= tau (t == -0 among them) is marked uncertain and recomputed
+        // exactly, so the sign bit of t stands for t < 0 on every bit kept.
+        uint32_t neg = 0, sure = 0;
+        const float4* sl4 = reinterpret_cast<const float4*>(smem + ly.sl2n) + 8 * c;
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) {
-          float t = __uint_as_float(t16[jj >> 4][jj & 15]);
-          if (m <= 128) t += __uint_as_float(u16[jj >> 4][jj & 15]);
-          const float tau = fmaf(reinterpret_cast<const float*>(smem + ly.sl2n)[32 * c + jj], eg.x, eg.y);
-          unsure |= (fabsf(t) > tau ? 0u : 1u) << jj;
-          word |= (t >= 0.f ? 1u : 0u) << jj;
+        for (int j4 = 0; j4 < 8; ++j4) {
+          const float4 s4 = sl4[j4];
+          const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int jj = 4 * j4 + i;
+            float t = __uint_as_float(t16[jj >> 4][jj & 15]);
+            if (m <= 128) t += __uint_as_float(u16[jj >> 4][jj & 15]);
+            const float tau = fmaf(sv[i], eg.x, eg.y);
+            neg = __funnelshift_l(__float_as_uint(t), neg, 1);
+            sure = __funnelshift_l(__float_as_uint(tau - fabsf(t)), sure, 1);
+          }
         }
+        const uint32_t word = ~__brev(neg), unsure = ~__brev(sure);
         st_signs[rr * 8 + c] = word;
         st_fmask[rr * 8 + c] = unsure;
         if (unsure && row0 + rr < n) atomicOr(&st_flag[rr], 1);
