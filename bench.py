@@ -44,15 +44,16 @@ FALLBACK_HBM_GBS = 6650.0
 # ------------------------------------------------------------------ helpers
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of
 # each stage's main kernel, from the ncu captures summarised in
-# profiles/kernels_llama8b_decode_step.md (the quantise kernels from the
-# later counter capture listed there).  It is reported only while the kernel
-# sources are the ones those captures measured (same source digest); after
-# any change to them the field is null until the capture is redone.
-TRAFFIC_SOURCES = "72362dc037274f4ae0ba8c7c15be62d73933dfbfcdd668112d36270b25a75866"
+# profiles/kernels_llama8b_decode_step.md (the quantise kernels and the
+# scorer from the later counter captures listed there).  It is reported only
+# while the kernel sources are the ones those captures measured (same source
+# digest); after any change to them the field is null until the capture is
+# redone.
+TRAFFIC_SOURCES = "cd73e2b3dcd830cc9c462f5573d37656dfa16f88cfa03b00cb1f6738003aa0c8"
 TRAFFIC = {
     "tq_quantize_K": 548_016_384 + 136_585_984,
     "tq_quantize_V": 539_167_744 + 124_734_208,
-    "tq_scores": 152_022_016 + 19_559_168,
+    "tq_scores": 151_660_288 + 19_469_568,
     "tq_attend": 293_933_056 + 6_545_152,
 }
 

@@ -17,6 +17,18 @@
 // holds round(v_k 2^(e - r)) split into four balanced base-256 s8 limbs, in
 // shared memory.  The s32 accumulation is exact; the epilogue rebuilds
 // I = sum_l 256^l D_l, scales by 2^-e and subtracts corr.
+//
+// Centroid-limb form (one segment of 3-bit codes): the plane identity needs
+// four odd plane subsets (16 source words at d = 128), one byte of K per
+// key bit.  Instead each coordinate's centroid, as the 16-bit fixed point
+// C = rint(cen * 2^f) split into two balanced s8 limbs, takes two bytes of
+// K: 8 source words for the first term, and 12 MMAs per tile in place of
+// 20.  Limb h of a word's 32 centroids goes to its own accumulator D_h
+// (the query image is the same for both), and the epilogue forms
+// sum_l 256^l (D_0l + 256 D_1l) 2^-(e+f).  The fixed point is the one
+// approximation: |cen - C 2^-f| <= 2^-(f+1) per coordinate, f = 13 for the
+// 3-bit codebooks (max |cen| < 4), so the first term moves by at most
+// 2^-14 ||q'||_1 / sqrt(d) <= 2^-14 ||q||.
 #include <math.h>
 
 #include <algorithm>
@@ -37,11 +49,27 @@ __host__ __device__ constexpr int term_mask(int bits, int t) {
 
 __host__ __device__ inline int ncols_for(int G) { return ((4 * G + 15) / 16) * 16; }
 
+// the centroid-limb form applies to one segment of 3-bit codes
+__host__ __device__ inline bool use_cl(const tq_params& p) { return p.nseg == 1 && p.bits[0] == 3; }
+
+// fixed-point exponent f of the centroid limbs: the largest f with
+// max |cen| * 2^f <= 32512, so that both balanced s8 limbs stay in range
+__host__ __device__ inline int cl_shift(const tq_params& p) {
+  int ex = 0;
+  frexpf(p.cmax > 0.f ? p.cmax : 1.f, &ex);  // cmax < 2^ex
+  int f = 15 - ex;
+  if (ldexpf(p.cmax, f) > 32512.f) --f;
+  return f;
+}
+
 struct Geom {
   int U_mse, U, Kt, N, G, lbo, bbytes, gstride;
+  bool cl;
   __host__ __device__ Geom(const tq_params& p, int G_) {
+    cl = use_cl(p);
     U_mse = 0;
     for (int s = 0; s < p.nseg; ++s) U_mse += p.nterms[s] * p.pw;
+    if (cl) U_mse = 2 * p.pw;
     U = U_mse + p.MS;
     Kt = 32 * U;
     G = G_;
@@ -80,8 +108,12 @@ __global__ void __launch_bounds__(256) tq_scores_bbuild_kernel(const tq_params p
       }
       qmax = tq_warp_max(qmax);
       qsum = tq_warp_sum(qsum);
-      mx = fmaxf(mx, 2.f * amax * qmax);
-      corr += asum * qsum;
+      if (g.cl) {
+        mx = qmax;  // centroid limbs: the image holds q' itself, no correction
+      } else {
+        mx = fmaxf(mx, 2.f * amax * qmax);
+        corr += asum * qsum;
+      }
     }
     float wmax = 0.f, wsum = 0.f;
     for (int j = lane; j < m; j += 32) {
@@ -119,8 +151,13 @@ __global__ void __launch_bounds__(256) tq_scores_bbuild_kernel(const tq_params p
       const float* qv = qprep + (size_t)(b * Hq + hk * g.G + gq) * (d + m);
       const int u = k / 32, r = (k % 32) / 4, j = k % 4, bp = r + 8 * j;
       float v;
-      int e;
-      if (u < g.U_mse) {
+      int e, sh = r;
+      if (u < g.U_mse && g.cl) {
+        // both limb slots of word u % pw: byte k % 32 is coordinate k % 32
+        v = qv[32 * (u % p.pw) + k % 32];
+        e = s_xmse[gq];
+        sh = 0;
+      } else if (u < g.U_mse) {
         const int s = (p.nseg == 2 && u >= u0) ? 1 : 0;
         const int uu = s ? u - u0 : u;
         const int t = uu / p.pw, w = uu % p.pw;
@@ -130,7 +167,7 @@ __global__ void __launch_bounds__(256) tq_scores_bbuild_kernel(const tq_params p
         v = 2.f * qv[d + 32 * (u - g.U_mse) + bp];
         e = s_xqjl[gq];
       }
-      int x = __float2int_rn(ldexpf(v, e - r));
+      int x = __float2int_rn(ldexpf(v, e - sh));
       // balanced base-256 digits
       int lv = 0;
 #pragma unroll
@@ -174,7 +211,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int W = (B0 + B1) * PW;
   constexpr int NT0 = B0 == 1 ? 1 : B0 == 2 ? 2 : B0 == 3 ? 4 : 8;
   constexpr int NT1 = B1 == 0 ? 0 : B1 == 1 ? 1 : B1 == 2 ? 2 : B1 == 3 ? 4 : 8;
-  constexpr int U_MSE = (NT0 + NT1) * PW;
+  constexpr bool CL = B0 == 3 && B1 == 0;  // centroid-limb form (use_cl)
+  constexpr int U_MSE = CL ? 2 * PW : (NT0 + NT1) * PW;
 
   extern __shared__ __align__(1024) unsigned char smem[];
   __shared__ uint64_t ring_full[kStages], ring_empty[kStages];
@@ -189,7 +227,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   unsigned char* bbuf = smem;                                     // [2][bstride]
   unsigned char* ring = smem + 2 * bstride;                       // [kStages][ring_stage_bytes]
   const int sbytes = ring_stage_bytes(W, MS);
-  const uint32_t acols = 8u * (uint32_t)g.U, dcols = 2u * (uint32_t)g.N;
+  // centroid-limb tables, indexed by the three plane nibbles of four
+  // coordinates (n0 | n1 << 4 | n2 << 8): byte j of entry h is limb h of the
+  // centroid of coordinate j (code bits: bit j of n0, n1, n2)
+  uint32_t* lut = reinterpret_cast<uint32_t*>(ring + (RING ? kStages * sbytes : 0));  // [2][4096]
+  const uint32_t acols = 8u * (uint32_t)g.U, dcols = (CL ? 3u : 2u) * (uint32_t)g.N;
 
   const int64_t t_begin = (int64_t)blockIdx.x * ntiles / gridDim.x;
   const int64_t t_end = (int64_t)(blockIdx.x + 1) * ntiles / gridDim.x;
@@ -212,6 +254,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     s_abort = 0;
   }
   if (warp == 0) tqtc::tmem_alloc(&s_tmem, 512);
+  if constexpr (CL) {
+    const float sc = ldexpf(1.f, cl_shift(p));
+    for (int i = tid; i < 4096; i += kThreads) {
+      uint32_t l0 = 0u, l1 = 0u;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int code = ((i >> j) & 1) | (((i >> (4 + j)) & 1) << 1) | (((i >> (8 + j)) & 1) << 2);
+        const int c = __float2int_rn(p.cen[0][code] * sc);
+        const int h0 = (int)(int8_t)(c & 0xFF), h1 = (c - h0) >> 8;
+        l0 |= (uint32_t)(h0 & 0xFF) << (8 * j);
+        l1 |= (uint32_t)(h1 & 0xFF) << (8 * j);
+      }
+      lut[i] = l0;
+      lut[4096 + i] = l1;
+    }
+  }
   tqtc::tc_fence_before();
   __syncthreads();
   tqtc::tc_fence_after();
@@ -269,7 +327,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 9) {
     // ---------------------------------------------------------- MMA issue
     if (lane == 0) {
-      const uint32_t idesc = tqtc::instr_desc(2, 0, 1, kKeys, (uint32_t)g.N);
+      const uint32_t idesc = tqtc::instr_desc(2, 0, 1, kKeys, (uint32_t)g.N);     // A u8, B s8
+      const uint32_t idesc_s8 = tqtc::instr_desc(2, 1, 1, kKeys, (uint32_t)g.N);  // A s8, B s8
       int64_t cur = -1;
       int gi = -1;
       for (int64_t i = 0; i < ntl && !s_abort; ++i) {
@@ -298,10 +357,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t d_mse = tbase + 2u * acols + (uint32_t)b * dcols, d_qjl = d_mse + (uint32_t)g.N;
         uint64_t desc = tqtc::smem_desc(tqtc::smem_u32(bbuf + (gi & 1) * bstride), (uint32_t)g.lbo, 128);
         const uint64_t step = (uint64_t)((2u * (uint32_t)g.lbo) >> 4);
-        for (int u = 0; u < g.U; ++u) {
-          const bool qjl = u >= g.U_mse;
-          tqtc::mma_i8_ts(qjl ? d_qjl : d_mse, a0 + 8u * (uint32_t)u, desc, idesc, !(u == 0 || u == g.U_mse));
-          desc += step;
+        if constexpr (CL) {
+          // limb 0 words -> D_0, limb 1 words -> D_1 (signed limbs: A is s8),
+          // sign words -> D_qjl (masked bytes up to 128: A is u8)
+          for (int u = 0; u < g.U; ++u) {
+            const uint32_t dst = u < PW ? d_mse : u < U_MSE ? d_mse + (uint32_t)g.N : d_mse + 2u * (uint32_t)g.N;
+            tqtc::mma_i8_ts(dst, a0 + 8u * (uint32_t)u, desc, u < U_MSE ? idesc_s8 : idesc,
+                            !(u == 0 || u == PW || u == U_MSE));
+            desc += step;
+          }
+        } else {
+          for (int u = 0; u < g.U; ++u) {
+            const bool qjl = u >= g.U_mse;
+            tqtc::mma_i8_ts(qjl ? d_qjl : d_mse, a0 + 8u * (uint32_t)u, desc, idesc, !(u == 0 || u == g.U_mse));
+            desc += step;
+          }
         }
         tqtc::mma_commit(&mma_done[b]);
       }
@@ -375,6 +445,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int r = 0; r < 8; ++r) regs[r] = word & (0x01010101u << r);
         tqtc::tmem_st8(tqtc::tmem_addr(tbase, lane_base, a0 + 8u * (uint32_t)u), regs);
       };
+      if constexpr (CL) {
+#pragma unroll
+        for (int w = 0; w < PW; ++w) {
+          uint32_t r0[8], r1[8];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint32_t ix = ((kcw[w] >> (4 * c)) & 0xFu) | (((kcw[PW + w] >> (4 * c)) & 0xFu) << 4) |
+                                (((kcw[2 * PW + w] >> (4 * c)) & 0xFu) << 8);
+            r0[c] = lut[ix];
+            r1[c] = lut[4096 + ix];
+          }
+          tqtc::tmem_st8(tqtc::tmem_addr(tbase, lane_base, a0 + 8u * (uint32_t)w), r0);
+          tqtc::tmem_st8(tqtc::tmem_addr(tbase, lane_base, a0 + 8u * (uint32_t)(PW + w)), r1);
+        }
+      } else {
 #pragma unroll
       for (int s = 0; s < NSEG; ++s) {
         const int bits = s ? B1 : B0;
@@ -396,6 +481,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      }
 #pragma unroll
       for (int k = 0; k < 8; ++k)
         if (k < MS) emit(U_MSE + k, ksw[k]);
@@ -407,6 +493,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------- epilogue (warps 4-7)
     const int et = tid - 128;
     const uint32_t lane_base = 32u * (uint32_t)(warp - 4);
+    const float kcl = CL ? ldexpf(p.inv_sqrt_d, -cl_shift(p)) : 0.f;  // 2^-f / sqrt(d)
     for (int64_t i = 0; i < ntl; ++i) {
       const int64_t tile = t_begin + i;
       const int64_t grp = tile / tiles_per_group;
@@ -423,12 +510,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tqtc::tc_fence_after();
-      const uint32_t d_mse = 2u * acols + (uint32_t)b * dcols, d_qjl = d_mse + (uint32_t)g.N;
+      const uint32_t d_mse = 2u * acols + (uint32_t)b * dcols;
+      const uint32_t d_qjl = d_mse + (CL ? 2u : 1u) * (uint32_t)g.N;
       const int bq = (int)(grp / Hkv), hk = (int)(grp % Hkv);
       const float cq = kgam * p.qjl_coef;
       for (int qc = 0; qc < g.N / 16; ++qc) {
-        uint32_t dm[16], dq[16];
+        uint32_t dm[16], dq[16], dm1[16];
         tqtc::tmem_ld16(tqtc::tmem_addr(tbase, lane_base, d_mse + 16u * qc), dm);
+        if (CL) tqtc::tmem_ld16(tqtc::tmem_addr(tbase, lane_base, d_mse + (uint32_t)g.N + 16u * qc), dm1);
         if (MS > 0) tqtc::tmem_ld16(tqtc::tmem_addr(tbase, lane_base, d_qjl + 16u * qc), dq);
         tqtc::tmem_wait_ld();
         if (qc == g.N / 16 - 1) {
@@ -440,11 +529,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int gq = 4 * qc + g4;
           if (gq < g.G && valid) {
             const float4 cs = __ldg(reinterpret_cast<const float4*>(cs_all) + gq);
-            float im = (float)(int)dm[4 * g4 + 3];
-            im = fmaf(im, 256.f, (float)(int)dm[4 * g4 + 2]);
-            im = fmaf(im, 256.f, (float)(int)dm[4 * g4 + 1]);
-            im = fmaf(im, 256.f, (float)(int)dm[4 * g4 + 0]);
-            float val = fmaf(im, cs.x, -cs.y) * p.inv_sqrt_d;
+            float val;
+            if constexpr (CL) {
+              // per query limb l: D_0l + 256 D_1l
+              float t4[4];
+#pragma unroll
+              for (int l = 0; l < 4; ++l) t4[l] = fmaf((float)(int)dm1[4 * g4 + l], 256.f, (float)(int)dm[4 * g4 + l]);
+              float im = t4[3];
+              im = fmaf(im, 256.f, t4[2]);
+              im = fmaf(im, 256.f, t4[1]);
+              im = fmaf(im, 256.f, t4[0]);
+              val = (im * cs.x) * kcl;
+            } else {
+              float im = (float)(int)dm[4 * g4 + 3];
+              im = fmaf(im, 256.f, (float)(int)dm[4 * g4 + 2]);
+              im = fmaf(im, 256.f, (float)(int)dm[4 * g4 + 1]);
+              im = fmaf(im, 256.f, (float)(int)dm[4 * g4 + 0]);
+              val = fmaf(im, cs.x, -cs.y) * p.inv_sqrt_d;
+            }
             if (MS > 0) {
               float iq = (float)(int)dq[4 * g4 + 3];
               iq = fmaf(iq, 256.f, (float)(int)dq[4 * g4 + 2]);
@@ -492,7 +594,7 @@ bool supported(const tq_params& p, int G, uint32_t* cols_out) {
   if (!(p.nseg == 1 || (p.bits[0] == 2 && p.bits[1] == 3))) return false;
   const Geom g(p, G);
   if (g.bbytes > 64 * 1024 || g.N > 128) return false;
-  const uint32_t need = 2u * (8u * g.U + 2u * g.N);  // double-buffered A and accumulators
+  const uint32_t need = 2u * (8u * g.U + (g.cl ? 3u : 2u) * g.N);  // double-buffered A and accumulators
   if (need > 512) return false;
   if (cols_out) *cols_out = 512;
   return true;
@@ -505,6 +607,7 @@ cudaError_t launch_scores_t(const tq_params& p, const tq_compressed& K, float* l
   const Geom g(p, Hq / Hkv);
   const size_t bstride = (size_t)((g.bbytes + 16 * g.G + 127) / 128) * 128;
   size_t smem = 2 * bstride + (RING ? (size_t)kStages * ring_stage_bytes(W, p.MS) : 0);
+  if (B0 == 3 && B1 == 0) smem += 2 * 4096 * sizeof(uint32_t);  // centroid-limb tables
   // the block takes all 512 TMEM columns: ask for more than half of the SM's
   // shared memory so that a second block never waits on the allocation
   smem = std::max(smem, (size_t)(smem_per_sm() / 2 + 1024));
