@@ -44,42 +44,46 @@ FALLBACK_HBM_GBS = 6650.0
 # ------------------------------------------------------------------ helpers
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of
 # each stage's main kernel, from the ncu captures summarised in
-# profiles/kernels_llama8b_decode_step.md (the quantise kernels and the
-# scorer from the later counter captures listed there).  It is reported only
-# while the kernel sources are the ones those captures measured (same source
-# digest); after any change to them the field is null until the capture is
-# redone.
-TRAFFIC_SOURCES = "cd73e2b3dcd830cc9c462f5573d37656dfa16f88cfa03b00cb1f6738003aa0c8"
-TRAFFIC = {
-    "tq_quantize_K": 548_016_384 + 136_585_984,
-    "tq_quantize_V": 539_167_744 + 124_734_208,
-    "tq_scores": 151_660_288 + 19_469_568,
-    "tq_attend": 293_933_056 + 6_545_152,
+# profiles/kernels_llama8b_decode_step.md, with the digest of the sources that
+# capture measured.  A stage's figure is reported only while its sources (its
+# kernel file plus the shared headers and host dispatch) still have that
+# digest; after any change to them it is null until the capture is redone.
+STEP_SHARED_SOURCES = ("tq_common.cuh", "tq_internal.h", "tq_tc.cuh", "tq_host.cpp", "tq_kernels.cu")
+STAGE_SOURCES = {
+    "tq_quantize_K": ("tq_quantize_tc.cu",),
+    "tq_quantize_V": ("tq_quantize_tc.cu",),
+    "tq_scores": ("tq_scores_tc.cu",),
+    "tq_attend": ("tq_attend.cuh", "tq_attend_d128.cu", "tq_attend_d64.cu"),
+}
+TRAFFIC = {  # stage: (bytes per launch, sources digest)
+    "tq_quantize_K": (548_016_384 + 136_585_984, "134db91880981d6bf9577980f98eb19c8d300b2ba4917ec31a7c3579ef3e9810"),
+    "tq_quantize_V": (539_167_744 + 124_734_208, "134db91880981d6bf9577980f98eb19c8d300b2ba4917ec31a7c3579ef3e9810"),
+    "tq_scores": (151_660_288 + 19_469_568, "cde1354c9006cd646724007cce67eb21b5b68e4f8afe0cb7f8e4b1f81f30f215"),
+    "tq_attend": (293_933_056 + 6_545_152, "cd88a868af76721130abf3b3cb72257c0c64db14a686b803d138aa8394b43c6c"),
 }
 
 
-# the sources of the decode step's kernels (the search and no-allocation
-# entry points are not part of the step)
-STEP_SOURCES_EXCLUDED = ("tq_search.cu", "tq_noalloc.cu")
-
-
-def kernel_sources_digest() -> str:
-    """sha256 over the decode step's kernel and header sources (names + bytes)."""
+def stage_sources_digest(stage: str) -> str:
+    """sha256 over a stage's kernel sources, the shared headers, the host
+    dispatch and tq.h (names + bytes)."""
     import hashlib
     csrc = os.path.join(ROOT, "kv_cache_vector_09_b200", "csrc")
     h = hashlib.sha256()
-    for n in sorted(os.listdir(csrc)):
-        if n.endswith((".cu", ".cuh", ".h", ".cpp")) and n not in STEP_SOURCES_EXCLUDED:
-            h.update(n.encode())
-            with open(os.path.join(csrc, n), "rb") as f:
-                h.update(f.read())
+    for n in sorted(STEP_SHARED_SOURCES + STAGE_SOURCES[stage]):
+        h.update(n.encode())
+        with open(os.path.join(csrc, n), "rb") as f:
+            h.update(f.read())
     with open(os.path.join(ROOT, "include", "tq.h"), "rb") as f:
         h.update(f.read())
     return h.hexdigest()
 
 
 def measured_traffic(stage: str):
-    return TRAFFIC.get(stage) if kernel_sources_digest() == TRAFFIC_SOURCES else None
+    if stage not in TRAFFIC:
+        return None
+    nbytes, digest = TRAFFIC[stage]
+    return nbytes if stage_sources_digest(stage) == digest else None
+
 
 
 def load_peaks():
