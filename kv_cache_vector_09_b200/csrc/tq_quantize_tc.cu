@@ -47,41 +47,14 @@ struct QBook {
   float bnd[2][TQ_MAX_LEVELS];
 };
 
-// Magnitude search: a = |w|, mt[k] = nu * (k-th positive boundary), k >= 1.
-// Returns the cell m and the distance to the nearest compared boundary (the
-// zero boundary included); the compared boundaries include both ends of the
-// final cell.
-template <int BITS>
-__device__ __forceinline__ void mag_search(float a, const float* mt, int& m, float& margin) {
-  if constexpr (BITS == 1) {
-    m = 0;
-    margin = a;
-  } else if constexpr (BITS == 2) {
-    const bool c = a >= mt[1];
-    m = c;
-    margin = fminf(a, fabsf(a - mt[1]));
-  } else if constexpr (BITS == 3) {
-    const bool m1 = a >= mt[2];
-    const float t = m1 ? mt[3] : mt[1];
-    const bool m0 = a >= t;
-    m = (m1 << 1) | m0;
-    margin = fminf(a, fminf(fabsf(a - mt[2]), fabsf(a - t)));
-  } else {
-    const bool m2 = a >= mt[4];
-    const float t1 = m2 ? mt[6] : mt[2];
-    const bool m1 = a >= t1;
-    const float t0 = m2 ? (m1 ? mt[7] : mt[5]) : (m1 ? mt[3] : mt[1]);
-    const bool m0 = a >= t0;
-    m = (m2 << 2) | (m1 << 1) | m0;
-    margin = fminf(fminf(a, fabsf(a - mt[4])), fminf(fabsf(a - t1), fabsf(a - t0)));
-  }
-}
-
-// The same search, returning for each magnitude bit p the difference
-// dd[p] = a - (boundary compared for bit p) and the bit itself, mb[p] =
-// (dd[p] >= 0), i.e. a >= that boundary.  For finite a the sign bit of dd[p]
-// is the complement of mb[p]: a - t rounds to zero only when a == t, and then
-// to +0.
+// Magnitude search: a = |w|, mt[k] = nu * (k-th positive boundary), k >= 1,
+// one binary-search step per magnitude bit.  Returns the distance to the
+// nearest compared boundary (the zero boundary included; the compared
+// boundaries include both ends of the final cell) and, for each magnitude bit
+// p, the difference dd[p] = a - (boundary compared for bit p) and the bit
+// itself, mb[p] = (dd[p] >= 0), i.e. a >= that boundary.  For finite a the
+// sign bit of dd[p] is the complement of mb[p]: a - t rounds to zero only when
+// a == t, and then to +0.
 template <int BITS>
 __device__ __forceinline__ void mag_diff(float a, const float* mt, float* dd, bool* mb, float& margin) {
   if constexpr (BITS == 1) {
