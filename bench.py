@@ -56,8 +56,8 @@ STAGE_SOURCES = {
     "tq_attend": ("tq_attend.cuh", "tq_attend_d128.cu", "tq_attend_d64.cu"),
 }
 TRAFFIC = {  # stage: (bytes per launch, sources digest)
-    "tq_quantize_K": (548_016_384 + 136_585_984, "babdb167626d9c5aa1534d0e03567ad8628b32e17fbc2f461663f271efedfcdb"),
-    "tq_quantize_V": (539_167_744 + 124_734_208, "babdb167626d9c5aa1534d0e03567ad8628b32e17fbc2f461663f271efedfcdb"),
+    "tq_quantize_K": (548_016_384 + 136_585_984, "78bf5806cb23a39ab020d5264b7ac3b9b46bdf3210637d7f6c2aed8c21b993af"),
+    "tq_quantize_V": (539_167_744 + 124_734_208, "78bf5806cb23a39ab020d5264b7ac3b9b46bdf3210637d7f6c2aed8c21b993af"),
     "tq_scores": (151_660_288 + 19_469_568, "cde1354c9006cd646724007cce67eb21b5b68e4f8afe0cb7f8e4b1f81f30f215"),
     "tq_attend": (293_933_056 + 6_545_152, "cd88a868af76721130abf3b3cb72257c0c64db14a686b803d138aa8394b43c6c"),
 }

@@ -788,7 +788,9 @@ cudaError_t launch_quad(const tq_params& p, const void* x, int64_t n, int64_t ld
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ly.total);
   if (e != cudaSuccess) return e;
   uint32_t cols = 32;  // accumulator: 2m columns when the sketch uses the merged N = 2m product
-  while (cols < (uint32_t)(m <= 128 ? 2 * m : m)) cols <<= 1;
+  if constexpr (SK) {
+    while (cols < (uint32_t)(m <= 128 ? 2 * m : m)) cols <<= 1;
+  }
   int per_sm = 0;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, NT, ly.total);
   if (e != cudaSuccess) return e;
