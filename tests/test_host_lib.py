@@ -127,3 +127,28 @@ def test_bench_search_batches_follow_the_library_rule():
     assert b.search_batches(768, 10) == 1
     assert b.search_batches(300, 32) == 2
     assert b.search_batches(1, 1) == 1
+
+
+def test_bench_traffic_is_reported_only_for_the_measured_sources(monkeypatch):
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("bench_mod2", os.path.join(ROOT, "bench.py"))
+    b = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(b)
+    stages = sorted(b.STAGE_SOURCES)
+    assert stages == sorted(b.TRAFFIC)
+    # every stage's digest covers its own kernel file and the shared sources
+    for st in stages:
+        for n in b.STAGE_SOURCES[st] + b.STEP_SHARED_SOURCES:
+            assert os.path.exists(os.path.join(ROOT, "kv_cache_vector_09_b200", "csrc", n)), n
+    # a figure recorded against the current sources is reported, one recorded
+    # against other sources is not, and one stage's digest does not gate another
+    cur = {st: b.stage_sources_digest(st) for st in stages}
+    monkeypatch.setattr(b, "TRAFFIC", {st: (1000 + i, cur[st]) for i, st in enumerate(stages)})
+    assert [b.measured_traffic(st) for st in stages] == [1000 + i for i in range(len(stages))]
+    stale = dict(b.TRAFFIC)
+    stale["tq_scores"] = (7, "0" * 64)
+    monkeypatch.setattr(b, "TRAFFIC", stale)
+    assert b.measured_traffic("tq_scores") is None
+    assert b.measured_traffic("tq_attend") == stale["tq_attend"][0]
+    assert b.measured_traffic("no_such_stage") is None
+    assert cur["tq_scores"] != cur["tq_attend"]
