@@ -13,6 +13,7 @@
 #include <vector>
 
 #include "tq_internal.h"
+#include "tq_trace.h"
 
 namespace {
 
@@ -196,6 +197,7 @@ static tq_status lloyd_max(int bits, int d, double tol, int max_iter, std::vecto
 
 extern "C" tq_status tq_make_codebook(int bits, int d, double tol, int max_iter, float* centroids,
                                       float* boundaries) {
+  const tqtrace::Range trace("tq_make_codebook");
   if (bits < 1 || bits > 4) return tq_fail(TQ_ERR_INVALID_ARG, "bits must be 1..4 (got %d)", bits);
   if (d < 4) return tq_fail(TQ_ERR_INVALID_ARG, "d must be >= 4 (got %d)", d);
   if (!centroids || !boundaries) return tq_fail(TQ_ERR_INVALID_ARG, "null output pointer");
@@ -230,6 +232,7 @@ static tq_status check_spec(const tq_spec* s) {
 static size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 extern "C" tq_status tq_codec_create(const tq_spec* spec, int device, tq_codec** out) {
+  const tqtrace::Range trace("tq_codec_create");
   tq_status st = check_spec(spec);
   if (st != TQ_OK) return st;
   if (!out) return tq_fail(TQ_ERR_INVALID_ARG, "null output pointer");
@@ -480,6 +483,7 @@ static tq_status launch_status(cudaError_t e, const char* what) {
 
 extern "C" tq_status tq_quantize(const tq_codec* c, const void* x, tq_dtype dt, int64_t n, int64_t ld,
                                  const tq_compressed* out, void* stream) {
+  const tqtrace::Range trace("tq_quantize");
   tq_status st = check_device_codec(c, "tq_quantize");
   if (st != TQ_OK) return st;
   if ((st = check_dtype(dt)) != TQ_OK) return st;
@@ -522,6 +526,7 @@ static tq_status check_heads(int B, int Hq, int Hkv, int64_t T, const char* name
 extern "C" tq_status tq_scores(const tq_codec* kc, const void* q, tq_dtype dt, int B, int Hq, int Hkv, int64_t T,
                                const tq_compressed* K, float* logits, void* workspace, size_t ws_bytes,
                                void* stream) {
+  const tqtrace::Range trace("tq_scores");
   tq_status st = check_device_codec(kc, "tq_scores");
   if (st != TQ_OK) return st;
   if ((st = check_dtype(dt)) != TQ_OK) return st;
@@ -567,6 +572,7 @@ extern "C" tq_status tq_attend_workspace_size(const tq_codec* kc, const tq_codec
 extern "C" tq_status tq_attend(const tq_codec* kc, const tq_codec* vc, const void* q, tq_dtype dt, int B, int Hq,
                                int Hkv, int64_t T, float scale, const tq_compressed* K, const tq_compressed* V,
                                void* workspace, size_t ws_bytes, float* out, void* stream) {
+  const tqtrace::Range trace("tq_attend");
   tq_status st = check_device_codec(kc, "tq_attend");
   if (st != TQ_OK) return st;
   if ((st = check_device_codec(vc, "tq_attend")) != TQ_OK) return st;
@@ -617,6 +623,7 @@ extern "C" tq_status tq_search_workspace_size(const tq_codec* c, int nq, int k, 
 extern "C" tq_status tq_search_topk(const tq_codec* c, const void* q, tq_dtype dt, int nq, const tq_compressed* X,
                                     int64_t n, int k, int32_t* idx, float* score, void* workspace, size_t ws_bytes,
                                     void* stream) {
+  const tqtrace::Range trace("tq_search_topk");
   tq_status st = check_device_codec(c, "tq_search_topk");
   if (st != TQ_OK) return st;
   if ((st = check_search_codec(c, "tq_search_topk")) != TQ_OK) return st;

@@ -27,6 +27,7 @@
 #include <mutex>
 
 #include "tq_internal.h"
+#include "tq_trace.h"
 
 #define TQ_SCORES_NOALLOC_SCRATCH (2u << 20)  // 2 MiB
 #define TQ_NOALLOC_MAX_DEVICES 64
@@ -57,6 +58,7 @@ tq_status scratch_address(int device, void** out) {
 
 extern "C" tq_status tq_scores_noalloc(const tq_codec* kc, const void* q, tq_dtype dtype, int B, int Hq, int Hkv,
                                        int64_t T, const tq_compressed* K, float* logits, void* stream) {
+  const tqtrace::Range trace("tq_scores_noalloc");
   if (!kc) return tq_fail(TQ_ERR_INVALID_ARG, "tq_scores_noalloc: null codec");
   if (kc->device < 0) return tq_fail(TQ_ERR_INVALID_ARG, "tq_scores_noalloc: host-only codec");
   size_t need = 0;
