@@ -43,9 +43,8 @@ FALLBACK_HBM_GBS = 6650.0
 
 # ------------------------------------------------------------------ helpers
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of
-# each stage's main kernel, from the ncu captures summarised in
-# profiles/kernels_llama8b_decode_step.md, with the digest of the sources that
-# capture measured.  A stage's figure is reported only while its sources (its
+# each stage's main kernel, from an ncu capture of that kernel, with the digest
+# of the sources that capture measured.  A stage's figure is reported only while its sources (its
 # kernel file plus the shared headers and host dispatch) still have that
 # digest; after any change to them it is null until the capture is redone.
 STEP_SHARED_SOURCES = ("tq_common.cuh", "tq_internal.h", "tq_tc.cuh", "tq_host.cpp", "tq_kernels.cu", "tq_trace.h")

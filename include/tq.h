@@ -191,7 +191,9 @@ TQ_API tq_status tq_scores(const tq_codec *kc, const void *q, tq_dtype dtype, in
  *   - Calls needing more scratch than that (tq_scores_workspace_size(kc, B, Hq,
  *     Hkv) above 2 MiB) return TQ_ERR_UNSUPPORTED and write nothing.
  *   - The first call on a device looks up the array's device address; make it
- *     before any stream capture.
+ *     before any stream capture.  The address is cached for the life of the
+ *     process and does not survive a device reset (cudaDeviceReset): no
+ *     tq_scores_noalloc call may follow one in the same process.
  *   - Every call shares the one array: calls whose kernels may overlap on the
  *     GPU (other streams, other host threads) race and must be serialised.
  *   - It calls no allocator (no cudaMalloc, cudaFree or allocating library). */

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <climits>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -500,16 +501,24 @@ extern "C" tq_status tq_quantize(const tq_codec* c, const void* x, tq_dtype dt, 
   return launch_status(e, "tq_quantize launch");
 }
 
-static size_t qprep_bytes(const tq_params& p, int nq) { return align256(sizeof(float) * (size_t)nq * (p.d + p.m)); }
+static size_t qprep_bytes(const tq_params& p, size_t nq) { return align256(sizeof(float) * nq * (size_t)(p.d + p.m)); }
+
+// B * Hq (and B * Hkv) index query and head arrays with int arithmetic in the
+// kernels and the size helpers: larger products are refused.
+static bool heads_fit_int(int B, int Hq, int Hkv) {
+  return (int64_t)B * Hq <= INT_MAX && (int64_t)B * Hkv <= INT_MAX;
+}
 
 static size_t scores_bytes(const tq_params& p, int B, int Hq, int Hkv) {
-  return qprep_bytes(p, B * Hq) + align256(tq_scores_tc_bytes(p, B, Hq, Hkv));
+  return qprep_bytes(p, (size_t)B * Hq) + align256(tq_scores_tc_bytes(p, B, Hq, Hkv));
 }
 
 extern "C" tq_status tq_scores_workspace_size(const tq_codec* kc, int B, int Hq, int Hkv, size_t* bytes) {
   if (!kc || !bytes) return tq_fail(TQ_ERR_INVALID_ARG, "tq_scores_workspace_size: null argument");
   if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv)
     return tq_fail(TQ_ERR_INVALID_ARG, "tq_scores_workspace_size: bad shape B=%d Hq=%d Hkv=%d", B, Hq, Hkv);
+  if (!heads_fit_int(B, Hq, Hkv))
+    return tq_fail(TQ_ERR_UNSUPPORTED, "tq_scores_workspace_size: B*Hq or B*Hkv above INT_MAX");
   *bytes = scores_bytes(kc->p, B, Hq, Hkv);
   return TQ_OK;
 }
@@ -519,6 +528,7 @@ static tq_status check_heads(int B, int Hq, int Hkv, int64_t T, const char* name
     return tq_fail(TQ_ERR_INVALID_ARG, "%s: bad shape B=%d Hq=%d Hkv=%d T=%lld", name, B, Hq, Hkv, (long long)T);
   if (Hq % Hkv != 0) return tq_fail(TQ_ERR_INVALID_ARG, "%s: Hq %d not a multiple of Hkv %d", name, Hq, Hkv);
   if (Hq / Hkv > 32) return tq_fail(TQ_ERR_UNSUPPORTED, "%s: Hq/Hkv = %d above 32", name, Hq / Hkv);
+  if (!heads_fit_int(B, Hq, Hkv)) return tq_fail(TQ_ERR_UNSUPPORTED, "%s: B*Hq or B*Hkv above INT_MAX", name);
   if (T > (int64_t)1 << 31) return tq_fail(TQ_ERR_UNSUPPORTED, "%s: T above 2^31", name);
   return TQ_OK;
 }
@@ -556,7 +566,7 @@ static int device_sms(int device) {
 }
 
 static size_t attend_bytes(const tq_params& kp, int B, int Hq, int nchunk) {
-  return qprep_bytes(kp, B * Hq) + align256(sizeof(float) * (size_t)B * Hq * nchunk * (kp.d + 2));
+  return qprep_bytes(kp, (size_t)B * Hq) + align256(sizeof(float) * (size_t)B * Hq * nchunk * (kp.d + 2));
 }
 
 extern "C" tq_status tq_attend_workspace_size(const tq_codec* kc, const tq_codec* vc, int B, int Hq, int Hkv,

@@ -15,7 +15,9 @@
 // is looked up with cudaGetSymbolAddress once per device, with that device
 // current, the first time this entry point runs on the device, and cached.
 // Make that first call before any stream capture, because the lookup may load
-// the module.
+// the module.  The cached address belongs to the device's primary context: a
+// device reset (cudaDeviceReset) destroys it, so no call of this entry point
+// may follow one in the same process.
 //
 // All calls share the one array and it keeps whatever the last call left in
 // it.  Calls whose kernels overlap on the GPU (different streams, or several

@@ -26,7 +26,7 @@ source pages):
 * The estimator of <q, x> that the library evaluates is
   nu * ( <Pi q, c_hat> / sqrt(d) + ||r|| * sqrt(pi/2) / m * <S Pi q, sign(S r)> ).
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
 
 * rotation Pi = H_d diag(D) / sqrt(d), H_d the Sylvester-Hadamard matrix
   H[i][j] = (-1)^popcount(i & j), D iid +-1; d = 1536 uses three 512-blocks;

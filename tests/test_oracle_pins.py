@@ -422,6 +422,56 @@ def test_attend_special_cases():
     assert np.allclose(out[0, 0], O.dequantize(V, vc)[3], atol=1e-6)
 
 
+
+
+def _test_rotation(codec):
+    """Pi built here from a Sylvester matrix and the codec's D."""
+    d = codec.d
+    return _kron_hadamard(d) * codec.D[None, :] / math.sqrt(d)
+
+
+def test_attend_softmax_weights_worked_by_hand():
+    # Every vector is x = nu Pi^T c_hat / ||c_hat|| for chosen codes (c_hat
+    # their centroids), so its norm is nu and its codes are the chosen ones
+    # (checked).  With m = 0 the key estimate is nu <Pi q, c_hat> / sqrt(d)
+    # and the rotated dequantised value nu c_hat / sqrt(d): both follow from
+    # the chosen codes by plain dot products.  q is chosen so that the logits
+    # are (0, sqrt(d) ln 2, 0): softmax weights (1/4, 1/2, 1/4) at the default
+    # temperature 1/sqrt(d), and (1/6, 4/6, 1/6) at an explicit scale 2/sqrt(d).
+    d = 64
+    kc = _codec(d, (2,), 0, seed=3)
+    vc = _codec(d, (3,), 0, seed=5)
+    Pk, Pv = _test_rotation(kc), _test_rotation(vc)
+    rng = np.random.default_rng(8)
+    # codes of Gaussian draws, so that ||c_hat||^2 / d is near 1 and the
+    # normalised centroids stay inside their cells
+    kcodes = [np.searchsorted(kc.bnd[0], rng.standard_normal(d), side="right") for _ in range(2)]
+    vcodes = [np.searchsorted(vc.bnd[0], rng.standard_normal(d), side="right") for _ in range(3)]
+    knu, vnu = (1.75, 0.625), (0.875, 2.0, 1.25)      # exact in fp32
+    kchat = [kc.cen[0].astype(np.float64)[c] for c in kcodes]
+    vchat = [vc.cen[0].astype(np.float64)[c] for c in vcodes]
+    keys = np.stack([knu[t] * (kchat[t] / np.linalg.norm(kchat[t])) @ Pk for t in (0, 1, 0)])
+    vals = np.stack([vnu[t] * (vchat[t] / np.linalg.norm(vchat[t])) @ Pv for t in range(3)])
+    K, V = O.quantize(keys, kc), O.quantize(vals, vc)
+    assert np.array_equal(K.code_idx, np.stack([kcodes[0], kcodes[1], kcodes[0]]))
+    assert np.array_equal(V.code_idx, np.stack(vcodes))
+    assert list(K.norms) == [1.75, 0.625, 1.75] and list(V.norms) == [0.875, 2.0, 1.25]
+    # rotated query q' in the span of the two key centroid vectors
+    a0, a1 = (knu[t] * kchat[t] / math.sqrt(d) for t in (0, 1))
+    G = np.array([[a0 @ a0, a0 @ a1], [a1 @ a0, a1 @ a1]])
+    c0, c1 = np.linalg.solve(G, [0.0, math.sqrt(d) * math.log(2.0)])
+    qrot = c0 * a0 + c1 * a1
+    q = (qrot @ Pk)[None, None]                        # q = Pi^T q'
+    vrot = [vnu[t] * vchat[t] / math.sqrt(d) for t in range(3)]
+    for scale, w in ((None, (0.25, 0.5, 0.25)), (2.0 / math.sqrt(d), (1 / 6, 4 / 6, 1 / 6))):
+        out = O.attend(q, K, V, kc, vc, 1, 1, 1, 3, scale=scale)[0, 0]
+        want = (w[0] * vrot[0] + w[1] * vrot[1] + w[2] * vrot[2]) @ Pv
+        assert np.abs(out - want).max() < 1e-12 * np.abs(want).max(), (scale, np.abs(out - want).max())
+    # a wrong temperature (1 instead of 1/sqrt(d)) moves the output far away
+    out1 = O.attend(q, K, V, kc, vc, 1, 1, 1, 3, scale=1.0)[0, 0]
+    want = (0.25 * vrot[0] + 0.5 * vrot[1] + 0.25 * vrot[2]) @ Pv
+    assert np.abs(out1 - want).max() > 0.1 * np.abs(want).max()
+
 # ----------------------------------------------------------------------- top-k
 def test_topk_order_and_ties():
     sc = np.array([[0.5, 2.0, 2.0, -1.0, 2.0, 0.7]])
@@ -459,3 +509,31 @@ def test_plane_identity_of_symmetric_codebooks(bits, d):
                 par = bin(c & S).count("1") & 1
                 rec += a * (2.0 * par - 1.0 if bin(S).count("1") % 2 else 1.0)
         assert abs(rec - cen[c]) < 1e-12 * (1 + abs(cen[c]))
+
+
+
+@pytest.mark.parametrize("m", [64, 0])
+def test_search_scores_are_the_estimator(m):
+    # The search ranks the index rows by the same estimator as tq_scores: each
+    # query against all n rows is one decode head (B = Hq = Hkv = 1, T = n).
+    # With k = n the search returns every row, so its scores can be compared
+    # row by row with estimate_scores, and its order with a plain sort.
+    d, n, nq = 64, 257, 4
+    codec = _codec(d, (3,), m, seed=4)
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((n, d)) * rng.uniform(0.1, 3.0, (n, 1))
+    x[200] = x[17]                          # two rows with equal scores
+    q = rng.standard_normal((nq, d))
+    comp = O.quantize(x, codec)
+    idx, score = O.search_topk(q, comp, codec, n, row_offset=5)
+    for i in range(nq):
+        full = O.estimate_scores(q[i][None, None], comp, codec, 1, 1, 1, n)[0, 0]
+        rows = idx[i] - 5
+        assert sorted(rows.tolist()) == list(range(n))
+        assert np.all(np.abs(score[i] - full[rows]) <= 1e-12 * np.abs(full).max())
+        want = sorted(range(n), key=lambda r: (-full[r], r))
+        assert rows.tolist() == want
+        assert rows.tolist().index(17) < rows.tolist().index(200)
+    # a smaller k is the prefix of the full order
+    idx3, score3 = O.search_topk(q, comp, codec, 3)
+    assert np.array_equal(idx3, idx[:, :3] - 5) and np.array_equal(score3, score[:, :3])
