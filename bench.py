@@ -576,6 +576,11 @@ def main():
     h2d = kh.numel() * kh.element_size() + vh.numel() * vh.element_size() + qh.numel() * qh.element_size()
     d2h = lh.numel() * 4 + oh.numel() * 4
     del kd, vd
+    # a kernel whose bounded wait gave up records it in its codec: such a run
+    # measured nothing and must not print a number
+    for c in (layer.kc, layer.vc):
+        if tq.tq_codec_device_error(c) != 0:
+            raise RuntimeError("a libtq kernel reported a timed-out wait during the benchmark")
 
     if pg:
         pg.barrier()

@@ -13,22 +13,32 @@
 // A (keys, M = 128 per tile) goes to TMEM as u8 bytes: source word u (a plane
 // word, an xor of plane words, or a sign word) becomes eight 32-bit columns
 // word & (0x01010101 << r), r < 8, so K index k = 32u + 4r + j holds
-// 2^r * bit(r + 8j).  B (queries, N = 4 limbs x G queries, padded to 16)
-// holds round(v_k 2^(e - r)) split into four balanced base-256 s8 limbs, in
-// shared memory.  The s32 accumulation is exact; the epilogue rebuilds
-// I = sum_l 256^l D_l, scales by 2^-e and subtracts corr.
+// 2^r * bit(r + 8j).  B (queries) holds round(v_k 2^(e - r)) split into four
+// balanced base-256 s8 limbs, in shared memory.  The s32 accumulation is
+// exact; the epilogue rebuilds I = sum_l 256^l D_l, scales by 2^-e and
+// subtracts corr.
 //
 // Centroid-limb form (one segment of 3-bit codes): the plane identity needs
-// four odd plane subsets (16 source words at d = 128), one byte of K per
-// key bit.  Instead each coordinate's centroid, as the 16-bit fixed point
-// C = rint(cen * 2^f) split into two balanced s8 limbs, takes two bytes of
-// K: 8 source words for the first term, and 12 MMAs per tile in place of
-// 20.  Limb h of a word's 32 centroids goes to its own accumulator D_h
-// (the query image is the same for both), and the epilogue forms
-// sum_l 256^l (D_0l + 256 D_1l) 2^-(e+f).  The fixed point is the one
-// approximation: |cen - C 2^-f| <= 2^-(f+1) per coordinate, f = 13 for the
-// 3-bit codebooks (max |cen| < 4), so the first term moves by at most
-// 2^-14 ||q'||_1 / sqrt(d) <= 2^-14 ||q||.
+// four odd plane subsets (16 source words at d = 128), one byte of K per key
+// bit.  Instead each coordinate's centroid, as the 16-bit fixed point
+// C = rint(cen * 2^f) = C_0 + 256 C_1 in two balanced s8 limbs, takes two bytes
+// of K: 8 source words for the first term, 12 MMAs per tile in place of 20.
+// The query image of limb-1 words holds the query limbs one slot up, so both
+// limbs accumulate into the same columns.  Two approximations, both far inside
+// the logit tolerance of 1e-3 of nu ||q|| / sqrt(d):
+//   |cen - C 2^-f| <= 2^-(f+1), f = 13 for the 3-bit codebooks (max |cen| < 4):
+//     the first term moves by at most 2^-14 ||q'||_1 / sqrt(d) <= 2^-14 ||q||;
+//   q' is rounded to 22 bits of its largest element (three limbs, so that the
+//     shifted limb-1 image still fits four): the first term moves by at most
+//     2^-22 ||q|| sqrt(d), i.e. d 2^-22 of the tolerance floor.
+//
+// The limb bytes come from byte permutes, not table gathers: a 3-bit code is
+// a prmt selector into the eight limb bytes of the codebook held in two
+// registers, so one prmt yields the limbs of four coordinates.  The selector
+// word of group g < 4 of a 32-coordinate word holds the code of coordinate
+// g + 4k in nibble k (masked shifts of the three plane words); its low half
+// feeds TMEM column 2g and its high half column 2g + 1, so byte j of column
+// 2g + h is coordinate g + 4j + 16h, and the query image uses the same order.
 #include <math.h>
 
 #include <algorithm>
@@ -47,8 +57,6 @@ __host__ __device__ constexpr int term_mask(int bits, int t) {
                      : (t < 4 ? (1 << t) : (t == 4 ? 7 : t == 5 ? 11 : t == 6 ? 13 : 14));
 }
 
-__host__ __device__ inline int ncols_for(int G) { return ((4 * G + 15) / 16) * 16; }
-
 // the centroid-limb form applies to one segment of 3-bit codes
 __host__ __device__ inline bool use_cl(const tq_params& p) { return p.nseg == 1 && p.bits[0] == 3; }
 
@@ -62,8 +70,15 @@ __host__ __device__ inline int cl_shift(const tq_params& p) {
   return f;
 }
 
+// Source words of a tile, in K order: the MSE words [0, U_mse) (plane form:
+// odd plane subsets; centroid-limb form: limb-0 words then limb-1 words), then
+// the MS sign words.  One accumulator per tile, N columns: the MSE columns
+// [0, 4G) and the QJL columns [QO, QO + 4G), four query limbs per query; the
+// query image holds zeros in the QJL columns of MSE words and in the MSE
+// columns of sign words, so every word of a tile accumulates into the same
+// TMEM region and the epilogue reads 2 * round16(4G) columns.
 struct Geom {
-  int U_mse, U, Kt, N, G, lbo, bbytes, gstride;
+  int U_mse, U, Kt, G, QO, N, lbo, bbytes, gstride;
   bool cl;
   __host__ __device__ Geom(const tq_params& p, int G_) {
     cl = use_cl(p);
@@ -73,17 +88,30 @@ struct Geom {
     U = U_mse + p.MS;
     Kt = 32 * U;
     G = G_;
-    N = ncols_for(G_);
+    QO = ((4 * G_ + 15) / 16) * 16;
+    N = 2 * QO;
     lbo = (N / 8) * 128;
     bbytes = Kt * N;
     gstride = ((bbytes + 16 * G_ + 127) / 128) * 128;  // B image + 4 floats per query
   }
+  // TMEM columns of one tile slot: A (8 per source word) and D (N)
+  __host__ __device__ uint32_t acols() const { return 8u * (uint32_t)U; }
+  __host__ __device__ uint32_t slot_cols() const { return acols() + (uint32_t)N; }
 };
+
+// K byte k of a centroid-limb word holds coordinate cl_coord(k) of the word's
+// 32 (see the expansion: byte j of TMEM column 2g + h is g + 4j + 16h)
+__host__ __device__ inline int cl_coord(int k) { return (k >> 3) + 4 * (k & 3) + 16 * ((k >> 2) & 1); }
 
 // ------------------------------------------------------------ B operand
 // Blocks (group, part): every block of a (batch, KV head) group computes the
 // group's per-query exponents, then writes part `blockIdx.y` of its image
 // (part 0 also the per-query constants).  qprep rows are [q' (d) | w (m)].
+//   MSE columns, plane words: limb l of round(2 alpha q'_i 2^(e - r)), |.| < 2^30
+//   MSE columns, centroid-limb words: the three limbs of round(q'_i 2^e),
+//       |.| < 2^22, in slots 0..2 for limb-0 words and 1..3 (times 256) for
+//       limb-1 words, so that slot l sums 256^l-weighted centroid limbs
+//   QJL columns, sign words: limb l of round(2 w_j 2^(e - r)), |.| < 2^30
 __global__ void __launch_bounds__(256) tq_scores_bbuild_kernel(const tq_params p, const float* __restrict__ qprep,
                                                                const int Hq, const int Hkv, uint8_t* __restrict__ ws) {
   const Geom g(p, Hq / Hkv);
@@ -126,7 +154,7 @@ __global__ void __launch_bounds__(256) tq_scores_bbuild_kernel(const tq_params p
     if (lane == 0) {
       int ex;
       frexpf(mx > 0.f ? mx : 1.f, &ex);
-      const int em = 30 - ex;  // |v| 2^em < 2^30
+      const int em = (g.cl ? 22 : 30) - ex;  // |v| 2^em < 2^22 (three limbs) or 2^30 (four)
       frexpf(wmax > 0.f ? 2.f * wmax : 1.f, &ex);
       const int eq = 30 - ex;
       s_xmse[gq] = em;
@@ -145,19 +173,23 @@ __global__ void __launch_bounds__(256) tq_scores_bbuild_kernel(const tq_params p
   const int i0 = blockIdx.y * per, i1 = min(total, i0 + per);
   for (int idx = i0 + threadIdx.x; idx < i1; idx += blockDim.x) {
     const int n = idx / g.Kt, k = idx % g.Kt;
-    const int gq = n / 4, l = n % 4;
+    const bool qjl_col = n >= g.QO;
+    const int gq = (qjl_col ? n - g.QO : n) / 4, l = n % 4;
+    const int u = k / 32, r = (k % 32) / 4, j = k % 4, bp = r + 8 * j;
+    const bool sign_word = u >= g.U_mse;
     int8_t limb = 0;
-    if (gq < g.G) {
+    if (gq < g.G && qjl_col == sign_word) {
       const float* qv = qprep + (size_t)(b * Hq + hk * g.G + gq) * (d + m);
-      const int u = k / 32, r = (k % 32) / 4, j = k % 4, bp = r + 8 * j;
       float v;
-      int e, sh = r;
-      if (u < g.U_mse && g.cl) {
-        // both limb slots of word u % pw: byte k % 32 is coordinate k % 32
-        v = qv[32 * (u % p.pw) + k % 32];
+      int e, sh = r, slot = l;
+      if (!sign_word && g.cl) {
+        // limb h = u / pw of the centroids of word u % pw, coordinates in the
+        // expansion's order; limb-1 words see the query limbs one slot up
+        v = qv[32 * (u % p.pw) + cl_coord(k % 32)];
         e = s_xmse[gq];
         sh = 0;
-      } else if (u < g.U_mse) {
+        slot = l - u / p.pw;
+      } else if (!sign_word) {
         const int s = (p.nseg == 2 && u >= u0) ? 1 : 0;
         const int uu = s ? u - u0 : u;
         const int t = uu / p.pw, w = uu % p.pw;
@@ -173,7 +205,7 @@ __global__ void __launch_bounds__(256) tq_scores_bbuild_kernel(const tq_params p
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const int dq = (int)(int8_t)(x & 0xFF);
-        if (q == l) lv = dq;
+        if (q == slot) lv = dq;
         x = (x - dq) >> 8;
       }
       limb = (int8_t)lv;
@@ -185,23 +217,61 @@ __global__ void __launch_bounds__(256) tq_scores_bbuild_kernel(const tq_params p
 
 // ------------------------------------------------------------ scoring
 // Warp-specialised, one block per SM, tiles of 128 keys of one (batch, KV
-// head) group; a block owns a contiguous range of tiles.
-//   warps 0-3  expansion: read a tile's codes/signs from the ring, build the u8
-//              planes in TMEM A[i % 2] (warp w owns lanes 32w..32w+31)
-//   warps 4-7  epilogue: read accumulator D[i % 2], rebuild the two sums, write
-//              the logits
-//   warp 8     producer: bulk copies of key tiles into a 4-stage ring and of
-//              each group's query operand into one of two buffers
-//   warp 9     MMA issue: U tcgen05.mma (kind::i8, A from TMEM) per tile
-// mbarriers: ring_full/ring_empty (producer <-> expansion), a_full (expansion
-// -> MMA), mma_done (MMA commit -> expansion for A reuse, epilogue for D),
-// d_empty (epilogue -> MMA), b_full/b_empty (producer <-> MMA, query operand).
-constexpr int kStages = 4;
-constexpr int kThreads = 320;
+// head) group; a block owns a contiguous range of tiles.  Tile i of the block
+// uses slot i % NI: A buffer and accumulator in TMEM, MMA issuer warp.
+//   warps 0-7   expansion, two groups of four: group i % 2 reads tile i's
+//               codes/signs from the ring and builds its A operand (u8 planes
+//               or s8 centroid limbs); warp w owns TMEM lanes 32(w%4)..+31
+//   warps 8-15  epilogue, two groups of four: group i % 2 reads tile i's
+//               accumulator, rebuilds the two sums and writes the logits
+//   warp 16     producer: bulk copies of key tiles into a ring and of each
+//               group's query operand into one of two buffers
+//   warps 17-20 MMA issue: warp 17 + j issues every MMA of the tiles in slot j
+// A tcgen05.mma stream from one thread costs about a hundred cycles per
+// instruction at these shapes, while streams from different warps into
+// different accumulators overlap on the tensor core: hence one issuer per slot.
+// mbarriers: ring_full/ring_empty (producer <-> expansion), a_full[j]
+// (expansion -> issuer j), a_free[j] (issuer j's commit -> expansion),
+// d_full[j] (issuer j's commit -> epilogue), d_empty[j] (epilogue -> issuer
+// j), b_full/b_empty (producer <-> issuers, query operand).  NI is even and
+// the expansion and epilogue groups split tiles by parity, so each barrier's
+// phases are waited for in order by one consumer: a wait on a phase parity
+// then never meets its barrier a phase behind (which would pass at once) or
+// two phases ahead (which would never pass).
+constexpr int kStages = 8;
+constexpr int kMaxSlots = 4;
+constexpr int kExpWarps = 8, kEpiWarps = 8;
+constexpr int kEpiWarp0 = kExpWarps, kProdWarp = kExpWarps + kEpiWarps, kIssWarp0 = kProdWarp + 1;
+constexpr int kThreads = 32 * (kIssWarp0 + kMaxSlots);
 
 __host__ __device__ inline int ring_stage_bytes(int W, int MS) { return kKeys * (W + MS) * 4; }
 
-template <int D, int B0, int B1, bool RING>
+// Position of a block's tile in (group, first key): one division at the start,
+// then a running count (a 64-bit division per tile costs hundreds of cycles in
+// a single-thread loop).
+struct TileCursor {
+  int64_t grp, t0;
+  __device__ TileCursor(int64_t tile, int64_t tpg) {
+    grp = tile / tpg;
+    t0 = (tile - grp * tpg) * kKeys;
+  }
+  // moves `step` tiles on; groups hold tpg tiles, i.e. tpg * kKeys keys
+  __device__ void advance(int step, int64_t tpg_keys) {
+    t0 += (int64_t)step * kKeys;
+    while (t0 >= tpg_keys) {
+      t0 -= tpg_keys;
+      ++grp;
+    }
+  }
+};
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+template <int D, int B0, int B1, bool RING, int NI>
 __global__ void __launch_bounds__(kThreads, 1)
     tq_scores_tc_kernel(const tq_params p, const tq_compressed K, float* __restrict__ logits,
                         const uint8_t* __restrict__ ws, const int Hq, const int Hkv, const int64_t T,
@@ -213,10 +283,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int NT1 = B1 == 0 ? 0 : B1 == 1 ? 1 : B1 == 2 ? 2 : B1 == 3 ? 4 : 8;
   constexpr bool CL = B0 == 3 && B1 == 0;  // centroid-limb form (use_cl)
   constexpr int U_MSE = CL ? 2 * PW : (NT0 + NT1) * PW;
+  static_assert(NI % 2 == 0 && NI <= kMaxSlots, "tile slots must split evenly between the two tile parities");
 
   extern __shared__ __align__(1024) unsigned char smem[];
   __shared__ uint64_t ring_full[kStages], ring_empty[kStages];
-  __shared__ uint64_t a_full[2], mma_done[2], d_empty[2], b_full[2], b_empty[2], drained;
+  __shared__ uint64_t a_full[NI], a_free[NI], d_full[NI], d_empty[NI], b_full[2], b_empty[2], drained[NI];
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_abort;
 
@@ -227,49 +298,33 @@ __global__ void __launch_bounds__(kThreads, 1)
   unsigned char* bbuf = smem;                                     // [2][bstride]
   unsigned char* ring = smem + 2 * bstride;                       // [kStages][ring_stage_bytes]
   const int sbytes = ring_stage_bytes(W, MS);
-  // centroid-limb tables, indexed by the three plane nibbles of four
-  // coordinates (n0 | n1 << 4 | n2 << 8): byte j of entry h is limb h of the
-  // centroid of coordinate j (code bits: bit j of n0, n1, n2)
-  uint32_t* lut = reinterpret_cast<uint32_t*>(ring + (RING ? kStages * sbytes : 0));  // [2][4096]
-  const uint32_t acols = 8u * (uint32_t)g.U, dcols = (CL ? 3u : 2u) * (uint32_t)g.N;
+  const uint32_t scols = g.slot_cols(), acols = g.acols();        // slot j: A at j * scols, D after it
 
   const int64_t t_begin = (int64_t)blockIdx.x * ntiles / gridDim.x;
   const int64_t t_end = (int64_t)(blockIdx.x + 1) * ntiles / gridDim.x;
   const int64_t ntl = t_end - t_begin;
+  const int64_t tpg_keys = tiles_per_group * kKeys;
 
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) {
       tqtc::mbar_init(&ring_full[i], 1);
       tqtc::mbar_init(&ring_empty[i], 128);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NI; ++i) {
       tqtc::mbar_init(&a_full[i], 128);
-      tqtc::mbar_init(&mma_done[i], 1);
+      tqtc::mbar_init(&a_free[i], 1);
+      tqtc::mbar_init(&d_full[i], 1);
       tqtc::mbar_init(&d_empty[i], 128);
-      tqtc::mbar_init(&b_full[i], 1);
-      tqtc::mbar_init(&b_empty[i], 1);
+      tqtc::mbar_init(&drained[i], 1);
     }
-    tqtc::mbar_init(&drained, 1);
+    for (int i = 0; i < 2; ++i) {
+      tqtc::mbar_init(&b_full[i], 1);
+      tqtc::mbar_init(&b_empty[i], (uint32_t)NI);
+    }
     tqtc::fence_mbar_init();
     s_abort = 0;
   }
   if (warp == 0) tqtc::tmem_alloc(&s_tmem, 512);
-  if constexpr (CL) {
-    const float sc = ldexpf(1.f, cl_shift(p));
-    for (int i = tid; i < 4096; i += kThreads) {
-      uint32_t l0 = 0u, l1 = 0u;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int code = ((i >> j) & 1) | (((i >> (4 + j)) & 1) << 1) | (((i >> (8 + j)) & 1) << 2);
-        const int c = __float2int_rn(p.cen[0][code] * sc);
-        const int h0 = (int)(int8_t)(c & 0xFF), h1 = (c - h0) >> 8;
-        l0 |= (uint32_t)(h0 & 0xFF) << (8 * j);
-        l1 |= (uint32_t)(h1 & 0xFF) << (8 * j);
-      }
-      lut[i] = l0;
-      lut[4096 + i] = l1;
-    }
-  }
   tqtc::tc_fence_before();
   __syncthreads();
   tqtc::tc_fence_after();
@@ -279,14 +334,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     s_abort = 1;
   };
 
-  if (warp == 8) {
+  if (warp == kProdWarp) {
     // ---------------------------------------------------------- producer
     if (lane == 0) {
       int64_t cur = -1, issued = 0;
       int gi = -1;
-      for (int64_t i = 0; i < ntl && !s_abort; ++i) {
-        const int64_t tile = t_begin + i;
-        const int64_t grp = tile / tiles_per_group;
+      TileCursor tc(t_begin, tiles_per_group);
+      for (int64_t i = 0; i < ntl && !s_abort; ++i, tc.advance(1, tpg_keys)) {
+        const int64_t grp = tc.grp;
         if (grp != cur) {
           cur = grp;
           ++gi;
@@ -305,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             fail(tqtc::kErrCopyWait);
             break;
           }
-          const int64_t t0 = (tile % tiles_per_group) * kKeys;
+          const int64_t t0 = tc.t0;
           const int64_t rows = (T - t0) < kKeys ? (T - t0) : kKeys;
           const int64_t row0 = grp * T + t0;
           unsigned char* dst = ring + (size_t)st * sbytes;
@@ -324,17 +379,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!tqtc::mbar_wait_or_abort(&b_full[j & 1], (uint32_t)((j / 2) & 1), nullptr))
           atomicExch(p.err, tqtc::kErrCopyWait);
     }
-  } else if (warp == 9) {
+  } else if (warp >= kIssWarp0) {
     // ---------------------------------------------------------- MMA issue
-    if (lane == 0) {
-      const uint32_t idesc = tqtc::instr_desc(2, 0, 1, kKeys, (uint32_t)g.N);     // A u8, B s8
+    const int js = warp - kIssWarp0;  // tile slot of this issuer
+    if (lane == 0 && js < NI) {
+      // centroid limbs are signed; masked plane and sign bytes reach 128
+      const uint32_t idesc_u8 = tqtc::instr_desc(2, 0, 1, kKeys, (uint32_t)g.N);  // A u8, B s8
       const uint32_t idesc_s8 = tqtc::instr_desc(2, 1, 1, kKeys, (uint32_t)g.N);  // A s8, B s8
+      const uint32_t a0 = tbase + (uint32_t)js * scols, dst = a0 + acols;
+      const uint64_t step = (uint64_t)((2u * (uint32_t)g.lbo) >> 4);
       int64_t cur = -1;
       int gi = -1;
-      for (int64_t i = 0; i < ntl && !s_abort; ++i) {
-        const int64_t tile = t_begin + i;
-        const int64_t grp = tile / tiles_per_group;
-        const int b = (int)(i & 1);
+      TileCursor tc(t_begin, tiles_per_group);
+      for (int64_t i = 0; i < ntl && !s_abort; ++i, tc.advance(1, tpg_keys)) {
+        const int64_t grp = tc.grp;
+        // every issuer follows the group changes (b_full, b_empty), whatever
+        // the slots of the tiles that carry them
         if (grp != cur) {
           if (gi >= 0) tqtc::mma_commit(&b_empty[gi & 1]);  // previous group's operand is free once done
           cur = grp;
@@ -344,50 +404,58 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
         }
-        if (!tqtc::mbar_wait_or_abort(&a_full[b], (uint32_t)((i / 2) & 1), &s_abort)) {
+        if ((int)(i % NI) != js) continue;
+        const uint32_t ph = (uint32_t)((i / NI) & 1);
+        if (!tqtc::mbar_wait_or_abort(&a_full[js], ph, &s_abort)) {
           fail(tqtc::kErrMmaWait);
           break;
         }
-        if (i >= 2 && !tqtc::mbar_wait_or_abort(&d_empty[b], (uint32_t)((i / 2 - 1) & 1), &s_abort)) {
+        if (i >= NI && !tqtc::mbar_wait_or_abort(&d_empty[js], ph ^ 1u, &s_abort)) {
           fail(tqtc::kErrMmaWait);
           break;
         }
         tqtc::tc_fence_after();
-        const uint32_t a0 = tbase + (uint32_t)b * acols;
-        const uint32_t d_mse = tbase + 2u * acols + (uint32_t)b * dcols, d_qjl = d_mse + (uint32_t)g.N;
         uint64_t desc = tqtc::smem_desc(tqtc::smem_u32(bbuf + (gi & 1) * bstride), (uint32_t)g.lbo, 128);
-        const uint64_t step = (uint64_t)((2u * (uint32_t)g.lbo) >> 4);
-        if constexpr (CL) {
-          // limb 0 words -> D_0, limb 1 words -> D_1 (signed limbs: A is s8),
-          // sign words -> D_qjl (masked bytes up to 128: A is u8)
-          for (int u = 0; u < g.U; ++u) {
-            const uint32_t dst = u < PW ? d_mse : u < U_MSE ? d_mse + (uint32_t)g.N : d_mse + 2u * (uint32_t)g.N;
-            tqtc::mma_i8_ts(dst, a0 + 8u * (uint32_t)u, desc, u < U_MSE ? idesc_s8 : idesc,
-                            !(u == 0 || u == PW || u == U_MSE));
-            desc += step;
-          }
-        } else {
-          for (int u = 0; u < g.U; ++u) {
-            const bool qjl = u >= g.U_mse;
-            tqtc::mma_i8_ts(qjl ? d_qjl : d_mse, a0 + 8u * (uint32_t)u, desc, idesc, !(u == 0 || u == g.U_mse));
-            desc += step;
-          }
+#pragma unroll 1
+        for (int u = 0; u < U_MSE + MS; ++u) {
+          tqtc::mma_i8_ts(dst, a0 + 8u * (uint32_t)u, desc, (CL && u < U_MSE) ? idesc_s8 : idesc_u8, u != 0);
+          desc += step;
         }
-        tqtc::mma_commit(&mma_done[b]);
+        tqtc::mma_commit(&a_free[js]);
+        tqtc::mma_commit(&d_full[js]);
       }
       // every MMA issued has completed before TMEM is released (bounded)
-      tqtc::mma_commit(&drained);
-      if (!tqtc::mbar_wait_or_abort(&drained, 0, nullptr)) atomicExch(p.err, tqtc::kErrMmaWait);
+      tqtc::mma_commit(&drained[js]);
+      if (!tqtc::mbar_wait_or_abort(&drained[js], 0, nullptr)) atomicExch(p.err, tqtc::kErrMmaWait);
     }
-  } else if (warp < 4) {
+  } else if (warp < kExpWarps) {
     // ---------------------------------------------------------- expansion
-    const uint32_t lane_base = 32u * (uint32_t)warp;
-    for (int64_t i = 0; i < ntl; ++i) {
-      const int64_t tile = t_begin + i;
-      const int64_t grp = tile / tiles_per_group;
-      const int64_t t0 = (tile % tiles_per_group) * kKeys;
-      const int b = (int)(i & 1);
-      const bool valid = t0 + tid < T;
+    const uint32_t lane_base = 32u * (uint32_t)(warp & 3);
+    const int xg = warp >> 2, kt = tid & 127;  // tile parity of this group, key of this thread
+    // centroid limbs as prmt tables: byte c of (tl, th) is limb h of code c
+    uint32_t tl0 = 0u, th0 = 0u, tl1 = 0u, th1 = 0u;
+    if constexpr (CL) {
+      const float sc = ldexpf(1.f, cl_shift(p));
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const int v = __float2int_rn(p.cen[0][c] * sc);
+        const int h0 = (int)(int8_t)(v & 0xFF), h1 = (v - h0) >> 8;
+        const uint32_t b0 = (uint32_t)(h0 & 0xFF), b1 = (uint32_t)(h1 & 0xFF);
+        if (c < 4) {
+          tl0 |= b0 << (8 * c);
+          tl1 |= b1 << (8 * c);
+        } else {
+          th0 |= b0 << (8 * (c - 4));
+          th1 |= b1 << (8 * (c - 4));
+        }
+      }
+    }
+    TileCursor tc(t_begin + xg, tiles_per_group);
+    for (int64_t i = xg; i < ntl; i += 2, tc.advance(2, tpg_keys)) {
+      const int64_t grp = tc.grp;
+      const int64_t t0 = tc.t0;
+      const int js = (int)(i % NI);
+      const bool valid = t0 + kt < T;
       uint32_t kcw[W], ksw[8];
 #pragma unroll
       for (int k = 0; k < W; ++k) kcw[k] = 0u;
@@ -401,7 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (valid) {
           const unsigned char* src = ring + (size_t)st * sbytes;
-          const uint32_t* c32 = reinterpret_cast<const uint32_t*>(src) + tid * W;
+          const uint32_t* c32 = reinterpret_cast<const uint32_t*>(src) + kt * W;
           if constexpr (W % 4 == 0) {
 #pragma unroll
             for (int k = 0; k < W; k += 4) {
@@ -418,27 +486,27 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int k = 0; k < W; ++k) kcw[k] = c32[k];
           }
-          const uint32_t* s32 = reinterpret_cast<const uint32_t*>(src + kKeys * W * 4) + tid * MS;
+          const uint32_t* s32 = reinterpret_cast<const uint32_t*>(src + kKeys * W * 4) + kt * MS;
 #pragma unroll
           for (int k = 0; k < 8; ++k)
             if (k < MS) ksw[k] = s32[k];
         }
         tqtc::mbar_arrive(&ring_empty[st]);
       } else if (valid) {
-        const int64_t row = grp * T + t0 + tid;
+        const int64_t row = grp * T + t0 + kt;
 #pragma unroll
         for (int k = 0; k < W; ++k) kcw[k] = __ldg(K.codes + row * W + k);
 #pragma unroll
         for (int k = 0; k < 8; ++k)
           if (k < MS) ksw[k] = __ldg(K.signs + row * MS + k);
       }
-      // A[b] is free once the MMAs of tile i - 2 are done
-      if (i >= 2 && !tqtc::mbar_wait_or_abort(&mma_done[b], (uint32_t)((i / 2 - 1) & 1), &s_abort)) {
+      // slot js's A is free once the MMAs of tile i - NI are done
+      if (i >= NI && !tqtc::mbar_wait_or_abort(&a_free[js], (uint32_t)((i / NI - 1) & 1), &s_abort)) {
         fail(tqtc::kErrMmaWait);
         break;
       }
       tqtc::tc_fence_after();
-      const uint32_t a0 = (uint32_t)b * acols;
+      const uint32_t a0 = (uint32_t)js * scols;
       auto emit = [&](int u, uint32_t word) {
         uint32_t regs[8];
 #pragma unroll
@@ -448,111 +516,131 @@ __global__ void __launch_bounds__(kThreads, 1)
       if constexpr (CL) {
 #pragma unroll
         for (int w = 0; w < PW; ++w) {
+          const uint32_t p0 = kcw[w], p1 = kcw[PW + w], p2 = kcw[2 * PW + w];
           uint32_t r0[8], r1[8];
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint32_t ix = ((kcw[w] >> (4 * c)) & 0xFu) | (((kcw[PW + w] >> (4 * c)) & 0xFu) << 4) |
-                                (((kcw[2 * PW + w] >> (4 * c)) & 0xFu) << 8);
-            r0[c] = lut[ix];
-            r1[c] = lut[4096 + ix];
+          for (int gg = 0; gg < 4; ++gg) {
+            // nibble k: code of coordinate gg + 4k (bit 4k + j from plane j)
+            const uint32_t x1 = gg >= 1 ? p1 >> (gg - 1) : p1 << 1;
+            const uint32_t x2 = gg >= 2 ? p2 >> (gg - 2) : p2 << (2 - gg);
+            const uint32_t sel = ((p0 >> gg) & 0x11111111u) | (x1 & 0x22222222u) | (x2 & 0x44444444u);
+            const uint32_t shi = sel >> 16;
+            r0[2 * gg] = prmt(tl0, th0, sel);
+            r1[2 * gg] = prmt(tl1, th1, sel);
+            r0[2 * gg + 1] = prmt(tl0, th0, shi);
+            r1[2 * gg + 1] = prmt(tl1, th1, shi);
           }
           tqtc::tmem_st8(tqtc::tmem_addr(tbase, lane_base, a0 + 8u * (uint32_t)w), r0);
           tqtc::tmem_st8(tqtc::tmem_addr(tbase, lane_base, a0 + 8u * (uint32_t)(PW + w)), r1);
         }
       } else {
 #pragma unroll
-      for (int s = 0; s < NSEG; ++s) {
-        const int bits = s ? B1 : B0;
-        const int base = s ? B0 * PW : 0;
-        const int nt = s ? NT1 : NT0;
-        const int ubase = s ? NT0 * PW : 0;
+        for (int s = 0; s < NSEG; ++s) {
+          const int bits = s ? B1 : B0;
+          const int base = s ? B0 * PW : 0;
+          const int nt = s ? NT1 : NT0;
+          const int ubase = s ? NT0 * PW : 0;
 #pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          if (t < nt) {
-            const int mask = term_mask(bits, t);
+          for (int t = 0; t < 8; ++t) {
+            if (t < nt) {
+              const int mask = term_mask(bits, t);
 #pragma unroll
-            for (int w = 0; w < PW; ++w) {
-              uint32_t word = 0u;
+              for (int w = 0; w < PW; ++w) {
+                uint32_t word = 0u;
 #pragma unroll
-              for (int k = 0; k < 4; ++k)
-                if ((mask >> k) & 1) word ^= kcw[base + k * PW + w];
-              emit(ubase + t * PW + w, word);
+                for (int k = 0; k < 4; ++k)
+                  if ((mask >> k) & 1) word ^= kcw[base + k * PW + w];
+                emit(ubase + t * PW + w, word);
+              }
             }
           }
         }
-      }
       }
 #pragma unroll
       for (int k = 0; k < 8; ++k)
         if (k < MS) emit(U_MSE + k, ksw[k]);
       tqtc::tmem_wait_st();
       tqtc::tc_fence_before();
-      tqtc::mbar_arrive(&a_full[b]);
+      tqtc::mbar_arrive(&a_full[js]);
     }
   } else {
-    // ---------------------------------------------------------- epilogue (warps 4-7)
-    const int et = tid - 128;
-    const uint32_t lane_base = 32u * (uint32_t)(warp - 4);
+    // ---------------------------------------------------------- epilogue
+    const int eg = (warp - kEpiWarp0) >> 2, et = (tid - 32 * kEpiWarp0) & 127;  // tile parity, key
+    const uint32_t lane_base = 32u * (uint32_t)(warp & 3);
     const float kcl = CL ? ldexpf(p.inv_sqrt_d, -cl_shift(p)) : 0.f;  // 2^-f / sqrt(d)
-    for (int64_t i = 0; i < ntl; ++i) {
-      const int64_t tile = t_begin + i;
-      const int64_t grp = tile / tiles_per_group;
-      const int64_t t0 = (tile % tiles_per_group) * kKeys;
-      const int b = (int)(i & 1);
+    TileCursor tc(t_begin + eg, tiles_per_group);
+    int64_t cur = -1;
+    int bq = 0, hk = 0;
+    // the key norms come from HBM: each tile's are loaded one tile ahead
+    auto load_norms = [&](const TileCursor& c, float& nu, float& gam) {
+      const bool ok = c.t0 + et < T;
+      const int64_t r = c.grp * T + c.t0 + et;
+      nu = ok ? __ldg(K.norms + r) : 0.f;
+      gam = (ok && MS > 0) ? __ldg(K.rnorms + r) : 0.f;
+    };
+    float nxt_nu = 0.f, nxt_gam = 0.f;
+    if (eg < ntl) load_norms(tc, nxt_nu, nxt_gam);
+    for (int64_t i = eg; i < ntl; i += 2, tc.advance(2, tpg_keys)) {
+      const int64_t grp = tc.grp;
+      const int64_t t0 = tc.t0;
+      const int js = (int)(i % NI);
+      if (grp != cur) {  // (batch, KV head) of the group, once per group
+        cur = grp;
+        bq = (int)(grp / Hkv);
+        hk = (int)(grp - (int64_t)bq * Hkv);
+      }
       const int64_t t = t0 + et;
       const bool valid = t < T;
-      const int64_t row = grp * T + t;
-      const float knu = valid ? __ldg(K.norms + row) : 0.f;
-      const float kgam = (valid && MS > 0) ? __ldg(K.rnorms + row) : 0.f;
+      const float knu = nxt_nu, kgam = nxt_gam;
+      if (i + 2 < ntl) {
+        TileCursor nc = tc;
+        nc.advance(2, tpg_keys);
+        load_norms(nc, nxt_nu, nxt_gam);
+      }
       const float* cs_all = reinterpret_cast<const float*>(ws + (size_t)grp * g.gstride + g.bbytes);
-      if (!tqtc::mbar_wait_or_abort(&mma_done[b], (uint32_t)((i / 2) & 1), &s_abort)) {
+      if (!tqtc::mbar_wait_or_abort(&d_full[js], (uint32_t)((i / NI) & 1), &s_abort)) {
         fail(tqtc::kErrMmaWait);
         break;
       }
       tqtc::tc_fence_after();
-      const uint32_t d_mse = 2u * acols + (uint32_t)b * dcols;
-      const uint32_t d_qjl = d_mse + (CL ? 2u : 1u) * (uint32_t)g.N;
-      const int bq = (int)(grp / Hkv), hk = (int)(grp % Hkv);
+      const uint32_t dset = (uint32_t)js * scols + acols;
       const float cq = kgam * p.qjl_coef;
-      for (int qc = 0; qc < g.N / 16; ++qc) {
-        uint32_t dm[16], dq[16], dm1[16];
-        tqtc::tmem_ld16(tqtc::tmem_addr(tbase, lane_base, d_mse + 16u * qc), dm);
-        if (CL) tqtc::tmem_ld16(tqtc::tmem_addr(tbase, lane_base, d_mse + (uint32_t)g.N + 16u * qc), dm1);
-        if (MS > 0) tqtc::tmem_ld16(tqtc::tmem_addr(tbase, lane_base, d_qjl + 16u * qc), dq);
+      for (int qc = 0; qc < g.QO / 16; ++qc) {
+        // per-query constants of the group (2^-e scales, correction sums),
+        // requested before the accumulator loads so that both latencies overlap
+        float4 cs[4];
+#pragma unroll
+        for (int g4 = 0; g4 < 4; ++g4)
+          cs[g4] = (4 * qc + g4 < g.G) ? __ldg(reinterpret_cast<const float4*>(cs_all) + 4 * qc + g4)
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+        uint32_t dm[16], dq[16];
+        tqtc::tmem_ld16(tqtc::tmem_addr(tbase, lane_base, dset + 16u * qc), dm);
+        if (MS > 0) tqtc::tmem_ld16(tqtc::tmem_addr(tbase, lane_base, dset + (uint32_t)g.QO + 16u * qc), dq);
         tqtc::tmem_wait_ld();
-        if (qc == g.N / 16 - 1) {
+        if (qc == g.QO / 16 - 1) {
           tqtc::tc_fence_before();
-          tqtc::mbar_arrive(&d_empty[b]);
+          tqtc::mbar_arrive(&d_empty[js]);
         }
 #pragma unroll
         for (int g4 = 0; g4 < 4; ++g4) {
           const int gq = 4 * qc + g4;
           if (gq < g.G && valid) {
-            const float4 cs = __ldg(reinterpret_cast<const float4*>(cs_all) + gq);
+            // I = sum_l 256^l D_l over the query's four limb columns (exact s32 sums)
+            float im = (float)(int)dm[4 * g4 + 3];
+            im = fmaf(im, 256.f, (float)(int)dm[4 * g4 + 2]);
+            im = fmaf(im, 256.f, (float)(int)dm[4 * g4 + 1]);
+            im = fmaf(im, 256.f, (float)(int)dm[4 * g4 + 0]);
             float val;
-            if constexpr (CL) {
-              // per query limb l: D_0l + 256 D_1l
-              float t4[4];
-#pragma unroll
-              for (int l = 0; l < 4; ++l) t4[l] = fmaf((float)(int)dm1[4 * g4 + l], 256.f, (float)(int)dm[4 * g4 + l]);
-              float im = t4[3];
-              im = fmaf(im, 256.f, t4[2]);
-              im = fmaf(im, 256.f, t4[1]);
-              im = fmaf(im, 256.f, t4[0]);
-              val = (im * cs.x) * kcl;
-            } else {
-              float im = (float)(int)dm[4 * g4 + 3];
-              im = fmaf(im, 256.f, (float)(int)dm[4 * g4 + 2]);
-              im = fmaf(im, 256.f, (float)(int)dm[4 * g4 + 1]);
-              im = fmaf(im, 256.f, (float)(int)dm[4 * g4 + 0]);
-              val = fmaf(im, cs.x, -cs.y) * p.inv_sqrt_d;
-            }
+            if constexpr (CL)
+              val = (im * cs[g4].x) * kcl;
+            else
+              val = fmaf(im, cs[g4].x, -cs[g4].y) * p.inv_sqrt_d;
             if (MS > 0) {
               float iq = (float)(int)dq[4 * g4 + 3];
               iq = fmaf(iq, 256.f, (float)(int)dq[4 * g4 + 2]);
               iq = fmaf(iq, 256.f, (float)(int)dq[4 * g4 + 1]);
               iq = fmaf(iq, 256.f, (float)(int)dq[4 * g4 + 0]);
-              val = fmaf(cq, fmaf(iq, cs.z, -cs.w), val);
+              val = fmaf(cq, fmaf(iq, cs[g4].z, -cs[g4].w), val);
             }
             logits[((int64_t)bq * Hq + hk * g.G + gq) * T + t] = knu * val;
           }
@@ -593,25 +681,23 @@ bool supported(const tq_params& p, int G, uint32_t* cols_out) {
   if (p.m > 256) return false;
   if (!(p.nseg == 1 || (p.bits[0] == 2 && p.bits[1] == 3))) return false;
   const Geom g(p, G);
-  if (g.bbytes > 64 * 1024 || g.N > 128) return false;
-  const uint32_t need = 2u * (8u * g.U + (g.cl ? 3u : 2u) * g.N);  // double-buffered A and accumulators
-  if (need > 512) return false;
+  if (g.bbytes > 64 * 1024 || g.N > 256) return false;
+  if (2u * g.slot_cols() > 512) return false;  // two tile slots at least
   if (cols_out) *cols_out = 512;
   return true;
 }
 
-template <int D, int B0, int B1, bool RING>
+template <int D, int B0, int B1, bool RING, int NI>
 cudaError_t launch_scores_t(const tq_params& p, const tq_compressed& K, float* logits, const uint8_t* ws, int B,
                             int Hq, int Hkv, int64_t T, cudaStream_t st) {
   constexpr int W = (B0 + B1) * ((D / (B1 > 0 ? 2 : 1)) / 32);
   const Geom g(p, Hq / Hkv);
   const size_t bstride = (size_t)((g.bbytes + 16 * g.G + 127) / 128) * 128;
   size_t smem = 2 * bstride + (RING ? (size_t)kStages * ring_stage_bytes(W, p.MS) : 0);
-  if (B0 == 3 && B1 == 0) smem += 2 * 4096 * sizeof(uint32_t);  // centroid-limb tables
   // the block takes all 512 TMEM columns: ask for more than half of the SM's
   // shared memory so that a second block never waits on the allocation
   smem = std::max(smem, (size_t)(smem_per_sm() / 2 + 1024));
-  auto fn = tq_scores_tc_kernel<D, B0, B1, RING>;
+  auto fn = tq_scores_tc_kernel<D, B0, B1, RING, NI>;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int64_t tpg = (T + kKeys - 1) / kKeys;
@@ -627,8 +713,13 @@ cudaError_t launch_scores(const tq_params& p, const tq_compressed& K, float* log
   (void)cols;
   // bulk copies need 16-byte aligned tile starts and sizes: T a multiple of 4
   const bool ring = (T % 4) == 0 && (uintptr_t)K.codes % 16 == 0 && (p.MS == 0 || (uintptr_t)K.signs % 16 == 0);
-  return ring ? launch_scores_t<D, B0, B1, true>(p, K, logits, ws, B, Hq, Hkv, T, st)
-              : launch_scores_t<D, B0, B1, false>(p, K, logits, ws, B, Hq, Hkv, T, st);
+  // four tile slots where TMEM holds them, else two (always an even count)
+  const Geom g(p, Hq / Hkv);
+  if ((uint32_t)kMaxSlots * g.slot_cols() <= 512u)
+    return ring ? launch_scores_t<D, B0, B1, true, kMaxSlots>(p, K, logits, ws, B, Hq, Hkv, T, st)
+                : launch_scores_t<D, B0, B1, false, kMaxSlots>(p, K, logits, ws, B, Hq, Hkv, T, st);
+  return ring ? launch_scores_t<D, B0, B1, true, 2>(p, K, logits, ws, B, Hq, Hkv, T, st)
+              : launch_scores_t<D, B0, B1, false, 2>(p, K, logits, ws, B, Hq, Hkv, T, st);
 }
 
 }  // namespace

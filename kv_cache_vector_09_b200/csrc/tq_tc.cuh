@@ -42,7 +42,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete; false on timeout.
+// The clock is read only once a first poll has failed: on the single-thread
+// paths of the pipelines most waits find the phase already complete.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
     if (clock64() - t0 > kWaitCycles) return false;
@@ -53,6 +56,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
 // As mbar_wait, but also gives up as soon as *abort becomes nonzero (another
 // warp of the block has already recorded a failure).
 __device__ __forceinline__ bool mbar_wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
     if ((abort && *abort) || clock64() - t0 > kWaitCycles) return false;
@@ -65,6 +69,7 @@ __device__ __forceinline__ bool mbar_wait_or_abort(uint64_t* bar, uint32_t parit
 // warps they wait for.
 __device__ __forceinline__ bool mbar_wait_sleep_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort,
                                                          unsigned ns) {
+  if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
     if ((abort && *abort) || clock64() - t0 > kWaitCycles) return false;
