@@ -550,11 +550,15 @@ extern "C" tq_status tq_scores(const tq_codec* kc, const void* q, tq_dtype dt, i
     return tq_fail(TQ_ERR_INVALID_ARG, "tq_scores: workspace null, misaligned or smaller than %zu bytes", need);
   const cudaStream_t s = (cudaStream_t)stream;
   float* qprep = (float*)workspace;
-  cudaError_t e = tq_launch_qprep(kc->p, q, dt, B * Hq, qprep, s);
+  cudaError_t e;
+  e = tq_launch_qprep(kc->p, q, dt, B * Hq, qprep, s);
   if (e == cudaSuccess) {
-    void* ws_tc = (char*)workspace + qprep_bytes(kc->p, B * Hq);
-    e = tq_launch_scores_tc(kc->p, qprep, B, Hq, Hkv, T, *K, logits, ws_tc, s);
-    if (e == cudaErrorNotSupported) e = tq_launch_scores(kc->p, qprep, B, Hq, Hkv, T, *K, logits, s);
+    if (tq_scores_tc_supported(kc->p, Hq, Hkv)) {
+      void* ws_tc = (char*)workspace + qprep_bytes(kc->p, (size_t)B * Hq);
+      e = tq_launch_scores_tc(kc->p, qprep, B, Hq, Hkv, T, *K, logits, ws_tc, s);
+    } else {
+      e = tq_launch_scores(kc->p, qprep, B, Hq, Hkv, T, *K, logits, s);
+    }
   }
   return launch_status(e, "tq_scores launch");
 }

@@ -83,8 +83,11 @@ cudaError_t tq_launch_quantize(const tq_params& p, const void* x, tq_dtype dt, i
 // has no tensor-core variant (the caller then uses the generic kernel)
 cudaError_t tq_launch_quantize_tc(const tq_params& p, const void* x, tq_dtype dt, int64_t n, int64_t ld,
                                   const tq_compressed& out, cudaStream_t st);
-// tensor-core scorer: workspace bytes it needs after the query-prep block (0
-// if the configuration has no tensor-core variant), and the launch
+// tensor-core scorer: whether it takes the shape, the workspace bytes it
+// needs after the query-prep block (0 if the configuration has no
+// tensor-core variant), and the launch (query image, then the scoring
+// kernel) on prepared queries
+bool tq_scores_tc_supported(const tq_params& p, int Hq, int Hkv);
 size_t tq_scores_tc_bytes(const tq_params& p, int B, int Hq, int Hkv);
 cudaError_t tq_launch_scores_tc(const tq_params& p, const float* qprep, int B, int Hq, int Hkv, int64_t T,
                                 const tq_compressed& K, float* logits, void* ws_tc, cudaStream_t st);

@@ -104,25 +104,34 @@ struct Geom {
 __host__ __device__ inline int cl_coord(int k) { return (k >> 3) + 4 * (k & 3) + 16 * ((k >> 2) & 1); }
 
 // ------------------------------------------------------------ B operand
-// Blocks (group, part): every block of a (batch, KV head) group computes the
-// group's per-query exponents, then writes part `blockIdx.y` of its image
-// (part 0 also the per-query constants).  qprep rows are [q' (d) | w (m)].
+// Query image.  Blocks (group, part): every block of a (batch, KV head) group
+// copies the group's G prepared query rows [q' (d) | w = S q' (m)] into shared
+// memory and computes the per-query exponents, then writes part `blockIdx.y`
+// of the group's image (part 0 also the per-query constants).
 //   MSE columns, plane words: limb l of round(2 alpha q'_i 2^(e - r)), |.| < 2^30
 //   MSE columns, centroid-limb words: the three limbs of round(q'_i 2^e),
 //       |.| < 2^22, in slots 0..2 for limb-0 words and 1..3 (times 256) for
 //       limb-1 words, so that slot l sums 256^l-weighted centroid limbs
 //   QJL columns, sign words: limb l of round(2 w_j 2^(e - r)), |.| < 2^30
+// The scoring kernel is launched as its programmatic dependent: it starts
+// streaming keys while this kernel runs and waits for its results only where
+// it reads them.
 __global__ void __launch_bounds__(256) tq_scores_bbuild_kernel(const tq_params p, const float* __restrict__ qprep,
                                                                const int Hq, const int Hkv, uint8_t* __restrict__ ws) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  extern __shared__ __align__(16) float qw[];  // [G][d + m]: q' then w
   const Geom g(p, Hq / Hkv);
   const int grp = blockIdx.x, b = grp / Hkv, hk = grp % Hkv;
-  const int d = p.d, m = p.m, L = p.seg_len;
+  const int d = p.d, m = p.m, L = p.seg_len, ld = d + m;
   __shared__ int s_xmse[32], s_xqjl[32];    // exponents e
   uint8_t* out = ws + (size_t)grp * g.gstride;
   float* consts = reinterpret_cast<float*>(out + g.bbytes);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int gq = warp; gq < g.G; gq += blockDim.x / 32) {
-    const float* qv = qprep + (size_t)(b * Hq + hk * g.G + gq) * (d + m);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x / 32;
+  for (int i = threadIdx.x; i < g.G * ld; i += blockDim.x)
+    qw[i] = qprep[(size_t)(b * Hq + hk * g.G) * ld + i];
+  __syncthreads();
+  for (int gq = warp; gq < g.G; gq += nw) {
+    const float* qv = qw + gq * ld;
     float mx = 0.f, corr = 0.f;
     for (int s = 0; s < p.nseg; ++s) {
       float amax = 0.f, qmax = 0.f, qsum = 0.f;
@@ -179,7 +188,7 @@ __global__ void __launch_bounds__(256) tq_scores_bbuild_kernel(const tq_params p
     const bool sign_word = u >= g.U_mse;
     int8_t limb = 0;
     if (gq < g.G && qjl_col == sign_word) {
-      const float* qv = qprep + (size_t)(b * Hq + hk * g.G + gq) * (d + m);
+      const float* qv = qw + gq * ld;
       float v;
       int e, sh = r, slot = l;
       if (!sign_word && g.cl) {
@@ -203,9 +212,9 @@ __global__ void __launch_bounds__(256) tq_scores_bbuild_kernel(const tq_params p
       // balanced base-256 digits
       int lv = 0;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int qd = 0; qd < 4; ++qd) {
         const int dq = (int)(int8_t)(x & 0xFF);
-        if (q == slot) lv = dq;
+        if (qd == slot) lv = dq;
         x = (x - dq) >> 8;
       }
       limb = (int8_t)lv;
@@ -224,9 +233,12 @@ __global__ void __launch_bounds__(256) tq_scores_bbuild_kernel(const tq_params p
 //               or s8 centroid limbs); warp w owns TMEM lanes 32(w%4)..+31
 //   warps 8-15  epilogue, two groups of four: group i % 2 reads tile i's
 //               accumulator, rebuilds the two sums and writes the logits
-//   warp 16     producer: bulk copies of key tiles into a ring and of each
-//               group's query operand into one of two buffers
-//   warps 17-20 MMA issue: warp 17 + j issues every MMA of the tiles in slot j
+//   warps 16-17 producers: warp 16 + x makes the bulk copies of the tiles of
+//               parity x (codes, signs, norms) into the ring; warp 16 also
+//               copies each group's query operand into one of two buffers.  A
+//               ring stage is free once the tile's expansion group (codes,
+//               signs) and epilogue group (norms) have both read it
+//   warps 18-21 MMA issue: warp 18 + j issues every MMA of the tiles in slot j
 // A tcgen05.mma stream from one thread costs about a hundred cycles per
 // instruction at these shapes, while streams from different warps into
 // different accumulators overlap on the tensor core: hence one issuer per slot.
@@ -238,13 +250,14 @@ __global__ void __launch_bounds__(256) tq_scores_bbuild_kernel(const tq_params p
 // phases are waited for in order by one consumer: a wait on a phase parity
 // then never meets its barrier a phase behind (which would pass at once) or
 // two phases ahead (which would never pass).
-constexpr int kStages = 8;
+constexpr int kStages = 12;  // even: stage st only ever holds tiles of parity st % 2
 constexpr int kMaxSlots = 4;
 constexpr int kExpWarps = 8, kEpiWarps = 8;
-constexpr int kEpiWarp0 = kExpWarps, kProdWarp = kExpWarps + kEpiWarps, kIssWarp0 = kProdWarp + 1;
+constexpr int kEpiWarp0 = kExpWarps, kProdWarp = kExpWarps + kEpiWarps, kIssWarp0 = kProdWarp + 2;
 constexpr int kThreads = 32 * (kIssWarp0 + kMaxSlots);
 
-__host__ __device__ inline int ring_stage_bytes(int W, int MS) { return kKeys * (W + MS) * 4; }
+// one ring stage: codes [128][W], signs [128][MS], norms [128], rnorms [128]
+__host__ __device__ inline int ring_stage_bytes(int W, int MS) { return kKeys * (W + MS + 2) * 4; }
 
 // Position of a block's tile in (group, first key): one division at the start,
 // then a running count (a 64-bit division per tile costs hundreds of cycles in
@@ -308,7 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) {
       tqtc::mbar_init(&ring_full[i], 1);
-      tqtc::mbar_init(&ring_empty[i], 128);
+      tqtc::mbar_init(&ring_empty[i], RING ? 256 : 128);
     }
     for (int i = 0; i < NI; ++i) {
       tqtc::mbar_init(&a_full[i], 128);
@@ -334,26 +347,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     s_abort = 1;
   };
 
-  if (warp == kProdWarp) {
-    // ---------------------------------------------------------- producer
+  if (warp == kProdWarp || warp == kProdWarp + 1) {
+    // ---------------------------------------------------------- producers
+    const int px = warp - kProdWarp;  // tile parity of this producer
     if (lane == 0) {
       int64_t cur = -1, issued = 0;
       int gi = -1;
       TileCursor tc(t_begin, tiles_per_group);
+      bool dep_done = false;
       for (int64_t i = 0; i < ntl && !s_abort; ++i, tc.advance(1, tpg_keys)) {
         const int64_t grp = tc.grp;
-        if (grp != cur) {
-          cur = grp;
-          ++gi;
-          const int gb = gi & 1;
-          if (gi >= 2 && !tqtc::mbar_wait_or_abort(&b_empty[gb], (uint32_t)((gi / 2 - 1) & 1), &s_abort)) {
-            fail(tqtc::kErrCopyWait);
-            break;
-          }
-          tqtc::mbar_arrive_expect_tx(&b_full[gb], (uint32_t)bstride);
-          tqtc::bulk_g2s(bbuf + gb * bstride, ws + (size_t)grp * g.gstride, (uint32_t)bstride, &b_full[gb]);
-        }
-        if (RING) {
+        if (RING && (int)(i & 1) == px) {
           const int st = (int)(i % kStages);
           if (i >= kStages &&
               !tqtc::mbar_wait_or_abort(&ring_empty[st], (uint32_t)((i / kStages - 1) & 1), &s_abort)) {
@@ -364,16 +368,35 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int64_t rows = (T - t0) < kKeys ? (T - t0) : kKeys;
           const int64_t row0 = grp * T + t0;
           unsigned char* dst = ring + (size_t)st * sbytes;
-          const uint32_t bc = (uint32_t)(rows * W * 4), bs = (uint32_t)(rows * MS * 4);
-          tqtc::mbar_arrive_expect_tx(&ring_full[st], bc + bs);
+          const uint32_t bc = (uint32_t)(rows * W * 4), bs = (uint32_t)(rows * MS * 4), bn = (uint32_t)(rows * 4);
+          tqtc::mbar_arrive_expect_tx(&ring_full[st], bc + bs + (MS > 0 ? 2u : 1u) * bn);
           tqtc::bulk_g2s(dst, K.codes + row0 * W, bc, &ring_full[st]);
           if (MS > 0) tqtc::bulk_g2s(dst + kKeys * W * 4, K.signs + row0 * MS, bs, &ring_full[st]);
+          unsigned char* dn = dst + kKeys * (W + MS) * 4;
+          tqtc::bulk_g2s(dn, K.norms + row0, bn, &ring_full[st]);
+          if (MS > 0) tqtc::bulk_g2s(dn + kKeys * 4, K.rnorms + row0, bn, &ring_full[st]);
           issued = i + 1;
+        }
+        if (px == 0 && grp != cur) {
+          if (!dep_done) {  // the query image comes from the preceding prep kernel
+            asm volatile("griddepcontrol.wait;" ::: "memory");
+            dep_done = true;
+          }
+          cur = grp;
+          ++gi;
+          const int gb = gi & 1;
+          if (gi >= 2 && !tqtc::mbar_wait_or_abort(&b_empty[gb], (uint32_t)((gi / 2 - 1) & 1), &s_abort)) {
+            fail(tqtc::kErrCopyWait);
+            break;
+          }
+          tqtc::mbar_arrive_expect_tx(&b_full[gb], (uint32_t)bstride);
+          tqtc::bulk_g2s(bbuf + gb * bstride, ws + (size_t)grp * g.gstride, (uint32_t)bstride, &b_full[gb]);
         }
       }
       // let every copy still in flight land before the block exits (bounded)
       for (int64_t i = issued > kStages ? issued - kStages : 0; i < issued; ++i)
-        if (!tqtc::mbar_wait_or_abort(&ring_full[i % kStages], (uint32_t)((i / kStages) & 1), nullptr))
+        if ((int)(i & 1) == px &&
+            !tqtc::mbar_wait_or_abort(&ring_full[i % kStages], (uint32_t)((i / kStages) & 1), nullptr))
           atomicExch(p.err, tqtc::kErrCopyWait);
       for (int j = gi > 0 ? gi - 1 : 0; j <= gi; ++j)
         if (!tqtc::mbar_wait_or_abort(&b_full[j & 1], (uint32_t)((j / 2) & 1), nullptr))
@@ -416,10 +439,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tqtc::tc_fence_after();
         uint64_t desc = tqtc::smem_desc(tqtc::smem_u32(bbuf + (gi & 1) * bstride), (uint32_t)g.lbo, 128);
-#pragma unroll 1
-        for (int u = 0; u < U_MSE + MS; ++u) {
-          tqtc::mma_i8_ts(dst, a0 + 8u * (uint32_t)u, desc, (CL && u < U_MSE) ? idesc_s8 : idesc_u8, u != 0);
-          desc += step;
+        // unrolled: the issuing thread shares its SMSP with busy warps, so
+        // every instruction between two MMAs costs several cycles
+#pragma unroll
+        for (int u = 0; u < U_MSE + 8; ++u) {
+          if (u < U_MSE + MS) {
+            tqtc::mma_i8_ts(dst, a0 + 8u * (uint32_t)u, desc, (CL && u < U_MSE) ? idesc_s8 : idesc_u8, u != 0);
+            desc += step;
+          }
         }
         tqtc::mma_commit(&a_free[js]);
         tqtc::mma_commit(&d_full[js]);
@@ -571,7 +598,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     TileCursor tc(t_begin + eg, tiles_per_group);
     int64_t cur = -1;
     int bq = 0, hk = 0;
-    // the key norms come from HBM: each tile's are loaded one tile ahead
+    // the key norms: from the tile's ring stage, or (no ring) loaded from
+    // global memory one tile ahead
     auto load_norms = [&](const TileCursor& c, float& nu, float& gam) {
       const bool ok = c.t0 + et < T;
       const int64_t r = c.grp * T + c.t0 + et;
@@ -579,7 +607,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       gam = (ok && MS > 0) ? __ldg(K.rnorms + r) : 0.f;
     };
     float nxt_nu = 0.f, nxt_gam = 0.f;
-    if (eg < ntl) load_norms(tc, nxt_nu, nxt_gam);
+    if (!RING && eg < ntl) load_norms(tc, nxt_nu, nxt_gam);
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // per-query constants of the prep kernel
     for (int64_t i = eg; i < ntl; i += 2, tc.advance(2, tpg_keys)) {
       const int64_t grp = tc.grp;
       const int64_t t0 = tc.t0;
@@ -591,11 +620,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const int64_t t = t0 + et;
       const bool valid = t < T;
-      const float knu = nxt_nu, kgam = nxt_gam;
-      if (i + 2 < ntl) {
-        TileCursor nc = tc;
-        nc.advance(2, tpg_keys);
-        load_norms(nc, nxt_nu, nxt_gam);
+      float knu, kgam;
+      if constexpr (RING) {
+        const int st = (int)(i % kStages);
+        if (!tqtc::mbar_wait_or_abort(&ring_full[st], (uint32_t)((i / kStages) & 1), &s_abort)) {
+          fail(tqtc::kErrCopyWait);
+          break;
+        }
+        const float* nr = reinterpret_cast<const float*>(ring + (size_t)st * sbytes + kKeys * (W + MS) * 4);
+        knu = valid ? nr[et] : 0.f;
+        kgam = (valid && MS > 0) ? nr[kKeys + et] : 0.f;
+        tqtc::mbar_arrive(&ring_empty[st]);
+      } else {
+        knu = nxt_nu;
+        kgam = nxt_gam;
+        if (i + 2 < ntl) {
+          TileCursor nc = tc;
+          nc.advance(2, tpg_keys);
+          load_norms(nc, nxt_nu, nxt_gam);
+        }
       }
       const float* cs_all = reinterpret_cast<const float*>(ws + (size_t)grp * g.gstride + g.bbytes);
       if (!tqtc::mbar_wait_or_abort(&d_full[js], (uint32_t)((i / NI) & 1), &s_abort)) {
@@ -683,6 +726,11 @@ bool supported(const tq_params& p, int G, uint32_t* cols_out) {
   const Geom g(p, G);
   if (g.bbytes > 64 * 1024 || g.N > 256) return false;
   if (2u * g.slot_cols() > 512) return false;  // two tile slots at least
+  // query-operand buffers and key ring in the shared memory of one block
+  int W = 0;
+  for (int s = 0; s < p.nseg; ++s) W += p.bits[s] * p.pw;
+  const size_t bstride = (size_t)((g.bbytes + 16 * G + 127) / 128) * 128;
+  if (2 * bstride + (size_t)kStages * ring_stage_bytes(W, p.MS) > 224u * 1024u) return false;
   if (cols_out) *cols_out = 512;
   return true;
 }
@@ -703,7 +751,20 @@ cudaError_t launch_scores_t(const tq_params& p, const tq_compressed& K, float* l
   const int64_t tpg = (T + kKeys - 1) / kKeys;
   const int64_t ntiles = (int64_t)B * Hkv * tpg;
   const int grid = (int)std::min<int64_t>(ntiles, (int64_t)sm_count());
-  fn<<<grid, kThreads, smem, st>>>(p, K, logits, ws, Hq, Hkv, T, tpg, ntiles);
+  // programmatic dependent launch: the block's set-up and key stream overlap
+  // the tail of the prep kernel
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, fn, p, K, logits, ws, Hq, Hkv, T, tpg, ntiles);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -731,12 +792,22 @@ size_t tq_scores_tc_bytes(const tq_params& p, int B, int Hq, int Hkv) {
   return (size_t)B * Hkv * g.gstride;
 }
 
+bool tq_scores_tc_supported(const tq_params& p, int Hq, int Hkv) {
+  return Hkv > 0 && Hq % Hkv == 0 && supported(p, Hq / Hkv, nullptr);
+}
+
 cudaError_t tq_launch_scores_tc(const tq_params& p, const float* qprep, int B, int Hq, int Hkv, int64_t T,
                                 const tq_compressed& K, float* logits, void* ws_tc, cudaStream_t st) {
   uint32_t cols = 0;
   if (!supported(p, Hq / Hkv, &cols)) return cudaErrorNotSupported;
   uint8_t* ws = reinterpret_cast<uint8_t*>(ws_tc);
-  tq_scores_bbuild_kernel<<<dim3((unsigned)(B * Hkv), 8), 256, 0, st>>>(p, qprep, Hq, Hkv, ws);
+  const size_t smem = sizeof(float) * (size_t)(Hq / Hkv) * (p.d + p.m);
+  if (smem > 48 * 1024) {
+    const cudaError_t e = cudaFuncSetAttribute(tq_scores_bbuild_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  tq_scores_bbuild_kernel<<<dim3((unsigned)(B * Hkv), 8), 256, smem, st>>>(p, qprep, Hq, Hkv, ws);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   switch (p.d * 100 + p.bits[0] * 10 + (p.nseg == 2 ? p.bits[1] : 0)) {
