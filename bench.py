@@ -316,6 +316,200 @@ def cpu_oracle_sample(w: synth.Workload, budget_s: float, rank_seed: int = 0):
     return keys / secs, secs, keys, threads, desc
 
 
+# ------------------------------------------------------------ per-config
+L2_FLUSH_BYTES = 256 << 20   # twice the B200's 126 MB L2
+
+
+def timed_calls(fn, iters: int, stream, flush=None):
+    """Per-call device times (ms) with CUDA events on `stream`; `flush` (a
+    buffer larger than L2) is overwritten before every call, outside the
+    timed interval."""
+    out = []
+    for _ in range(iters):
+        if flush is not None:
+            flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        b.synchronize()
+        out.append(a.elapsed_time(b))
+    return out
+
+
+def hbm_roof(nbytes: float, ms: float, hbm: float, peak_src: str):
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(gbs / hbm, 4),
+            "traffic": None, "peak_source": f"{peak_src} hbm_gbs", "bytes_per_launch": nbytes}
+
+
+def config_longctx(tq, dev, stream, flush, iters, hbm, peak_src):
+    """Long-context scoring: 1 x 8 KV heads x 131072 keys (2 + 3 bits, m = 64),
+    32 query heads, L2 flushed before every call."""
+    w = synth.WORKLOADS["longctx"]
+    kc = tq.Codec(w.d, w.k_bits, w.k_m, w.codec_seed, device=dev.index)
+    K = tq.Compressed.empty(kc, w.n_keys, dev)
+    for h in range(w.Hkv):
+        tq.tq_quantize(kc, synth.kv_slab(w, "K", 0, h).to(dev), K.rows(h * w.T, (h + 1) * w.T))
+    q = synth.queries(w).to(dev).contiguous()
+    logits = torch.empty((w.B, w.Hq, w.T), device=dev)
+    ws = tq.workspace(tq.tq_scores_workspace_size(kc, w.B, w.Hq, w.Hkv), dev)
+    fn = lambda: tq.tq_scores(kc, q, w.B, w.Hq, w.Hkv, w.T, K, logits, ws)
+    for _ in range(3):
+        fn()
+    ms = statistics.median(timed_calls(fn, iters, stream, flush))
+    if tq.tq_codec_device_error(kc) != 0:
+        raise RuntimeError("tq_scores reported a timed-out wait (long context)")
+    krow = 4 * kc.code_words + 4 * kc.sign_words + 8
+    nbytes = w.n_keys * (krow + 4 * w.G)
+    return {"workload": w.name, "call": "tq_scores", "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "T": w.T,
+            "k_bits": list(w.k_bits), "k_m": w.k_m, "ms": round(ms, 5), "keys_per_s": w.n_keys / (ms * 1e-3),
+            "unit": "keys/s", "key_row_bytes": krow, "l2": "256 MB written before every call (outside the timing)",
+            "roofline": hbm_roof(nbytes, ms, hbm, peak_src)}
+
+
+def config_esm_prefill(tq, dev, stream, flush, iters, hbm, peak_src):
+    """Prefill quantisation, ESM-2-650M-shaped: K and V [4, 20, 4096, 64] bf16,
+    2 bits + QJL m = 64.  Two forms: keys RoPE'd by the generator then
+    tq_quantize, and raw keys through tq_quantize_rope (RoPE fused)."""
+    import dataclasses
+    w = synth.WORKLOADS["esm_prefill"]
+    d, n = w.d, w.n_keys
+    kc = tq.Codec(d, w.k_bits, w.k_m, w.codec_seed, device=dev.index)
+    vc = tq.Codec(d, w.v_bits, w.v_m, w.codec_seed + 1, device=dev.index)
+    k_rope = synth.kv_full(w, "K").reshape(-1, d).to(dev)
+    k_raw = synth.kv_full(dataclasses.replace(w, rope=False), "K").reshape(-1, d).to(dev)
+    v = synth.kv_full(w, "V").reshape(-1, d).to(dev)
+    pos = (torch.arange(n, dtype=torch.int64, device=dev) % w.T).to(torch.int32)
+    cs = tq.tq_rope_cache(w.rope_theta, d, w.T, device=dev)
+    K, V = tq.Compressed.empty(kc, n, dev), tq.Compressed.empty(vc, n, dev)
+    calls = {
+        "K": lambda: tq.tq_quantize(kc, k_rope, K),
+        "K_rope_fused": lambda: tq.tq_quantize_rope(kc, k_raw, cs, pos, K),
+        "V": lambda: tq.tq_quantize(vc, v, V),
+    }
+    ms = {}
+    for name, fn in calls.items():
+        for _ in range(3):
+            fn()
+        ms[name] = statistics.median(timed_calls(fn, iters, stream, flush))
+    for c in (kc, vc):
+        if tq.tq_codec_device_error(c) != 0:
+            raise RuntimeError("tq_quantize reported a device error (prefill)")
+    tokens = w.B * w.T
+    row_k = 4 * kc.code_words + 4 * kc.sign_words + 8
+    row_v = 4 * vc.code_words + 4 * vc.sign_words + 8
+    bytes_kv = n * (2 * d + row_k) + n * (2 * d + row_v)
+    bytes_kv_fused = bytes_kv + 4 * n          # the positions
+    sketch_flops = 2.0 * w.k_m * d * n + 2.0 * w.v_m * d * n
+    t_plain, t_fused = ms["K"] + ms["V"], ms["K_rope_fused"] + ms["V"]
+    return {"workload": w.name, "call": "tq_quantize K + V", "B": w.B, "H": w.Hkv, "T": w.T, "d": d,
+            "bits": list(w.k_bits), "m": w.k_m, "tokens_per_call": tokens,
+            "ms": {k: round(x, 5) for k, x in ms.items()},
+            "tokens_quantised_per_s": tokens / (t_plain * 1e-3), "unit": "tokens/s",
+            "tokens_quantised_per_s_rope_fused": tokens / (t_fused * 1e-3),
+            "vectors_per_s": 2 * n / (t_plain * 1e-3),
+            "sketch_tflops_achieved": round(sketch_flops / (t_plain * 1e-3) / 1e12, 3),
+            "l2": "256 MB written before every call (outside the timing)",
+            "roofline": hbm_roof(bytes_kv, t_plain, hbm, peak_src),
+            "roofline_rope_fused": hbm_roof(bytes_kv_fused, t_fused, hbm, peak_src)}
+
+
+def config_vsearch(tq, dev, stream, iters):
+    """Vector search over the 1M x 1536 compressed index, top-10 per query,
+    with recall@10 against exact fp32 inner products computed on the GPU."""
+    w = synth.VSEARCH
+    codec = tq.Codec(w.d, w.bits, w.m, w.codec_seed, device=dev.index)
+    X = tq.Compressed.empty(codec, w.n, dev)
+    X32 = torch.empty((w.n, w.d), dtype=torch.float32, device=dev)
+    for r0 in range(0, w.n, w.row_block):
+        r1 = min(w.n, r0 + w.row_block)
+        X32[r0:r1] = synth.search_rows(w, r0, r1).to(dev)
+        tq.tq_quantize(codec, X32[r0:r1], X.rows(r0, r1))
+    q = synth.search_queries(w).to(dev).contiguous()
+    idx = torch.empty((w.nq, w.k), dtype=torch.int32, device=dev)
+    sc = torch.empty((w.nq, w.k), dtype=torch.float32, device=dev)
+    ws = tq.workspace(tq.tq_search_workspace_size(codec, w.nq, w.k), dev)
+    fn = lambda: tq.tq_search_topk(codec, q, X, w.n, w.k, idx, sc, ws)
+    for _ in range(2):
+        fn()
+    ms = statistics.median(timed_calls(fn, iters, stream))
+    if tq.tq_codec_device_error(codec) != 0:
+        raise RuntimeError("tq_search_topk reported a timed-out wait")
+    # exact top-10 of the fp32 inner products, block by block
+    prev = torch.backends.cuda.matmul.allow_tf32
+    torch.backends.cuda.matmul.allow_tf32 = False
+    best_v = torch.full((w.nq, w.k), -float("inf"), device=dev)
+    best_i = torch.zeros((w.nq, w.k), dtype=torch.int64, device=dev)
+    for r0 in range(0, w.n, 131072):
+        r1 = min(w.n, r0 + 131072)
+        s = q @ X32[r0:r1].T
+        v, i = torch.topk(s, w.k, dim=1)
+        cv, ci = torch.cat([best_v, v], 1), torch.cat([best_i, i + r0], 1)
+        best_v, sel = torch.topk(cv, w.k, dim=1)
+        best_i = torch.gather(ci, 1, sel)
+    torch.backends.cuda.matmul.allow_tf32 = prev
+    got = idx.to(torch.int64)
+    hits = (got[:, :, None] == best_i[:, None, :]).any(dim=2).sum().item()
+    recall = hits / (w.nq * w.k)
+    del X32
+    peak, peak_src = load_tensor_peak()
+    pairs = w.nq * w.n
+    alg = 2.0 * (w.d + w.m) * pairs
+    ach = alg / (ms * 1e-3) / 1e12
+    return {"workload": w.name, "call": "tq_search_topk", "n": w.n, "nq": w.nq, "d": w.d, "bits": list(w.bits),
+            "m": w.m, "k": w.k, "ms": round(ms, 4), "pairs_per_s": pairs / (ms * 1e-3), "unit": "pairs/s",
+            "queries_per_s": w.nq / (ms * 1e-3), "recall_at_10": round(recall, 4),
+            "recall_reference": "exact fp32 inner products of the uncompressed rows (torch.matmul on the GPU, "
+                                "TF32 off), top-10 per query",
+            "l2": "index 616 MB read per call, larger than L2",
+            "roofline": {"bound": "tensor", "achieved": round(ach, 1), "peak": peak, "unit": "TFLOP/s",
+                         "frac": round(ach / peak, 4), "traffic": None, "peak_source": peak_src,
+                         "flops_per_launch": alg}}
+
+
+def decode_append_step(tq, layer, dev, stream, iters, hbm, peak_src):
+    """One decode step of the Llama-8B-shaped layer at 32k context: append the
+    new token's key (RoPE at its position, fused) and value into their fixed
+    slots, then tq_attend over the whole cache (the cache stays in HBM)."""
+    w = layer.w
+    d, rows = w.d, w.B * w.Hkv
+    t = w.T - 1
+    cs = tq.tq_rope_cache(10000.0, d, w.T, device=dev)
+    kn = synth.gaussian_rows(31, rows, d, dtype=torch.bfloat16).to(dev)
+    vn = synth.gaussian_rows(32, rows, d, dtype=torch.bfloat16).to(dev)
+
+    def step():
+        tq.tq_append(layer.kc, kn, t, w.T, layer.K, cs)
+        tq.tq_append(layer.vc, vn, t, w.T, layer.V)
+        tq.tq_attend(layer.kc, layer.vc, layer.q, w.B, w.Hq, w.Hkv, w.T, layer.K, layer.V, layer.out, layer.ws_a)
+
+    for _ in range(3):
+        step()
+    ms = statistics.median(timed_calls(step, iters, stream))
+    for c in (layer.kc, layer.vc):
+        if tq.tq_codec_device_error(c) != 0:
+            raise RuntimeError("append/attend reported a device error")
+    krow = 4 * layer.kc.code_words + 4 * layer.kc.sign_words + 8
+    vrow = 4 * layer.vc.code_words + 4 * layer.vc.sign_words + 4
+    nbytes = w.n_keys * (krow + vrow) + rows * 2 * (2 * d + krow)
+    return {"workload": w.name, "step": "tq_append K (RoPE fused) + tq_append V + tq_attend", "T": w.T,
+            "ms": round(ms, 5), "decode_tokens_per_s": w.B / (ms * 1e-3), "unit": "tokens/s",
+            "keys_attended_per_s": w.n_keys / (ms * 1e-3), "roofline": hbm_roof(nbytes, ms, hbm, peak_src)}
+
+
+def run_configs(tq, layer, dev, stream, iters: int):
+    hbm, peak_src = load_peaks()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    out = {"decode_append_attend": decode_append_step(tq, layer, dev, stream, iters, hbm, peak_src)}
+    out["longctx"] = config_longctx(tq, dev, stream, flush, iters, hbm, peak_src)
+    out["esm_prefill"] = config_esm_prefill(tq, dev, stream, flush, iters, hbm, peak_src)
+    del flush
+    torch.cuda.empty_cache()
+    out["vsearch"] = config_vsearch(tq, dev, stream, max(3, iters // 4))
+    return out
+
+
 # ------------------------------------------------------------------- main
 def run_reference(args, rank, world):
     """The oracle as the reference arm: rank 0 only, bounded samples per step."""
@@ -503,6 +697,9 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-step-seconds", type=float, default=3.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--config-iters", type=int, default=20,
+                    help="timed calls per per-config measurement (long context, prefill, search, decode "
+                         "append); 0 skips them")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -587,6 +784,7 @@ def main():
         pg.destroy_process_group()
     if rank != 0:
         return 0
+    configs = run_configs(tq, layer, dev, stream, args.config_iters) if world == 1 and args.config_iters > 0 else None
 
     hbm, peak_src = load_peaks()
     alg, rows = layer.algorithmic_bytes()
@@ -614,8 +812,6 @@ def main():
                    "step": "tq_quantize K, tq_quantize V, tq_scores, tq_attend",
                    "l2": "inputs larger than L2: 1.07 GB of bf16 K/V read per step",
                    "key_row_bytes": rows["key_row"], "value_row_bytes": rows["value_row"]},
-        "tokens_quantised_per_s": w.B * w.T * world / ((stages["tq_quantize_K"]["ms"] + stages["tq_quantize_V"]["ms"])
-                                                       * 1e-3),
         "stages": stages,
         "exact_rows_per_call": {"K": exact_k, "V": exact_v, "of": w.n_keys},
         "roofline": roof(dom),
@@ -625,10 +821,18 @@ def main():
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "clocks": clocks.summary(t_wall0, t_wall1),
     }
+    if configs is not None:
+        line["tokens_quantised_per_s"] = configs["esm_prefill"]["tokens_quantised_per_s"]
+        line["configs"] = configs
     if world == 1 and not args.no_cpu_baseline:
+        from threadpoolctl import threadpool_limits
         kps, secs, keys, threads, desc = cpu_oracle_sample(w, args.cpu_seconds)
         line["cpu_baseline"] = {"value": kps, "unit": "keys/s", "cores": threads, "kind": "oracle",
-                                "sample": desc, "seconds": round(secs, 2)}
+                                "sample": desc, "seconds": round(secs, 2), "nproc": os.cpu_count()}
+        with threadpool_limits(limits=1):
+            kps1, secs1, _, _, _ = cpu_oracle_sample(w, args.cpu_seconds)
+        line["cpu_baseline_single_thread"] = {"value": kps1, "unit": "keys/s", "cores": 1, "kind": "oracle",
+                                              "sample": desc, "seconds": round(secs1, 2)}
     print(json.dumps(line), flush=True)
     return 0
 

@@ -164,6 +164,59 @@ TQ_API tq_status tq_quantize(const tq_codec *codec, const void *x, tq_dtype dtyp
                       int64_t n, int64_t ld, const tq_compressed *out,
                       void *stream);
 
+/* Rotary position embedding fused into the encoder (TurboESM page, "Resumo
+ * tecnico" section 2, "Pipeline de Transformacao Ortogonal Invariante ao
+ * RoPE": RoPE is applied first and the orthogonal rotation after it, so the
+ * attention scores of the rotated vectors equal those of the RoPE'd ones).
+ * Rotate-half convention, pairs (i, i + d/2), theta_i = theta^(-2i/d):
+ *   x'_i       = x_i cos(pos theta_i) - x_{i+d/2} sin(pos theta_i)
+ *   x'_{i+d/2} = x_i sin(pos theta_i) + x_{i+d/2} cos(pos theta_i),  i < d/2.
+ *   cos_sin    device [max_pos][d] fp32, 16-byte aligned: entry (pos, i) is
+ *              cos(pos theta_i) for i < d/2 and sin(pos theta_{i-d/2}) for
+ *              i >= d/2 (tq_rope_cache fills it)
+ *   positions  device [n] int32, the position of each row (tq_quantize_rope);
+ *              tq_append ignores it (every appended row is at position t).
+ * x' is evaluated in fp32 with a fixed operation order and then encoded
+ * exactly as tq_quantize encodes an fp32 row; it differs from real-arithmetic
+ * RoPE by a few fp32 rounding errors, so only coordinates whose rotated value
+ * lies within about 1e-6 of a decision boundary can take the other code.     */
+typedef struct {
+  const float *cos_sin;
+  int32_t max_pos;
+  const int32_t *positions;
+} tq_rope;
+
+/* Fill a cos/sin cache [max_pos][d] for tq_rope on the current device (fp64
+ * arithmetic, rounded to fp32).  theta > 1 (10000 for the ESM-2 and Llama
+ * models), d even.                                                          */
+TQ_API tq_status tq_rope_cache(double theta, int d, int max_pos, float *cos_sin,
+                               void *stream);
+
+/* tq_quantize of the RoPE'd rows: row i is rotated by RoPE at position
+ * rope->positions[i] before normalisation.  A position outside [0, max_pos)
+ * is replaced by 0 and recorded as code 3 in the codec's device error word
+ * (tq_codec_device_error).  Requires d = 64 or 128, TQ_BF16 or TQ_F32 rows
+ * and m <= 256 (else TQ_ERR_UNSUPPORTED).                                    */
+TQ_API tq_status tq_quantize_rope(const tq_codec *codec, const void *x, tq_dtype dtype,
+                                  int64_t n, int64_t ld, const tq_rope *rope,
+                                  const tq_compressed *out, void *stream);
+
+/* Single-token decode append: compress one new row per (batch, KV head) into
+ * its fixed slot of the cache (FibQuant page, section 1: every token's record
+ * has a fixed size and address, so any token is written and decoded on its
+ * own).
+ *   x      [rows][ld] new key or value rows, row r = b * Hkv + h_kv
+ *   cache  compressed arrays of rows * T rows; row r goes to cache row
+ *          r * T + t, the layout tq_scores and tq_attend read
+ *   t      position of the new token, 0 <= t < T
+ *   rope   NULL, or the RoPE of the new rows at position t (t < max_pos;
+ *          positions is ignored)
+ * Other rows of the cache are not touched.  With RoPE the same shape limits
+ * as tq_quantize_rope apply.                                                  */
+TQ_API tq_status tq_append(const tq_codec *codec, const void *x, tq_dtype dtype,
+                           int64_t rows, int64_t ld, const tq_rope *rope, int64_t t,
+                           int64_t T, const tq_compressed *cache, void *stream);
+
 /* Workspace bytes for tq_scores with B batches of Hq query heads over Hkv KV
  * heads (the query side is prepared per (batch, KV head) group).            */
 TQ_API tq_status tq_scores_workspace_size(const tq_codec *kc, int B, int Hq,

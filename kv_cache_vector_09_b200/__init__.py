@@ -41,6 +41,10 @@ class tq_compressed(ctypes.Structure):
                 ("rnorms", ctypes.c_void_p)]
 
 
+class tq_rope(ctypes.Structure):
+    _fields_ = [("cos_sin", ctypes.c_void_p), ("max_pos", ctypes.c_int32), ("positions", ctypes.c_void_p)]
+
+
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: build it with `python kv_cache_vector_09_b200/build.py`")
@@ -53,6 +57,9 @@ def _load() -> ctypes.CDLL:
         "tq_codec_export": [P, P, P, P, P],
         "tq_codec_layout": [P, ctypes.POINTER(I), ctypes.POINTER(I)],
         "tq_quantize": [P, P, I, I64, I64, P, P],
+        "tq_rope_cache": [ctypes.c_double, I, I, P, P],
+        "tq_quantize_rope": [P, P, I, I64, I64, P, P, P],
+        "tq_append": [P, P, I, I64, I64, P, I64, I64, P, P],
         "tq_scores_workspace_size": [P, I, I, I, ctypes.POINTER(SZ)],
         "tq_scores": [P, P, I, I, I, I, I64, P, P, P, SZ, P],
         "tq_scores_noalloc": [P, P, I, I, I, I, I64, P, P, P],
@@ -195,6 +202,46 @@ def tq_quantize(codec: Codec, x: torch.Tensor, out: Compressed, stream=None) -> 
     _check(_lib.tq_quantize(codec.handle, x.data_ptr(), _DTYPES[x.dtype], x.shape[0], x.stride(0),
                             ctypes.byref(st), _stream(stream)), "tq_quantize")
     return out
+
+
+def tq_rope_cache(theta: float, d: int, max_pos: int, device=None, stream=None) -> torch.Tensor:
+    """RoPE cos/sin cache [max_pos, d] fp32 on the device (cos(pos theta_i) in
+    columns i < d/2, sin(pos theta_i) in columns d/2 + i)."""
+    device = device if device is not None else torch.device("cuda", torch.cuda.current_device())
+    cs = torch.empty((max_pos, d), dtype=torch.float32, device=device)
+    _check(_lib.tq_rope_cache(float(theta), d, max_pos, cs.data_ptr(), _stream(stream)), "tq_rope_cache")
+    return cs
+
+
+def _rope_struct(cos_sin: torch.Tensor, positions: Optional[torch.Tensor]) -> tq_rope:
+    assert cos_sin.dtype == torch.float32 and cos_sin.is_contiguous()
+    if positions is not None:
+        assert positions.dtype == torch.int32 and positions.is_contiguous()
+    return tq_rope(cos_sin.data_ptr(), cos_sin.shape[0], _ptr(positions))
+
+
+def tq_quantize_rope(codec: Codec, x: torch.Tensor, cos_sin: torch.Tensor, positions: torch.Tensor,
+                     out: Compressed, stream=None) -> Compressed:
+    """Compress the rows of x after rotate-half RoPE at positions[i] (int32)."""
+    assert x.dim() == 2 and x.stride(1) == 1, "x must be [n, ld] with contiguous rows"
+    st = out.struct()
+    rp = _rope_struct(cos_sin, positions)
+    _check(_lib.tq_quantize_rope(codec.handle, x.data_ptr(), _DTYPES[x.dtype], x.shape[0], x.stride(0),
+                                 ctypes.byref(rp), ctypes.byref(st), _stream(stream)), "tq_quantize_rope")
+    return out
+
+
+def tq_append(codec: Codec, x: torch.Tensor, t: int, T: int, cache: Compressed, cos_sin: Optional[torch.Tensor] = None,
+              stream=None) -> Compressed:
+    """Compress row r of x ([rows, ld]) into cache row r * T + t, after RoPE at
+    position t when cos_sin is given."""
+    assert x.dim() == 2 and x.stride(1) == 1, "x must be [rows, ld] with contiguous rows"
+    st = cache.struct()
+    rp = _rope_struct(cos_sin, None) if cos_sin is not None else None
+    _check(_lib.tq_append(codec.handle, x.data_ptr(), _DTYPES[x.dtype], x.shape[0], x.stride(0),
+                          ctypes.byref(rp) if rp is not None else None, t, T, ctypes.byref(st), _stream(stream)),
+           "tq_append")
+    return cache
 
 
 def tq_scores_workspace_size(kc: Codec, B: int, Hq: int, Hkv: int) -> int:

@@ -246,6 +246,7 @@ extern "C" tq_status tq_codec_create(const tq_spec* spec, int device, tq_codec**
   const int d = spec->d, m = spec->m;
   tq_params& p = c->p;
   std::memset(&p, 0, sizeof p);
+  p.out_stride = 1;  // compressed row r is output row r (tq_append changes the map per call)
   p.d = d;
   p.nseg = spec->nseg;
   p.seg_len = d / spec->nseg;
@@ -499,6 +500,93 @@ extern "C" tq_status tq_quantize(const tq_codec* c, const void* x, tq_dtype dt, 
   cudaError_t e = tq_launch_quantize_tc(c->p, x, dt, n, ld, *out, (cudaStream_t)stream);
   if (e == cudaErrorNotSupported) e = tq_launch_quantize(c->p, x, dt, n, ld, *out, (cudaStream_t)stream);
   return launch_status(e, "tq_quantize launch");
+}
+
+// row checks shared by tq_quantize_rope and tq_append
+static tq_status check_rows(const tq_codec* c, const void* x, tq_dtype dt, int64_t n, int64_t ld, const char* name) {
+  tq_status st = check_device_codec(c, name);
+  if (st != TQ_OK) return st;
+  if ((st = check_dtype(dt)) != TQ_OK) return st;
+  if (n < 0) return tq_fail(TQ_ERR_INVALID_ARG, "%s: n = %lld", name, (long long)n);
+  if (ld < c->p.d) return tq_fail(TQ_ERR_INVALID_ARG, "%s: ld %lld < d %d", name, (long long)ld, c->p.d);
+  if ((ld * (int64_t)dtype_size(dt)) % 16 != 0)
+    return tq_fail(TQ_ERR_INVALID_ARG, "%s: row pitch %lld bytes is not a multiple of 16", name,
+                   (long long)(ld * (int64_t)dtype_size(dt)));
+  if (n > 0 && (!x || !aligned16(x))) return tq_fail(TQ_ERR_INVALID_ARG, "%s: x null or not 16-byte aligned", name);
+  return TQ_OK;
+}
+
+static tq_status check_rope(const tq_codec* c, const tq_rope* rope, bool need_positions, const char* name) {
+  if (!rope) return tq_fail(TQ_ERR_INVALID_ARG, "%s: rope null", name);
+  if (!rope->cos_sin || !aligned16(rope->cos_sin))
+    return tq_fail(TQ_ERR_INVALID_ARG, "%s: rope cos_sin null or not 16-byte aligned", name);
+  if (rope->max_pos <= 0) return tq_fail(TQ_ERR_INVALID_ARG, "%s: rope max_pos = %d", name, (int)rope->max_pos);
+  if (need_positions && (!rope->positions || ((uintptr_t)rope->positions & 3u)))
+    return tq_fail(TQ_ERR_INVALID_ARG, "%s: rope positions null or not 4-byte aligned", name);
+  if (c->p.d % 2 != 0) return tq_fail(TQ_ERR_UNSUPPORTED, "%s: odd d", name);
+  return TQ_OK;
+}
+
+extern "C" tq_status tq_rope_cache(double theta, int d, int max_pos, float* cos_sin, void* stream) {
+  const tqtrace::Range trace("tq_rope_cache");
+  if (!(theta > 1.0) || d <= 0 || d % 2 != 0 || max_pos < 0)
+    return tq_fail(TQ_ERR_INVALID_ARG, "tq_rope_cache: theta %g, d %d, max_pos %d", theta, d, max_pos);
+  if (max_pos == 0) return TQ_OK;
+  if (!cos_sin || !aligned16(cos_sin)) return tq_fail(TQ_ERR_INVALID_ARG, "tq_rope_cache: cos_sin null or misaligned");
+  return launch_status(tq_launch_rope_cache(theta, d, max_pos, cos_sin, (cudaStream_t)stream), "tq_rope_cache launch");
+}
+
+extern "C" tq_status tq_quantize_rope(const tq_codec* c, const void* x, tq_dtype dt, int64_t n, int64_t ld,
+                                      const tq_rope* rope, const tq_compressed* out, void* stream) {
+  const tqtrace::Range trace("tq_quantize_rope");
+  tq_status st = check_rows(c, x, dt, n, ld, "tq_quantize_rope");
+  if (st != TQ_OK) return st;
+  if ((st = check_rope(c, rope, true, "tq_quantize_rope")) != TQ_OK) return st;
+  if (n == 0) return TQ_OK;
+  if ((st = check_compressed(c, out, "out")) != TQ_OK) return st;
+  tq_params p = c->p;
+  p.rope_cs = rope->cos_sin;
+  p.rope_pos = rope->positions;
+  p.rope_max_pos = rope->max_pos;
+  const cudaError_t e = tq_launch_quantize_tc_rope(p, x, dt, n, ld, *out, (cudaStream_t)stream);
+  if (e == cudaErrorNotSupported)
+    return tq_fail(TQ_ERR_UNSUPPORTED, "tq_quantize_rope: needs d of 64 or 128, bf16 or fp32 rows and m <= 256");
+  return launch_status(e, "tq_quantize_rope launch");
+}
+
+extern "C" tq_status tq_append(const tq_codec* c, const void* x, tq_dtype dt, int64_t rows, int64_t ld,
+                               const tq_rope* rope, int64_t t, int64_t T, const tq_compressed* cache, void* stream) {
+  const tqtrace::Range trace("tq_append");
+  tq_status st = check_rows(c, x, dt, rows, ld, "tq_append");
+  if (st != TQ_OK) return st;
+  if (T <= 0 || t < 0 || t >= T)
+    return tq_fail(TQ_ERR_INVALID_ARG, "tq_append: position t = %lld outside [0, T = %lld)", (long long)t,
+                   (long long)T);
+  if (rope) {
+    if ((st = check_rope(c, rope, false, "tq_append")) != TQ_OK) return st;
+    if (t >= rope->max_pos)
+      return tq_fail(TQ_ERR_INVALID_ARG, "tq_append: t = %lld beyond the RoPE cache (%d positions)", (long long)t,
+                     (int)rope->max_pos);
+  }
+  if (rows == 0) return TQ_OK;
+  if ((st = check_compressed(c, cache, "cache")) != TQ_OK) return st;
+  tq_params p = c->p;
+  p.out_stride = T;  // input row r -> cache row r * T + t
+  p.out_offset = t;
+  cudaError_t e;
+  if (rope) {
+    p.rope_cs = rope->cos_sin;
+    p.rope_pos = nullptr;
+    p.rope_pos_fixed = (int)t;
+    p.rope_max_pos = rope->max_pos;
+    e = tq_launch_quantize_tc_rope(p, x, dt, rows, ld, *cache, (cudaStream_t)stream);
+    if (e == cudaErrorNotSupported)
+      return tq_fail(TQ_ERR_UNSUPPORTED, "tq_append with RoPE: needs d of 64 or 128, bf16 or fp32 rows and m <= 256");
+  } else {
+    e = tq_launch_quantize_tc(p, x, dt, rows, ld, *cache, (cudaStream_t)stream);
+    if (e == cudaErrorNotSupported) e = tq_launch_quantize(p, x, dt, rows, ld, *cache, (cudaStream_t)stream);
+  }
+  return launch_status(e, "tq_append launch");
 }
 
 static size_t qprep_bytes(const tq_params& p, size_t nq) { return align256(sizeof(float) * nq * (size_t)(p.d + p.m)); }

@@ -44,6 +44,17 @@ struct tq_params {
   const uint32_t* dmask;  // [d] 0x80000000 where D_i = -1, else 0
   const float* sl1n;      // [m] sum_i |S_ji| (natural row order)
   const float* sl2n;      // [m] ||S_j||_2
+  // fused rotate-half RoPE of tq_quantize_rope and tq_append (rope_cs null:
+  // none): cos/sin cache [rope_max_pos][d] with cos(pos theta_i) at i < d/2 and
+  // sin(pos theta_i) at d/2 + i; row r takes position rope_pos[r], or
+  // rope_pos_fixed when rope_pos is null
+  const float* rope_cs;
+  const int32_t* rope_pos;
+  int rope_max_pos;
+  int rope_pos_fixed;
+  // output rows: input row r is written to compressed row r * out_stride + out_offset
+  int64_t out_stride;
+  int64_t out_offset;
   uint32_t* err;          // device error word (bounded waits that gave up), zero when healthy
   unsigned long long* exact_rows;  // rows re-evaluated in fp64 since the last reset
   // plane identity of the symmetric codebooks: with s_k = 2 bit_k - 1,
@@ -83,6 +94,11 @@ cudaError_t tq_launch_quantize(const tq_params& p, const void* x, tq_dtype dt, i
 // has no tensor-core variant (the caller then uses the generic kernel)
 cudaError_t tq_launch_quantize_tc(const tq_params& p, const void* x, tq_dtype dt, int64_t n, int64_t ld,
                                   const tq_compressed& out, cudaStream_t st);
+// the same with the fused RoPE of p.rope_cs (tq_quantize_rope.cu)
+cudaError_t tq_launch_quantize_tc_rope(const tq_params& p, const void* x, tq_dtype dt, int64_t n, int64_t ld,
+                                       const tq_compressed& out, cudaStream_t st);
+// fills a RoPE cos/sin cache [max_pos][d] in fp64, rounded to fp32
+cudaError_t tq_launch_rope_cache(double theta, int d, int max_pos, float* cs, cudaStream_t st);
 // tensor-core scorer: whether it takes the shape, the workspace bytes it
 // needs after the query-prep block (0 if the configuration has no
 // tensor-core variant), and the launch (query image, then the scoring

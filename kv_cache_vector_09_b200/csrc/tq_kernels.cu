@@ -193,15 +193,16 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
           if (sl == (widx >> 5) && lane == (widx & 31)) cw[sl] = wv;
       }
     }
-    uint32_t* orow = out.codes + row * p.W;
+    const int64_t dst = row * p.out_stride + p.out_offset;  // compressed row written
+    uint32_t* orow = out.codes + dst * p.W;
 #pragma unroll
     for (int sl = 0; sl < SLOTS; ++sl)
       if (sl * 32 + lane < p.W) orow[sl * 32 + lane] = cw[sl];
     if (Q > 0) {
-      if (lane < Q) out.signs[row * Q + lane] = signword;
-      if (lane == 0) out.rnorms[row] = gamma;
+      if (lane < Q) out.signs[dst * Q + lane] = signword;
+      if (lane == 0) out.rnorms[dst] = gamma;
     }
-    if (lane == 0) out.norms[row] = (float)nu64;
+    if (lane == 0) out.norms[dst] = (float)nu64;
   }
 }
 

@@ -14,7 +14,7 @@ namespace tqtc {
 constexpr long long kWaitCycles = 4ll << 30;  // ~2 s at 2 GHz
 
 // error codes recorded in the device error word
-enum : uint32_t { kErrNone = 0, kErrMmaWait = 1, kErrCopyWait = 2 };
+enum : uint32_t { kErrNone = 0, kErrMmaWait = 1, kErrCopyWait = 2, kErrRopePosition = 3 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

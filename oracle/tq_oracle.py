@@ -23,6 +23,9 @@ source pages):
 * "TurboESM ...", "Resumo tecnico" section 2 (RoPE first, then the orthogonal
   rotation, so attention scores are preserved exactly; a fused decode that
   dequantises and runs an online softmax without an intermediate copy).
+  ``rope_rotate_half`` is that RoPE (rotate-half pairs (i, i + d/2), angle
+  pos * theta^(-2i/d)); the encoder of RoPE'd keys is ``quantize`` of its
+  output.
 * The estimator of <q, x> that the library evaluates is
   nu * ( <Pi q, c_hat> / sqrt(d) + ||r|| * sqrt(pi/2) / m * <S Pi q, sign(S r)> ).
 
@@ -64,6 +67,7 @@ __all__ = [
     "fd_density", "fd_normaliser", "gaussian_density", "lloyd_max", "published_codebook",
     "Compressed", "quantize", "quantize_with", "pack_codes", "unpack_codes", "pack_bits", "unpack_bits",
     "estimate_scores", "attend", "dequantize", "search_topk", "exact_topk", "topk_rows", "hadamard_block",
+    "rope_rotate_half",
 ]
 
 MASK64 = (1 << 64) - 1
@@ -136,6 +140,25 @@ def rotation_matrix(D: np.ndarray) -> np.ndarray:
     for s in range(0, d, p):
         Pi[s:s + p, s:s + p] = Hp * D[None, s:s + p] / math.sqrt(p)
     return Pi
+
+
+# --------------------------------------------------------------------------- RoPE
+def rope_rotate_half(x: np.ndarray, positions: np.ndarray, theta: float) -> np.ndarray:
+    """Rotary position embedding in the rotate-half convention, in double:
+    for i < d/2 the pair (x_i, x_{i+d/2}) of a row at position pos is rotated
+    by the angle pos * theta^(-2i/d):
+        x'_i       = x_i cos(a) - x_{i+d/2} sin(a)
+        x'_{i+d/2} = x_i sin(a) + x_{i+d/2} cos(a)."""
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    h = d // 2
+    pos = np.asarray(positions, dtype=np.float64).reshape(-1, 1)
+    ang = pos * np.power(float(theta), -2.0 * np.arange(h, dtype=np.float64) / d)[None, :]
+    c, s = np.cos(ang), np.sin(ang)
+    out = np.empty_like(x)
+    out[:, :h] = x[:, :h] * c - x[:, h:] * s
+    out[:, h:] = x[:, :h] * s + x[:, h:] * c
+    return out
 
 
 # ----------------------------------------------------------------------- codebook

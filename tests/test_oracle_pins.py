@@ -115,6 +115,45 @@ def test_rope_before_rotation_keeps_scores():
     assert np.abs(lhs - rhs).max() < 1e-11
 
 
+def test_rope_rotates_a_plane_by_position_times_frequency():
+    # d = 2: one pair rotated by pos * theta^0 = pos radians
+    out = O.rope_rotate_half(np.array([[1.0, 0.0], [0.0, 1.0]]), np.array([1, 1]), 10000.0)
+    assert np.allclose(out, [[math.cos(1), math.sin(1)], [-math.sin(1), math.cos(1)]], atol=1e-15)
+    # d = 4, theta = 100: pairs (0, 2) and (1, 3); frequencies 100^0 = 1 and
+    # 100^(-2/4) = 0.1; at position 3 the angles are 3 and 0.3 rad
+    x = np.array([[1.0, 2.0, 3.0, 4.0]])
+    a0, a1 = 3.0, 0.3
+    want = [1 * math.cos(a0) - 3 * math.sin(a0), 2 * math.cos(a1) - 4 * math.sin(a1),
+            1 * math.sin(a0) + 3 * math.cos(a0), 2 * math.sin(a1) + 4 * math.cos(a1)]
+    assert np.allclose(O.rope_rotate_half(x, np.array([3]), 100.0)[0], want, atol=1e-14)
+    # position 0 is the identity
+    y = np.random.default_rng(0).standard_normal((3, 64))
+    assert np.array_equal(O.rope_rotate_half(y, np.zeros(3), 10000.0), y)
+
+
+def test_rope_scores_depend_only_on_relative_position():
+    # <RoPE(q, a), RoPE(k, b)> depends on a - b only (and norms are kept)
+    rng = np.random.default_rng(4)
+    q, k = rng.standard_normal((2, 1, 64))
+    def dot(a, b):
+        return float(O.rope_rotate_half(q, [a], 10000.0)[0] @ O.rope_rotate_half(k, [b], 10000.0)[0])
+    assert abs(dot(5, 3) - dot(4002, 4000)) < 1e-10
+    assert abs(dot(0, 0) - float(q[0] @ k[0])) < 1e-12
+    assert abs(np.linalg.norm(O.rope_rotate_half(q, [777], 10000.0)) - np.linalg.norm(q)) < 1e-12
+
+
+def test_oracle_rope_agrees_with_the_generator_and_commutes_with_pi():
+    # two independent implementations of the same definition agree, and the
+    # rotation Pi after RoPE keeps every score (TurboESM, "Resumo tecnico" 2)
+    rng = np.random.default_rng(9)
+    x = rng.standard_normal((6, 128))
+    pos = np.array([0, 1, 2, 100, 4095, 31])
+    assert np.abs(O.rope_rotate_half(x, pos, 10000.0) - synth.rope_rotate_half(x, pos, 10000.0)).max() < 1e-12
+    Pi = O.rotation_matrix(O.rademacher_signs(2, 128))
+    r = O.rope_rotate_half(x, pos, 10000.0)
+    assert np.abs((r @ Pi.T) @ (r @ Pi.T).T - r @ r.T).max() < 1e-10
+
+
 # --------------------------------------------------------------------- codebook
 def _golden_max():
     rows = {}
