@@ -263,10 +263,14 @@ TQ_API tq_status tq_attend_workspace_size(const tq_codec *kc, const tq_codec *vc
 /* Decode attention over compressed keys and values (fused decode of the
  * TurboESM page, "Resumo tecnico" section 2): for each (b, h):
  *   p   = softmax over t of scale * logit(b, h, t)   (scale 0 -> 1/sqrt(d))
- *   out = Pi_v^T  sum_t p_t nu_v,t cen_v[code_v,t] / sqrt(d)
- * i.e. the values are dequantised with their own codec `vc` (vc->m is not
- * used) and never written out.  Shapes as tq_scores; out [B][Hq][d] fp32.
- * kc and vc must have the same d.  T >= 1.                                 */
+ *   out = Pi_v^T  sum_t p_t v~_t,  v~_t = nu_v,t cen_v[code_v,t] / sqrt(d)
+ *         + nu_v,t gamma_v,t sqrt(pi/2)/m_v S_v^T (2 bit_v,t - 1)
+ * i.e. the values are dequantised with their own codec `vc` and never
+ * written out.  When vc has a sketch (m_v > 0, at most 128) the second term,
+ * the QJL residual estimate, makes every v~_t unbiased for its value (the
+ * TurboQuant pages' unbiasing stage applied to values); with m_v = 0 it is
+ * absent.  Shapes as tq_scores; out [B][Hq][d] fp32.  kc and vc must have the
+ * same d.  T >= 1.                                                         */
 TQ_API tq_status tq_attend(const tq_codec *kc, const tq_codec *vc, const void *q,
                     tq_dtype dtype, int B, int Hq, int Hkv, int64_t T,
                     float scale, const tq_compressed *K,

@@ -22,6 +22,14 @@
 // Values (phase 3): lanes own consecutive coordinates and warps take keys in
 // turn from double-buffered cp.async tiles; the probability weights are
 // warp-uniform loads and the centroids 4-byte lane-indexed loads.
+//
+// QJL-corrected values (value codec with m > 0; TurboQuant pages: the 1-bit
+// QJL stage removes the first stage's bias): the value estimate is
+//   v~_t = nu_t (c_hat_t / sqrt(d) + gamma_t sqrt(pi/2)/m S^T s_t),
+// and attention is linear in the values, so a block also accumulates the
+// m-vector a = sum_t p_t nu_t gamma_t s_t (lane l owns entries l + 32u); the
+// combine kernel applies sqrt(pi/2)/m S^T a once per (b, h) before the
+// inverse rotation.
 #pragma once
 
 #include <math.h>
@@ -196,22 +204,28 @@ __device__ __forceinline__ void qjl_nib(const uint32_t (&s)[8], const int MS, co
   }
 }
 
-// shared-memory layout (floats), identical on host and device
+// shared-memory layout (floats), identical on host and device; vq: QJL-
+// corrected values (value sign words staged with the codes, gamma per token)
 struct AttLayout {
-  int q, nib, L, stage, total;
-  __host__ __device__ AttLayout(const tq_params& kp, const tq_params& vp, int D, int NG, int chunk_len) {
+  int q, nib, L, gm, stage, total;
+  __host__ __device__ AttLayout(const tq_params& kp, const tq_params& vp, int D, int NG, int chunk_len, bool vq) {
+    const int vms = vq ? vp.MS : 0;
     q = 0;                              // [D][NG]  q' / sqrt(d)
     nib = q + D * NG;                   // [m/4][16][NG]
     L = nib + (kp.m / 4) * 16 * NG;     // [chunk_len][NG]
-    stage = L + ((chunk_len * NG + 3) / 4) * 4;
-    const int vstage = 2 * kValTile * vp.W;
-    const int accb = kWarps * D * NG;
+    gm = L + ((chunk_len * NG + 3) / 4) * 4;  // [chunk_len] value gamma (vq only)
+    stage = gm + (vq ? ((chunk_len + 3) / 4) * 4 : 0);
+    const int vstage = 2 * kValTile * (vp.W + vms);
+    const int accb = kWarps * (D + 32 * vms) * NG;
     const int st = vstage > accb ? vstage : accb;
     total = stage + ((st + 3) / 4) * 4;
   }
 };
 
-template <int D, int NG, int KB0, int KB1>
+// floats per (b, hq, chunk) partial: acc[d], max, sum, then a[m] when vq
+__host__ __device__ inline int att_partial_stride(int d, int vm, bool vq) { return d + 2 + (vq ? vm : 0); }
+
+template <int D, int NG, int KB0, int KB1, bool VQ>
 __global__ void __launch_bounds__(kThreads, 2)
     attend_kernel(const tq_params kp, const tq_params vp, const float* __restrict__ qprep, const int Hq,
                   const int Hkv, const int nsub, const int64_t T, const float scale_log2e, const tq_compressed K,
@@ -225,10 +239,12 @@ __global__ void __launch_bounds__(kThreads, 2)
   __shared__ float s_red[kWarps][NG];
   __shared__ float s_max[NG], s_sum[NG];
 
-  const AttLayout lay(kp, vp, D, NG, chunk_len);
+  const AttLayout lay(kp, vp, D, NG, chunk_len, VQ);
   float* sq = smem + lay.q;
   float* nib = smem + lay.nib;
   float* L = smem + lay.L;
+  float* gm = smem + lay.gm;
+  const int VMS = VQ ? vp.MS : 0;  // value sign words (<= 4)
   uint32_t* stage = reinterpret_cast<uint32_t*>(smem + lay.stage);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -330,6 +346,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   for (int g = 0; g < NG; ++g) lsum[g] = 0.f;
   for (int64_t t = t0 + tid; t < t1; t += kThreads) {
     const float nv = __ldg(V.norms + rowbase + t);
+    if constexpr (VQ) gm[t - t0] = __ldg(V.rnorms + rowbase + t);
     float* lr = L + (t - t0) * NG;
 #pragma unroll
     for (int g = 0; g < NG; ++g) {
@@ -360,15 +377,24 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int boff = il & 31;
   const int vpw = vp.pw;
   const float* cenv = s_cenv[vs];
+  const int Ws = Wv + VMS;  // staged words per token: codes, then sign words
   auto issue_vals = [&](int buf, int64_t start) {
     const int n = (int)(t1 - start < kValTile ? t1 - start : kValTile);
-    uint32_t* st = stage + buf * kValTile * Wv;
+    uint32_t* st = stage + buf * kValTile * Ws;
     const uint32_t* gv = V.codes + (rowbase + start) * Wv;
     for (int idx = tid; idx < n * Wv; idx += kThreads) cp_async4(st + idx, gv + idx);
+    if constexpr (VQ) {
+      uint32_t* ss = st + kValTile * Wv;
+      const uint32_t* gs = V.signs + (rowbase + start) * VMS;
+      for (int idx = tid; idx < n * VMS; idx += kThreads) cp_async4(ss + idx, gs + idx);
+    }
   };
   QVec<NG> acc[CPL];
 #pragma unroll
   for (int r = 0; r < CPL; ++r) acc[r].zero();
+  QVec<NG> accs[VQ ? 4 : 1];  // a[lane + 32u]
+#pragma unroll
+  for (int u = 0; u < (VQ ? 4 : 1); ++u) accs[u].zero();
   __syncthreads();  // L complete
   if (t0 < t1) issue_vals(0, t0);
   cp_async_commit();
@@ -379,7 +405,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     cp_async_wait<1>();
     __syncthreads();
     const int n = (int)(t1 - tile < kValTile ? t1 - tile : kValTile);
-    const uint32_t* st = stage + (it & 1) * kValTile * Wv;
+    const uint32_t* st = stage + (it & 1) * kValTile * Ws;
     for (int kk = warp; kk < n; kk += kWarps) {
       const uint32_t* row = st + kk * Wv + woff;
       QVec<NG> p;
@@ -399,25 +425,45 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
 #pragma unroll
       for (int r = 0; r < CPL; ++r) acc[r].fma(p, ld_at(cenv, (x[r >> 2] >> (8 * (r & 3))) & 0xFFu));
+      if constexpr (VQ) {
+        const uint32_t* sw = st + kValTile * Wv + kk * VMS;
+        const float g = gm[tile + kk - t0];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (u < VMS) accs[u].fma(p, ((sw[u] >> lane) & 1u) ? g : -g);
+      }
     }
     __syncthreads();
   }
 
-  // ---- reduce the warps' partial sums and write (acc[d], max, sum)
-  float* accb = reinterpret_cast<float*>(stage);  // [kWarps][D][NG]
+  // ---- reduce the warps' partial sums and write (acc[d], max, sum[, a[m]])
+  const int DA = D + 32 * VMS;                    // accumulated entries: d values, then m sketch entries
+  const int PS = att_partial_stride(D, vp.m, VQ);
+  float* accb = reinterpret_cast<float*>(stage);  // [kWarps][DA][NG]
 #pragma unroll
   for (int r = 0; r < CPL; ++r)
 #pragma unroll
-    for (int g = 0; g < NG; ++g) accb[((size_t)warp * D + i0 + r) * NG + g] = acc[r].get(g);
+    for (int g = 0; g < NG; ++g) accb[((size_t)warp * DA + i0 + r) * NG + g] = acc[r].get(g);
+  if constexpr (VQ) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (u < VMS)
+#pragma unroll
+        for (int g = 0; g < NG; ++g) accb[((size_t)warp * DA + D + lane + 32 * u) * NG + g] = accs[u].get(g);
+  }
   __syncthreads();
-  for (int idx = tid; idx < NG * D; idx += kThreads) {
-    const int g = idx / D, i = idx % D;
+  for (int idx = tid; idx < NG * DA; idx += kThreads) {
+    const int g = idx / DA, i = idx % DA;
     if (g0 + g >= G) continue;
     float v = 0.f;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) v += accb[((size_t)w * D + i) * NG + g];
-    float* pr = partials + ((size_t)(b * Hq + hk * G + g0 + g) * nchunk + chunk) * (D + 2);
-    pr[i] = v * vp.inv_sqrt_d;
+    for (int w = 0; w < kWarps; ++w) v += accb[((size_t)w * DA + i) * NG + g];
+    float* pr = partials + ((size_t)(b * Hq + hk * G + g0 + g) * nchunk + chunk) * PS;
+    if (i < D) {
+      pr[i] = v * vp.inv_sqrt_d;
+    } else {
+      pr[D + 2 + (i - D)] = v;  // a_j, j = i - D
+    }
     if (i == 0) {
       pr[D] = s_max[g];
       pr[D + 1] = s_sum[g];
@@ -425,15 +471,15 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
 }
 
-template <int D, int NG, int KB0, int KB1>
-cudaError_t launch_attend(const tq_params& kp, const tq_params& vp, const float* qprep, int B, int Hq, int Hkv,
-                          int64_t T, float scale, const tq_compressed& K, const tq_compressed& V, float* partials,
-                          int nchunk, cudaStream_t st) {
+template <int D, int NG, int KB0, int KB1, bool VQ>
+cudaError_t launch_attend_q(const tq_params& kp, const tq_params& vp, const float* qprep, int B, int Hq, int Hkv,
+                            int64_t T, float scale, const tq_compressed& K, const tq_compressed& V, float* partials,
+                            int nchunk, cudaStream_t st) {
   const int chunk_len = (int)((T + nchunk - 1) / nchunk);
-  const AttLayout lay(kp, vp, D, NG, chunk_len);
+  const AttLayout lay(kp, vp, D, NG, chunk_len, VQ);
   const size_t smem = sizeof(float) * (size_t)lay.total;
   if (smem > 200 * 1024) return cudaErrorNotSupported;
-  auto fn = attend_kernel<D, NG, KB0, KB1>;
+  auto fn = attend_kernel<D, NG, KB0, KB1, VQ>;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int G = Hq / Hkv, nsub = (G + NG - 1) / NG;
@@ -441,6 +487,17 @@ cudaError_t launch_attend(const tq_params& kp, const tq_params& vp, const float*
   fn<<<grid, kThreads, smem, st>>>(kp, vp, qprep, Hq, Hkv, nsub, T, scale * 1.4426950408889634f, K, V, partials,
                                    nchunk, chunk_len);
   return cudaGetLastError();
+}
+
+// values with a sketch of 32, 64 or 128 rows take the QJL-corrected kernel
+template <int D, int NG, int KB0, int KB1>
+cudaError_t launch_attend(const tq_params& kp, const tq_params& vp, const float* qprep, int B, int Hq, int Hkv,
+                          int64_t T, float scale, const tq_compressed& K, const tq_compressed& V, float* partials,
+                          int nchunk, cudaStream_t st) {
+  if (vp.m == 0)
+    return launch_attend_q<D, NG, KB0, KB1, false>(kp, vp, qprep, B, Hq, Hkv, T, scale, K, V, partials, nchunk, st);
+  if (vp.m > 128) return cudaErrorNotSupported;
+  return launch_attend_q<D, NG, KB0, KB1, true>(kp, vp, qprep, B, Hq, Hkv, T, scale, K, V, partials, nchunk, st);
 }
 
 template <int D, int KB0, int KB1>

@@ -657,8 +657,11 @@ static int device_sms(int device) {
   return v;
 }
 
-static size_t attend_bytes(const tq_params& kp, int B, int Hq, int nchunk) {
-  return qprep_bytes(kp, (size_t)B * Hq) + align256(sizeof(float) * (size_t)B * Hq * nchunk * (kp.d + 2));
+// partials per (b, hq, chunk): acc[d], max, sum, and the values' sketch
+// accumulator a[m] when the value codec has m > 0 (QJL-corrected values)
+static size_t attend_bytes(const tq_params& kp, const tq_params& vp, int B, int Hq, int nchunk) {
+  return qprep_bytes(kp, (size_t)B * Hq) +
+         align256(sizeof(float) * (size_t)B * Hq * nchunk * (size_t)(kp.d + 2 + vp.m));
 }
 
 extern "C" tq_status tq_attend_workspace_size(const tq_codec* kc, const tq_codec* vc, int B, int Hq, int Hkv,
@@ -667,7 +670,7 @@ extern "C" tq_status tq_attend_workspace_size(const tq_codec* kc, const tq_codec
   tq_status st = check_heads(B, Hq, Hkv, T, "tq_attend_workspace_size");
   if (st != TQ_OK) return st;
   const int nchunk = tq_attend_chunks(B, Hq, Hkv, T, device_sms(kc->device < 0 ? 0 : kc->device));
-  *bytes = attend_bytes(kc->p, B, Hq, nchunk);
+  *bytes = attend_bytes(kc->p, vc->p, B, Hq, nchunk);
   return TQ_OK;
 }
 
@@ -690,8 +693,13 @@ extern "C" tq_status tq_attend(const tq_codec* kc, const tq_codec* vc, const voi
   if ((st = check_compressed(kc, K, "K")) != TQ_OK) return st;
   if (!V || !V->codes || !aligned16(V->codes) || !V->norms || !aligned16(V->norms))
     return tq_fail(TQ_ERR_INVALID_ARG, "tq_attend: V.codes / V.norms null or not 16-byte aligned");
+  if (vc->p.m > 0) {
+    if ((st = check_compressed(vc, V, "V")) != TQ_OK) return st;
+    if (vc->p.m > 128)
+      return tq_fail(TQ_ERR_UNSUPPORTED, "tq_attend: QJL-corrected values need a value sketch of m <= 128");
+  }
   const int nchunk = tq_attend_chunks(B, Hq, Hkv, T, device_sms(kc->device));
-  const size_t need = attend_bytes(kc->p, B, Hq, nchunk);
+  const size_t need = attend_bytes(kc->p, vc->p, B, Hq, nchunk);
   if (!workspace || !aligned16(workspace) || ws_bytes < need)
     return tq_fail(TQ_ERR_INVALID_ARG, "tq_attend: workspace null, misaligned or smaller than %zu bytes", need);
   if (scale == 0.0f) scale = kc->p.inv_sqrt_d;
@@ -701,6 +709,8 @@ extern "C" tq_status tq_attend(const tq_codec* kc, const tq_codec* vc, const voi
   cudaError_t e = tq_launch_qprep(kc->p, q, dt, B * Hq, qprep, s);
   if (e == cudaSuccess)
     e = tq_launch_attend(kc->p, vc->p, qprep, B, Hq, Hkv, T, scale, *K, *V, partials, nchunk, out, s);
+  if (e == cudaErrorNotSupported)
+    return tq_fail(TQ_ERR_UNSUPPORTED, "tq_attend: no kernel for this key layout with QJL-corrected values");
   return launch_status(e, "tq_attend launch");
 }
 

@@ -482,32 +482,53 @@ __global__ void __launch_bounds__(kAttThreads)
 }
 
 // Merge the chunks of one (b, h) and rotate back: out = D * (H acc) / sqrt(p).
+// Merges the chunks' (acc[d], max, sum[, a[m]]) by log-sum-exp weights, adds
+// the values' QJL correction sqrt(pi/2)/m S^T a when vm > 0 (a = sum_t p_t
+// nu_t gamma_t s_t, m = vm <= 128), and rotates back: out = Pi^T acc.
 template <int VPL>
 __global__ void __launch_bounds__(256)
     tq_attend_combine_kernel(const tq_params vp, const float* __restrict__ partials, const int nchunk, const int nbh,
-                             float* __restrict__ out) {
+                             const int vm, float* __restrict__ out) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int bh = blockIdx.x * (blockDim.x >> 5) + warp;
   if (bh >= nbh) return;
-  const int d = vp.d;
-  const float* pr = partials + (size_t)bh * nchunk * (d + 2);
+  const int d = vp.d, ps = d + 2 + vm;
+  const float* pr = partials + (size_t)bh * nchunk * ps;
   float M = -INFINITY;
-  for (int c = lane; c < nchunk; c += 32) M = fmaxf(M, pr[(size_t)c * (d + 2) + d]);
+  for (int c = lane; c < nchunk; c += 32) M = fmaxf(M, pr[(size_t)c * ps + d]);
   M = tq_warp_max(M);
-  float acc[VPL];
+  float acc[VPL], as[4];
 #pragma unroll
   for (int k = 0; k < VPL; ++k) acc[k] = 0.f;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) as[u] = 0.f;
   float den = 0.f;
   for (int c = 0; c < nchunk; ++c) {
-    const float* pc = pr + (size_t)c * (d + 2);
+    const float* pc = pr + (size_t)c * ps;
     const float wgt = exp2f(pc[d] - M);
     den = fmaf(pc[d + 1], wgt, den);
 #pragma unroll
     for (int k = 0; k < VPL; ++k) acc[k] = fmaf(pc[lane + 32 * k], wgt, acc[k]);
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (32 * u < vm) as[u] = fmaf(pc[d + 2 + lane + 32 * u], wgt, as[u]);
   }
   const float inv = 1.0f / den;
 #pragma unroll
   for (int k = 0; k < VPL; ++k) acc[k] *= inv;
+  if (vm > 0) {
+    // acc_i += sqrt(pi/2)/m sum_j S_ji a_j / den, rows of S read coalesced
+    for (int j = 0; j < vm; ++j) {
+      float aj = 0.f;
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (u == (j >> 5)) aj = __shfl_sync(TQ_FULL_MASK, as[u], j & 31);
+      aj *= inv * vp.qjl_coef;
+      const float* Sj = vp.S + (size_t)j * d;
+#pragma unroll
+      for (int k = 0; k < VPL; ++k) acc[k] = fmaf(__ldg(Sj + lane + 32 * k), aj, acc[k]);
+    }
+  }
   tq_fwht_warp<VPL>(acc, lane);
 #pragma unroll
   for (int k = 0; k < VPL; ++k) {
@@ -617,7 +638,7 @@ cudaError_t launch_attend_g(const tq_params& kp, const tq_params& vp, const floa
 template <int VPL>
 cudaError_t launch_combine_v(const tq_params& vp, const float* partials, int nchunk, int nbh, float* out,
                              cudaStream_t st) {
-  tq_attend_combine_kernel<VPL><<<(nbh + 7) / 8, 256, 0, st>>>(vp, partials, nchunk, nbh, out);
+  tq_attend_combine_kernel<VPL><<<(nbh + 7) / 8, 256, 0, st>>>(vp, partials, nchunk, nbh, vp.m, out);
   return cudaGetLastError();
 }
 
@@ -676,7 +697,8 @@ cudaError_t tq_launch_attend(const tq_params& kp, const tq_params& vp, const flo
                              int64_t T, float scale, const tq_compressed& K, const tq_compressed& V, float* partials,
                              int nchunk, float* out, cudaStream_t st) {
   cudaError_t e = tq_launch_attend_fused(kp, vp, qprep, B, Hq, Hkv, T, scale, K, V, partials, nchunk, st);
-  if (e == cudaErrorNotSupported) {
+  // the CUDA-core fallback has no QJL-corrected values
+  if (e == cudaErrorNotSupported && vp.m == 0) {
     auto run = [&]() -> cudaError_t {
       TQ_DISPATCH_NG(Hq / Hkv, (launch_attend_g<NG>(kp, vp, qprep, B, Hq, Hkv, T, scale, K, V, partials, nchunk, st)));
     };

@@ -394,11 +394,19 @@ def quantize_with(z: np.ndarray, y: np.ndarray, nu: np.ndarray, codec: Codec) ->
                       codes, z, margin, t, nu, gamma)
 
 
-def dequantize(comp: Compressed, codec: Codec, rotated: bool = False) -> np.ndarray:
+def dequantize(comp: Compressed, codec: Codec, rotated: bool = False, qjl: bool = False) -> np.ndarray:
     """Decoder: codes -> centroids -> inverse rotation -> times the norm.
-    ``rotated=True`` stops before the inverse rotation."""
+    ``rotated=True`` stops before the inverse rotation.  ``qjl=True`` adds the
+    QJL residual estimate, x~ = nu (c_hat / sqrt(d) + ||r|| sqrt(pi/2) / m S^T s)
+    in the rotated space with s = 2 bit - 1: since E[sign(S_j r) S_j] =
+    sqrt(2/pi) r / ||r|| for a Gaussian row S_j, it is unbiased for x over S
+    (the same correction the score estimator applies to <q, x>)."""
     codes = unpack_codes(comp.codes, codec)
     yhat = codec.coord_cen(codes) / math.sqrt(codec.d)
+    if qjl and codec.m > 0:
+        s = 2.0 * unpack_bits(comp.signs, codec.m) - 1.0
+        corr = s @ codec.S.astype(np.float64)
+        yhat = yhat + comp.rnorms.astype(np.float64)[:, None] * (math.sqrt(math.pi / 2) / codec.m) * corr
     yhat = yhat * comp.norms.astype(np.float64)[:, None]
     return yhat if rotated else yhat @ codec.Pi
 
@@ -435,13 +443,15 @@ def attend(q: np.ndarray, K: Compressed, V: Compressed, kc: Codec, vc: Codec,
            B: int, Hq: int, Hkv: int, T: int, scale: Optional[float] = None) -> np.ndarray:
     """Decode attention [B, Hq, d]: p = softmax(scale * l) over the T keys of
     the query's KV head (scale defaults to 1/sqrt(d)), then
-    out = Pi^T sum_t p_t nu_t c_hat_t / sqrt(d) with the values' own codec."""
+    out = Pi^T sum_t p_t v~_t with the values' own codec, v~ the QJL-corrected
+    rotated value when the value codec has a sketch (m > 0) and
+    nu c_hat / sqrt(d) otherwise."""
     d = kc.d
     G = Hq // Hkv
     if scale is None or scale == 0.0:
         scale = 1.0 / math.sqrt(d)
     logits = estimate_scores(q, K, kc, B, Hq, Hkv, T) * scale
-    vrot = dequantize(V, vc, rotated=True)
+    vrot = dequantize(V, vc, rotated=True, qjl=True)
     out = np.empty((B, Hq, d))
     for b in range(B):
         for h in range(Hq):

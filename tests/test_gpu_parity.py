@@ -188,24 +188,28 @@ def test_scores_match_oracle(case):
 
 # ------------------------------------------------------------------- attend
 ATTEND_CASES = [
-    # name, B, Hq, Hkv, T, d, kbits, km, vbits, scale
-    ("gqa", 2, 8, 2, 3000, 128, (3,), 128, (4,), 0.0),
-    ("t1", 1, 4, 1, 1, 128, (3,), 128, (4,), 0.0),
-    ("t5_scale", 1, 2, 2, 5, 128, (2,), 64, (3,), 0.3),
-    ("d64_g1", 3, 4, 4, 1111, 64, (2,), 64, (2,), 0.0),
-    ("g16_long", 1, 16, 1, 9000, 128, (2, 3), 64, (4,), 0.0),
+    # name, B, Hq, Hkv, T, d, kbits, km, vbits, scale, vm (value sketch rows:
+    # > 0 makes tq_attend use the QJL-corrected values)
+    ("gqa", 2, 8, 2, 3000, 128, (3,), 128, (4,), 0.0, 0),
+    ("t1", 1, 4, 1, 1, 128, (3,), 128, (4,), 0.0, 0),
+    ("t5_scale", 1, 2, 2, 5, 128, (2,), 64, (3,), 0.3, 0),
+    ("d64_g1", 3, 4, 4, 1111, 64, (2,), 64, (2,), 0.0, 0),
+    ("g16_long", 1, 16, 1, 9000, 128, (2, 3), 64, (4,), 0.0, 0),
+    ("vqjl_gqa", 2, 8, 2, 2500, 128, (3,), 128, (2,), 0.0, 128),
+    ("vqjl_t1", 1, 4, 1, 1, 128, (3,), 64, (3,), 0.0, 32),
+    ("vqjl_g8_long", 1, 8, 1, 5000, 64, (2,), 64, (2,), 0.0, 64),
 ]
 
 
 @pytest.mark.parametrize("case", ATTEND_CASES, ids=[c[0] for c in ATTEND_CASES])
 def test_attend_matches_oracle(case):
-    name, B, Hq, Hkv, T, d, kb, km, vb, scale = case
+    name, B, Hq, Hkv, T, d, kb, km, vb, scale, vm = case
     dtype = torch.bfloat16
     k = synth.heavy_rows(T + 1, B * Hkv * T, d, n_out=2, dtype=dtype)
     v = synth.heavy_rows(T + 2, B * Hkv * T, d, n_out=2, dtype=dtype)
     q = synth.gaussian_rows(T + 3, B * Hq, d, dtype=dtype).reshape(B, Hq, d) * 2.0
-    kc, vc = tq.Codec(d, kb, km, 0), tq.Codec(d, vb, 0, 1)
-    okc, ovc = o_codec(d, kb, km, 0), o_codec(d, vb, 0, 1)
+    kc, vc = tq.Codec(d, kb, km, 0), tq.Codec(d, vb, vm, 1)
+    okc, ovc = o_codec(d, kb, km, 0), o_codec(d, vb, vm, 1)
     K, V = gpu_quantize(kc, k), gpu_quantize(vc, v)
     ws = tq.workspace(tq.tq_attend_workspace_size(kc, vc, B, Hq, Hkv, T), DEV)
     out = torch.empty((B, Hq, d), device=DEV)
@@ -216,18 +220,46 @@ def test_attend_matches_oracle(case):
     Vo = O.quantize(v.to(torch.float64).numpy(), ovc)
     sk = compare_compressed(K, Ko, okc)
     sv = compare_compressed(V, Vo, ovc)
-    assert sk["code_mismatch"] == sk["sign_mismatch"] == sv["code_mismatch"] == 0, (sk, sv)
+    assert sk["code_mismatch"] == sk["sign_mismatch"] == sv["code_mismatch"] == sv["sign_mismatch"] == 0, (sk, sv)
     oo = O.attend(q.to(torch.float64).numpy(), Ko, Vo, okc, ovc, B, Hq, Hkv, T, scale=scale or None)
     err = attend_errors(out.cpu().numpy().astype(np.float64), oo)
     assert err.max() <= ATTEND_RTOL, err.max()
     # isolated: oracle-compressed keys and values
     out2 = torch.empty_like(out)
-    tq.tq_attend(kc, vc, qg, B, Hq, Hkv, T, oracle_compressed_to_gpu(Ko, km), oracle_compressed_to_gpu(Vo, 0),
+    tq.tq_attend(kc, vc, qg, B, Hq, Hkv, T, oracle_compressed_to_gpu(Ko, km), oracle_compressed_to_gpu(Vo, vm),
                  out2, ws, scale=scale)
     torch.cuda.synchronize()
     err2 = attend_errors(out2.cpu().numpy().astype(np.float64), oo)
     assert err2.max() <= ATTEND_RTOL, err2.max()
     print(name, "max rel err", err.max(), err2.max())
+
+
+def test_attend_qjl_values_on_the_prefill_shape():
+    # the ESM-2-shaped prefill config's keys (after RoPE) and values, both
+    # 2 bits + QJL m = 64: one full (batch, head) slab of 4096 tokens attended
+    # by its query head with QJL-corrected values, against the oracle
+    w = synth.WORKLOADS["esm_prefill"]
+    d, T = w.d, w.T
+    kc, vc = tq.Codec(d, w.k_bits, w.k_m, w.codec_seed), tq.Codec(d, w.v_bits, w.v_m, w.codec_seed + 1)
+    okc, ovc = o_codec(d, w.k_bits, w.k_m, w.codec_seed), o_codec(d, w.v_bits, w.v_m, w.codec_seed + 1)
+    k = synth.kv_slab(w, "K", 2, 11)
+    v = synth.kv_slab(w, "V", 2, 11)
+    q = synth.gaussian_rows(77, 1, d, dtype=torch.bfloat16).reshape(1, 1, d) * 2.0
+    Ko = O.quantize(k.to(torch.float64).numpy(), okc)
+    Vo = O.quantize(v.to(torch.float64).numpy(), ovc)
+    ws = tq.workspace(tq.tq_attend_workspace_size(kc, vc, 1, 1, 1, T), DEV)
+    out = torch.empty((1, 1, d), device=DEV)
+    tq.tq_attend(kc, vc, q.to(DEV).contiguous(), 1, 1, 1, T, oracle_compressed_to_gpu(Ko, w.k_m),
+                 oracle_compressed_to_gpu(Vo, w.v_m), out, ws)
+    torch.cuda.synchronize()
+    assert tq.tq_codec_device_error(kc) == 0
+    oo = O.attend(q.to(torch.float64).numpy(), Ko, Vo, okc, ovc, 1, 1, 1, T)
+    err = attend_errors(out.cpu().numpy().astype(np.float64), oo)
+    assert err.max() <= ATTEND_RTOL, err.max()
+    # the correction is really applied: the MSE-only output is far from it
+    plain = O.attend(q.to(torch.float64).numpy(), Ko, Vo, okc, o_codec(d, w.v_bits, 0, w.codec_seed + 1),
+                     1, 1, 1, T)
+    assert attend_errors(plain, oo).max() > 10 * ATTEND_RTOL
 
 
 # ------------------------------------------------------- full-size (sampled)

@@ -511,6 +511,48 @@ def test_attend_softmax_weights_worked_by_hand():
     want = (0.25 * vrot[0] + 0.5 * vrot[1] + 0.25 * vrot[2]) @ Pv
     assert np.abs(out1 - want).max() > 0.1 * np.abs(want).max()
 
+def test_qjl_corrected_values_are_unbiased_monte_carlo():
+    # Given the codes (fixed D), x~ = nu (c_hat/sqrt(d) + gamma sqrt(pi/2)/m
+    # S^T s) averages to x over independent Gaussian S; the MSE-only
+    # reconstruction does not.  Each S draw is a fresh seed of the generator.
+    d, m, N = 64, 32, 3000
+    rng = np.random.default_rng(12)
+    x = rng.standard_normal((1, d)) * 2.0
+    D = O.rademacher_signs(3, d)
+    draws = []
+    for k in range(N):
+        c = O.make_codec(d, (2,), m, seed=1000 + k, D=D)
+        draws.append(O.dequantize(O.quantize(x, c), c, qjl=True)[0])
+    draws = np.array(draws)
+    c0 = O.make_codec(d, (2,), m, seed=0, D=D)
+    mse_only = O.dequantize(O.quantize(x, c0), c0)[0]
+    sem = draws.std(axis=0) / math.sqrt(N)
+    assert np.all(np.abs(draws.mean(axis=0) - x[0]) < 4.5 * sem + 1e-12)
+    # the MSE-only reconstruction is off by far more than the Monte-Carlo error
+    assert np.linalg.norm(mse_only - x[0]) > 20 * np.linalg.norm(sem)
+
+
+def test_qjl_corrected_values_special_cases():
+    d = 64
+    rng = np.random.default_rng(13)
+    c = _codec(d, (3,), 64, seed=2)
+    x = rng.standard_normal((5, d))
+    comp = O.quantize(x, c)
+    # without a sketch the correction is absent
+    c0 = _codec(d, (3,), 0, seed=2)
+    comp0 = O.quantize(x, c0)
+    assert np.array_equal(O.dequantize(comp0, c0, qjl=True), O.dequantize(comp0, c0))
+    # a residual of norm zero adds nothing (gamma = 0)
+    comp.rnorms[:] = 0.0
+    assert np.allclose(O.dequantize(comp, c, qjl=True), O.dequantize(comp, c), atol=1e-15)
+    # T = 1 attention returns the corrected value itself
+    comp = O.quantize(x[:1], c)
+    kc = _codec(d, (2,), 64, seed=4)
+    K = O.quantize(rng.standard_normal((1, d)), kc)
+    out = O.attend(rng.standard_normal((1, 1, d)), K, comp, kc, c, 1, 1, 1, 1)
+    assert np.allclose(out[0, 0], O.dequantize(comp, c, qjl=True)[0], atol=1e-12)
+
+
 # ----------------------------------------------------------------------- top-k
 def test_topk_order_and_ties():
     sc = np.array([[0.5, 2.0, 2.0, -1.0, 2.0, 0.7]])
