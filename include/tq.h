@@ -86,14 +86,32 @@ typedef enum { TQ_F32 = 0, TQ_BF16 = 1, TQ_F16 = 2 } tq_dtype;
  *              multiple of 32, at most 1024
  *   seed     : draws D (splitmix64 from `seed`, top bit 1 -> -1) and S
  *              (splitmix64 from seed ^ 0x5851F42D4C957F2D, Box-Muller cosine
- *              branch on output pairs, double, rounded to fp32, row-major m x d) */
+ *              branch on output pairs, double, rounded to fp32, row-major m x d)
+ *   residual : TQ_RESIDUAL_QJL (0) or TQ_RESIDUAL_SIGN (1), see tq_residual */
 typedef struct {
   int32_t d;
   int32_t nseg;
   int32_t seg_bits[2];
   int32_t m;
   uint64_t seed;
+  int32_t residual;   /* tq_residual: form of the 1-bit residual stage */
 } tq_spec;
+
+/* Residual stage (tq_spec.residual).
+ *   TQ_RESIDUAL_QJL  : sign(S r) with the seeded Gaussian S (m rows) and
+ *                      gamma = ||r|| stored per row (the TurboQuant pages).
+ *   TQ_RESIDUAL_SIGN : one sign bit per coordinate, sign(r_i), with a constant
+ *                      magnitude mu (TurboESM page, "Resumo tecnico" section 2,
+ *                      "Correcao de Residuo QJL de 1 Bit": the sign of the
+ *                      quantisation residual per element plus a first-order
+ *                      correction by the residual's mean magnitude).  mu is
+ *                      E|z - cen[code(z)]| under the rotated-coordinate law
+ *                      f_d, computed from the codebook (no data calibration).
+ *                      Requires nseg = 1 and m = d; the codec then uses S = I,
+ *                      and the stored per-row "rnorms" hold the constant
+ *                      mu sqrt(2d/pi), so that every estimator term reads
+ *                        nu (<Pi q, cen[code]> + mu <Pi q, 2 bit - 1>) / sqrt(d). */
+typedef enum { TQ_RESIDUAL_QJL = 0, TQ_RESIDUAL_SIGN = 1 } tq_residual;
 
 /* One compressed row per vector, structure-of-arrays, all caller-owned device
  * memory with n rows:

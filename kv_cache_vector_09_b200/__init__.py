@@ -31,9 +31,12 @@ class TQError(RuntimeError):
         super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}: {detail}")
 
 
+TQ_RESIDUAL_QJL, TQ_RESIDUAL_SIGN = 0, 1
+
+
 class tq_spec(ctypes.Structure):
     _fields_ = [("d", ctypes.c_int32), ("nseg", ctypes.c_int32), ("seg_bits", ctypes.c_int32 * 2),
-                ("m", ctypes.c_int32), ("seed", ctypes.c_uint64)]
+                ("m", ctypes.c_int32), ("seed", ctypes.c_uint64), ("residual", ctypes.c_int32)]
 
 
 class tq_compressed(ctypes.Structure):
@@ -122,10 +125,13 @@ def tq_make_codebook(bits: int, d: int, tol: float = 0.0, max_iter: int = 0) -> 
 class Codec:
     """A tq_codec handle (freed with the object)."""
 
-    def __init__(self, d: int, seg_bits: Sequence[int], m: int, seed: int = 0, device: int = 0):
+    def __init__(self, d: int, seg_bits: Sequence[int], m: int, seed: int = 0, device: int = 0,
+                 residual: int = TQ_RESIDUAL_QJL):
         seg_bits = tuple(int(b) for b in seg_bits)
         self.d, self.seg_bits, self.m, self.seed, self.device = d, seg_bits, m, seed, device
-        spec = tq_spec(d, len(seg_bits), (ctypes.c_int32 * 2)(*(seg_bits + (0,) * (2 - len(seg_bits)))), m, seed)
+        self.residual = residual
+        spec = tq_spec(d, len(seg_bits), (ctypes.c_int32 * 2)(*(seg_bits + (0,) * (2 - len(seg_bits)))), m, seed,
+                       residual)
         h = ctypes.c_void_p()
         _check(_lib.tq_codec_create(ctypes.byref(spec), device, ctypes.byref(h)), "tq_codec_create")
         self._h = h

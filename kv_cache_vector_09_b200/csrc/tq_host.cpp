@@ -227,7 +227,31 @@ static tq_status check_spec(const tq_spec* s) {
       return tq_fail(TQ_ERR_INVALID_ARG, "seg_bits[%d] = %d not in 1..4", i, s->seg_bits[i]);
   if (s->m < 0 || s->m % 32 != 0 || s->m > TQ_MAX_M)
     return tq_fail(TQ_ERR_INVALID_ARG, "m = %d: need 0 or a multiple of 32 up to %d", s->m, TQ_MAX_M);
+  if (s->residual != TQ_RESIDUAL_QJL && s->residual != TQ_RESIDUAL_SIGN)
+    return tq_fail(TQ_ERR_INVALID_ARG, "residual = %d: need TQ_RESIDUAL_QJL or TQ_RESIDUAL_SIGN", s->residual);
+  if (s->residual == TQ_RESIDUAL_SIGN && (s->nseg != 1 || s->m != d))
+    return tq_fail(TQ_ERR_INVALID_ARG, "TQ_RESIDUAL_SIGN needs one segment and m = d (got nseg %d, m %d)", s->nseg,
+                   s->m);
   return TQ_OK;
+}
+
+// Mean residual magnitude mu = E|z - cen[code(z)]| under f_d for a published
+// codebook (fp32 centroids and boundaries, ascending): per cell, split at its
+// centroid,
+//   int_cell |z - c| f = c (P(lo, c) - P(c, hi)) - M1(lo, c) + M1(c, hi),
+// with P and M1 the probability and first moment of f_d between the limits.
+static double residual_mean_magnitude(int d, const std::vector<float>& cen, const std::vector<float>& bnd) {
+  const SphereMarginal f(d);
+  const double edge = std::sqrt((double)d);
+  double mu = 0.0;
+  const int L = (int)cen.size();
+  for (int k = 0; k < L; ++k) {
+    const double lo = k == 0 ? -edge : (double)bnd[k - 1];
+    const double hi = k == L - 1 ? edge : (double)bnd[k];
+    const double c = (double)cen[k];
+    mu += c * (f.prob(lo, c) - f.prob(c, hi)) - f.first_moment(lo, c) + f.first_moment(c, hi);
+  }
+  return mu;
 }
 
 static size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
@@ -314,7 +338,18 @@ extern "C" tq_status tq_codec_create(const tq_spec* spec, int device, tq_codec**
     }
   }
   draw_signs(spec->seed, d, c->dbits_host);
-  if (m > 0) draw_sketch(spec->seed, m, d, c->S_host);
+  if (spec->residual == TQ_RESIDUAL_SIGN) {
+    // per-element residual sign: S = I (m = d), every row's stored residual
+    // scale is the constant mu sqrt(2d/pi), so that the estimator's
+    // gamma sqrt(pi/2)/m factor equals mu / sqrt(d)
+    c->S_host.assign((size_t)d * d, 0.0f);
+    for (int i = 0; i < d; ++i) c->S_host[(size_t)i * d + i] = 1.0f;
+    c->mu = residual_mean_magnitude(d, c->cen_host[0], c->bnd_host[0]);
+    p.rnorm_const = (float)(c->mu * std::sqrt(2.0 * d / 3.14159265358979323846));
+    p.rnorm_is_const = 1;
+  } else if (m > 0) {
+    draw_sketch(spec->seed, m, d, c->S_host);
+  }
 
   if (device >= 0) {
     int cur = -1;

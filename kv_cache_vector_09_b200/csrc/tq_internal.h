@@ -52,6 +52,10 @@ struct tq_params {
   const int32_t* rope_pos;
   int rope_max_pos;
   int rope_pos_fixed;
+  // per-element residual sign (TQ_RESIDUAL_SIGN): rnorms hold this constant
+  // instead of ||r|| (0 with the QJL sketch)
+  float rnorm_const;
+  int rnorm_is_const;
   // output rows: input row r is written to compressed row r * out_stride + out_offset
   int64_t out_stride;
   int64_t out_offset;
@@ -79,6 +83,7 @@ struct tq_codec {
   std::vector<uint32_t> dbits_host; // [ceil(d/32)]
   std::vector<float> cen_host[2];
   std::vector<float> bnd_host[2];
+  double mu = 0.0;  // TQ_RESIDUAL_SIGN: mean residual magnitude (z units)
   // device allocations (one block)
   void* dev_block = nullptr;
 };

@@ -200,7 +200,7 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
       if (sl * 32 + lane < p.W) orow[sl * 32 + lane] = cw[sl];
     if (Q > 0) {
       if (lane < Q) out.signs[dst * Q + lane] = signword;
-      if (lane == 0) out.rnorms[dst] = gamma;
+      if (lane == 0) out.rnorms[dst] = p.rnorm_is_const ? p.rnorm_const : gamma;
     }
     if (lane == 0) out.norms[dst] = (float)nu64;
   }

@@ -280,7 +280,7 @@ __device__ void exact_row(const tq_params& p, const QBook& qb, const TIn* __rest
   }
   if (lane == 0) {
     out.norms[orow] = (float)nu;
-    if (MS > 0) out.rnorms[orow] = (float)sqrt(g2);
+    if (MS > 0) out.rnorms[orow] = p.rnorm_is_const ? p.rnorm_const : (float)sqrt(g2);
   }
   __syncwarp();
 }
@@ -684,7 +684,7 @@ __global__ void __launch_bounds__(kRows * (D / 32), SK ? 1 : 2)
     if (q == 0) {
       st_nu[r] = nu;
       if constexpr (SK) {
-        st_gam[r] = sqrtf(g2) / (nu * sqrtD);
+        st_gam[r] = p.rnorm_is_const ? p.rnorm_const : sqrtf(g2) / (nu * sqrtD);
         const float R2 = rscale * sqrtf(g2) * 1.00001f;
         const float E = 1.1f * (rscale * 1.1f * (kU * (float)L * sqrtD * nu + (e_nu + kU) * sqrtf(cv2) +
                                                  kU * sqrtf(g2)) +

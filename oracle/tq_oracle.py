@@ -67,7 +67,7 @@ __all__ = [
     "fd_density", "fd_normaliser", "gaussian_density", "lloyd_max", "published_codebook",
     "Compressed", "quantize", "quantize_with", "pack_codes", "unpack_codes", "pack_bits", "unpack_bits",
     "estimate_scores", "attend", "dequantize", "search_topk", "exact_topk", "topk_rows", "hadamard_block",
-    "rope_rotate_half",
+    "rope_rotate_half", "residual_mean_magnitude",
 ]
 
 MASK64 = (1 << 64) - 1
@@ -233,6 +233,20 @@ def published_codebook(bits: int, d: int) -> Tuple[np.ndarray, np.ndarray]:
 
 
 # -------------------------------------------------------------------------- codec
+def residual_mean_magnitude(cen: np.ndarray, bnd: np.ndarray, d: int) -> float:
+    """mu = E|z - cen[code(z)]| for z with density f_d and the published
+    codebook (the constant of the per-element residual sign): the integral of
+    |z - c_k| f_d(z) over every cell, by adaptive quadrature."""
+    f, edge = fd_density(d)
+    e = np.concatenate([[-edge], np.asarray(bnd, np.float64), [edge]])
+    mu = 0.0
+    for k, c in enumerate(np.asarray(cen, np.float64)):
+        for lo, hi in ((e[k], min(c, e[k + 1])), (max(c, e[k]), e[k + 1])):
+            if hi > lo:
+                mu += integrate.quad(lambda z: abs(z - c) * f(z), lo, hi, epsabs=0.0, epsrel=1e-13, limit=400)[0]
+    return mu
+
+
 @dataclasses.dataclass
 class Codec:
     d: int
@@ -243,6 +257,10 @@ class Codec:
     S: np.ndarray                     # (m, d) fp32
     cen: List[np.ndarray]             # per segment, fp32, ascending
     bnd: List[np.ndarray]             # per segment, fp32, ascending
+    # residual stage: "qjl" (sign(S r) and ||r||) or "sign" (TurboESM: sign(r_i)
+    # per coordinate and the constant mean magnitude mu; then S = I, m = d)
+    residual: str = "qjl"
+    mu: float = 0.0
 
     @property
     def nseg(self) -> int:
@@ -275,19 +293,27 @@ class Codec:
 
 
 def make_codec(d: int, seg_bits: Sequence[int], m: int, seed: int,
-               D: Optional[np.ndarray] = None, S: Optional[np.ndarray] = None) -> Codec:
-    """Codec from the seed (or from explicit D and S, for Monte-Carlo tests)."""
+               D: Optional[np.ndarray] = None, S: Optional[np.ndarray] = None, residual: str = "qjl") -> Codec:
+    """Codec from the seed (or from explicit D and S, for Monte-Carlo tests).
+    residual="sign" is TurboESM's per-element residual sign: one segment,
+    m = d, S = I, and mu from the codebook."""
     seg_bits = tuple(int(b) for b in seg_bits)
     if D is None:
         D = rademacher_signs(seed, d)
-    if S is None:
-        S = gaussian_sketch(seed, m, d) if m > 0 else np.zeros((0, d), dtype=np.float32)
     cen, bnd = [], []
     for b in seg_bits:
         c, bb = published_codebook(b, d)
         cen.append(c)
         bnd.append(bb)
-    return Codec(d, seg_bits, m, seed, np.asarray(D, dtype=np.float64), np.asarray(S), cen, bnd)
+    mu = 0.0
+    if residual == "sign":
+        if len(seg_bits) != 1 or m != d:
+            raise ValueError("the per-element residual sign needs one segment and m = d")
+        S = np.eye(d, dtype=np.float32)
+        mu = residual_mean_magnitude(cen[0], bnd[0], d)
+    elif S is None:
+        S = gaussian_sketch(seed, m, d) if m > 0 else np.zeros((0, d), dtype=np.float32)
+    return Codec(d, seg_bits, m, seed, np.asarray(D, dtype=np.float64), np.asarray(S), cen, bnd, residual, mu)
 
 
 # ---------------------------------------------------------------------- bit packing
@@ -389,9 +415,13 @@ def quantize_with(z: np.ndarray, y: np.ndarray, nu: np.ndarray, codec: Codec) ->
     else:
         t = np.zeros((z.shape[0], 0))
         signs = np.zeros((z.shape[0], 0), dtype=np.uint32)
-    return Compressed(pack_codes(codes, codec), signs, nu.astype(np.float32),
-                      gamma.astype(np.float32) if codec.m > 0 else np.zeros(0, np.float32),
-                      codes, z, margin, t, nu, gamma)
+    if codec.residual == "sign":
+        # the stored residual scale is the constant mu sqrt(2d/pi) of the
+        # format (every estimator then reads mu / sqrt(d) per sign)
+        rn = np.full(z.shape[0], np.float32(codec.mu * math.sqrt(2.0 * d / math.pi)), dtype=np.float32)
+    else:
+        rn = gamma.astype(np.float32) if codec.m > 0 else np.zeros(0, np.float32)
+    return Compressed(pack_codes(codes, codec), signs, nu.astype(np.float32), rn, codes, z, margin, t, nu, gamma)
 
 
 def dequantize(comp: Compressed, codec: Codec, rotated: bool = False, qjl: bool = False) -> np.ndarray:
@@ -403,7 +433,11 @@ def dequantize(comp: Compressed, codec: Codec, rotated: bool = False, qjl: bool 
     (the same correction the score estimator applies to <q, x>)."""
     codes = unpack_codes(comp.codes, codec)
     yhat = codec.coord_cen(codes) / math.sqrt(codec.d)
-    if qjl and codec.m > 0:
+    if qjl and codec.residual == "sign":
+        # TurboESM: the first-order correction mu sign(r_i) per coordinate
+        s = 2.0 * unpack_bits(comp.signs, codec.d) - 1.0
+        yhat = yhat + codec.mu * s / math.sqrt(codec.d)
+    elif qjl and codec.m > 0:
         s = 2.0 * unpack_bits(comp.signs, codec.m) - 1.0
         corr = s @ codec.S.astype(np.float64)
         yhat = yhat + comp.rnorms.astype(np.float64)[:, None] * (math.sqrt(math.pi / 2) / codec.m) * corr
@@ -433,7 +467,10 @@ def estimate_scores(q: np.ndarray, comp: Compressed, codec: Codec,
         for h in range(Hq):
             rows = (b * Hkv + h // G) * T + np.arange(T)
             val = chat[rows] @ qr[b, h] / math.sqrt(d)
-            if m > 0:
+            if codec.residual == "sign":
+                # TurboESM: nu (<q', c_hat> + mu <q', sign(r)>) / sqrt(d)
+                val = val + codec.mu / math.sqrt(d) * (s[rows] @ qr[b, h])
+            elif m > 0:
                 val = val + gam[rows] * math.sqrt(math.pi / 2) / m * (s[rows] @ w[b, h])
             out[b, h] = nu[rows] * val
     return out

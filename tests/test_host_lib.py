@@ -152,3 +152,16 @@ def test_bench_traffic_is_reported_only_for_the_measured_sources(monkeypatch):
     assert b.measured_traffic("tq_attend") == stale["tq_attend"][0]
     assert b.measured_traffic("no_such_stage") is None
     assert cur["tq_scores"] != cur["tq_attend"]
+
+
+def test_sign_residual_codec_checks_and_tables():
+    # TurboESM's per-element residual sign: one segment, m = d, S = I; the
+    # codec's mu equals the oracle's (independent quadratures)
+    import oracle as O
+    with pytest.raises(tq.TQError):
+        tq.Codec(128, (2, 3), 128, 0, device=-1, residual=tq.TQ_RESIDUAL_SIGN)
+    with pytest.raises(tq.TQError):
+        tq.Codec(128, (3,), 64, 0, device=-1, residual=tq.TQ_RESIDUAL_SIGN)
+    c = tq.Codec(128, (3,), 128, 0, device=-1, residual=tq.TQ_RESIDUAL_SIGN)
+    S, _, _, _ = c.export()
+    assert np.array_equal(S, np.eye(128, dtype=np.float32))

@@ -553,6 +553,72 @@ def test_qjl_corrected_values_special_cases():
     assert np.allclose(out[0, 0], O.dequantize(comp, c, qjl=True)[0], atol=1e-12)
 
 
+def _sphere_marginal_samples(d, n, seed):
+    """z = sqrt(d) u_1 for u uniform on the sphere S^{d-1} (u = g / ||g||)."""
+    rng = np.random.default_rng(seed)
+    out = np.empty(n)
+    for i in range(0, n, 4096):
+        g = rng.standard_normal((min(4096, n - i), d))
+        out[i:i + g.shape[0]] = math.sqrt(d) * g[:, 0] / np.linalg.norm(g, axis=1)
+    return out
+
+
+@pytest.mark.parametrize("bits,d", [(2, 64), (3, 128)])
+def test_residual_mean_magnitude_monte_carlo(bits, d):
+    # mu = E|z - Q(z)| under the sphere marginal, and the first-order
+    # correction by mu sign(r) lowers the squared error by exactly mu^2:
+    # E (r - mu sign r)^2 = E r^2 - 2 mu E|r| + mu^2 = D - mu^2
+    c = O.make_codec(d, (bits,), d, 0, residual="sign")
+    z = _sphere_marginal_samples(d, 200_000, bits + d)
+    cen, bnd = c.cen[0].astype(np.float64), c.bnd[0].astype(np.float64)
+    r = z - cen[np.searchsorted(bnd, z, side="right")]
+    a = np.abs(r)
+    assert abs(a.mean() - c.mu) < 4 * a.std() / math.sqrt(z.size), (a.mean(), c.mu)
+    e = (r - c.mu * np.sign(r)) ** 2
+    want = np.mean(r * r) - c.mu ** 2
+    assert abs(e.mean() - want) < 4 * e.std() / math.sqrt(z.size) + 1e-3 * want
+
+
+def test_residual_mean_magnitude_gaussian_limit():
+    # for large d the sphere marginal tends to N(0, 1) and the codebook to
+    # Max's table (fixture), so mu tends to E|Z - Q_Max(Z)|
+    rows = _golden_max()
+    levels = [v for v, _ in rows[3][0]]
+    cen = np.array(sorted([-v for v in levels] + levels))
+    bnd = 0.5 * (cen[:-1] + cen[1:])
+    phi = lambda z: math.exp(-0.5 * z * z) / math.sqrt(2 * math.pi)
+    from scipy import integrate
+    e = np.concatenate([[-np.inf], bnd, [np.inf]])
+    mu_g = 0.0
+    for k, ck in enumerate(cen):
+        mu_g += integrate.quad(lambda z: abs(z - ck) * phi(z), e[k], ck)[0]
+        mu_g += integrate.quad(lambda z: abs(z - ck) * phi(z), ck, e[k + 1])[0]
+    c = O.make_codec(1536, (3,), 1536, 0, residual="sign")
+    assert abs(c.mu - mu_g) < 3e-3, (c.mu, mu_g)
+
+
+def test_sign_residual_estimator_and_format():
+    # the estimator reads nu (<q', c_hat> + mu <q', sign(r)>) / sqrt(d): its
+    # error is smaller than the MSE-only one on average, and the stored scale
+    # is the constant mu sqrt(2d/pi)
+    d = 128
+    c = O.make_codec(d, (3,), d, 1, residual="sign")
+    c0 = O.make_codec(d, (3,), 0, 1)
+    rng = np.random.default_rng(21)
+    x = rng.standard_normal((400, d))
+    q = rng.standard_normal((1, 1, d))
+    comp, comp0 = O.quantize(x, c), O.quantize(x, c0)
+    assert np.all(comp.rnorms == np.float32(c.mu * math.sqrt(2 * d / math.pi)))
+    exact = x @ q[0, 0]
+    est = O.estimate_scores(q, comp, c, 1, 1, 1, 400)[0, 0]
+    est0 = O.estimate_scores(q, comp0, c0, 1, 1, 1, 400)[0, 0]
+    assert np.mean((est - exact) ** 2) < 0.8 * np.mean((est0 - exact) ** 2)
+    # and the corrected reconstruction is closer to x than the MSE-only one
+    err = np.linalg.norm(O.dequantize(comp, c, qjl=True) - x, axis=1)
+    err0 = np.linalg.norm(O.dequantize(comp0, c0) - x, axis=1)
+    assert np.mean(err ** 2) < np.mean(err0 ** 2)
+
+
 # ----------------------------------------------------------------------- top-k
 def test_topk_order_and_ties():
     sc = np.array([[0.5, 2.0, 2.0, -1.0, 2.0, 0.7]])
