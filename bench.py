@@ -49,15 +49,15 @@ FALLBACK_HBM_GBS = 6650.0
 # digest; after any change to them it is null until the capture is redone.
 STEP_SHARED_SOURCES = ("tq_common.cuh", "tq_internal.h", "tq_tc.cuh", "tq_host.cpp", "tq_kernels.cu", "tq_trace.h")
 STAGE_SOURCES = {
-    "tq_quantize_K": ("tq_quantize_tc.cu",),
-    "tq_quantize_V": ("tq_quantize_tc.cu",),
+    "tq_quantize_K": ("tq_quantize_tc.cu", "tq_quantize_tc.cuh"),
+    "tq_quantize_V": ("tq_quantize_tc.cu", "tq_quantize_tc.cuh"),
     "tq_scores": ("tq_scores_tc.cu",),
     "tq_attend": ("tq_attend.cuh", "tq_attend_d128.cu", "tq_attend_d64.cu"),
 }
 TRAFFIC = {  # stage: (bytes per launch, sources digest)
     "tq_quantize_K": (548_016_384 + 136_585_984, "26ada5d12091b490aedbca72de0379a59c1d43f8d2302d4423ebd3492e99b32b"),
     "tq_quantize_V": (539_167_744 + 124_734_208, "26ada5d12091b490aedbca72de0379a59c1d43f8d2302d4423ebd3492e99b32b"),
-    "tq_scores": (151_660_288 + 19_469_568, "0a5e05e82703af4d03657d7eada259f87d1a23fec455ede7a9980fa8a5360f68"),
+    "tq_scores": (152_448_768 + 20_797_440, "efc9132fa0b5f4277ea303f22773632b626ddac9682ed89271d989a890dca52c"),
     "tq_attend": (293_933_056 + 6_545_152, "853a0d84650adc29ff6221ba2b913f6880341e9e3376bae69430231e8357d47e"),
 }
 
