@@ -87,7 +87,8 @@ typedef enum { TQ_F32 = 0, TQ_BF16 = 1, TQ_F16 = 2 } tq_dtype;
  *   seed     : draws D (splitmix64 from `seed`, top bit 1 -> -1) and S
  *              (splitmix64 from seed ^ 0x5851F42D4C957F2D, Box-Muller cosine
  *              branch on output pairs, double, rounded to fp32, row-major m x d)
- *   residual : TQ_RESIDUAL_QJL (0) or TQ_RESIDUAL_SIGN (1), see tq_residual */
+ *   residual : TQ_RESIDUAL_QJL (0) or TQ_RESIDUAL_SIGN (1), see tq_residual
+ *   rotation : TQ_ROTATION_RHT (0) or TQ_ROTATION_HAAR (1), see tq_rotation  */
 typedef struct {
   int32_t d;
   int32_t nseg;
@@ -95,7 +96,21 @@ typedef struct {
   int32_t m;
   uint64_t seed;
   int32_t residual;   /* tq_residual: form of the 1-bit residual stage */
+  int32_t rotation;   /* tq_rotation: the shared random rotation Pi */
 } tq_spec;
+
+/* Rotation (tq_spec.rotation).
+ *   TQ_ROTATION_RHT  : Pi = blockdiag(H_p) diag(D) / sqrt(p), the randomized
+ *                      Hadamard transform (TurboQuant news page).
+ *   TQ_ROTATION_HAAR : a dense Haar-distributed orthogonal Pi (FibQuant page,
+ *                      section 1, step 2, "rotacao ortogonal aleatoria
+ *                      compartilhada (Haar)"): the Q of the QR factorisation,
+ *                      R with a positive diagonal, of a d x d matrix of iid
+ *                      N(0, 1) drawn like S from splitmix64(seed ^
+ *                      0x2545F4914F6CDD1D); D = I.  d <= 256; it is applied
+ *                      as dense products (encoder, query preparation, inverse
+ *                      rotation of the attention output).                    */
+typedef enum { TQ_ROTATION_RHT = 0, TQ_ROTATION_HAAR = 1 } tq_rotation;
 
 /* Residual stage (tq_spec.residual).
  *   TQ_RESIDUAL_QJL  : sign(S r) with the seeded Gaussian S (m rows) and
@@ -163,6 +178,10 @@ TQ_API tq_status tq_codec_destroy(tq_codec *codec);
  *   bnd    [sum_s 2^seg_bits[s] - 1]  per-segment boundaries, concatenated    */
 TQ_API tq_status tq_codec_export(const tq_codec *codec, float *S, uint32_t *dsigns,
                           float *cen, float *bnd);
+
+/* The codec's rotation as a dense matrix: Pi [d][d] fp32 row-major, y = Pi u
+ * (host copy, for checking; the Hadamard rotation is expanded).            */
+TQ_API tq_status tq_codec_rotation(const tq_codec *codec, float *Pi);
 
 /* Row sizes of the compressed format in 32-bit words (either pointer may be
  * NULL): code_words = W, sign_words = m / 32.                               */

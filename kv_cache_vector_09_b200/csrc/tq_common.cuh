@@ -61,3 +61,26 @@ __device__ __forceinline__ void tq_fwht_warp(F (&v)[VPL], int lane) {
 __device__ __forceinline__ bool tq_dneg(const uint32_t* dbits, int k, int lane) {
   return (__ldg(dbits + k) >> lane) & 1u;
 }
+
+// Dense rotation of a vector spread over a warp (lane holds coordinates
+// j = lane + 32 k, k < VPL, d = 32 VPL): v_j <- sum_i Pi_ji v_i with piT
+// [d][d] holding Pi_ji at (i, j), so the lanes' loads at fixed i are
+// coalesced.  buf: d elements of this warp's scratch (shared memory).
+template <int VPL, typename F>
+__device__ __forceinline__ void tq_dense_rotate_warp(F (&v)[VPL], int lane, const float* __restrict__ piT, F* buf) {
+  constexpr int d = 32 * VPL;
+#pragma unroll
+  for (int k = 0; k < VPL; ++k) buf[lane + 32 * k] = v[k];
+  __syncwarp();
+  F acc[VPL];
+#pragma unroll
+  for (int k = 0; k < VPL; ++k) acc[k] = F(0);
+  for (int i = 0; i < d; ++i) {
+    const F bi = buf[i];
+#pragma unroll
+    for (int k = 0; k < VPL; ++k) acc[k] = fma((F)__ldg(piT + (size_t)i * d + lane + 32 * k), bi, acc[k]);
+  }
+  __syncwarp();
+#pragma unroll
+  for (int k = 0; k < VPL; ++k) v[k] = acc[k];
+}

@@ -59,6 +59,43 @@ void draw_sketch(uint64_t seed, int m, int d, std::vector<float>& S) {
   }
 }
 
+// Haar rotation (tq_spec.rotation = TQ_ROTATION_HAAR): G, a d x d matrix of
+// iid N(0, 1) drawn like S from splitmix64(seed ^ kHaarSeedXor), row-major;
+// its columns are orthonormalised by Gram-Schmidt in fp64 with a second
+// reorthogonalisation pass.  The result Q has a positive diagonal in R
+// (G = QR), which makes it the unique Haar-distributed orthogonal matrix of
+// the QR of G; the rotation is Pi = Q, y = Pi u.  Returned as Pi[j][i]
+// (row-major) in fp64.
+constexpr uint64_t kHaarSeedXor = 0x2545F4914F6CDD1Dull;
+
+void draw_haar(uint64_t seed, int d, std::vector<double>& Pi) {
+  std::vector<double> G((size_t)d * d);
+  SplitMix64 g(seed ^ kHaarSeedXor);
+  const double two_pi = 6.283185307179586476925286766559;
+  for (size_t k = 0; k < G.size(); ++k) {
+    const double u1 = (double)((g.next() >> 11) + 1) * 0x1.0p-53;
+    const double u2 = (double)(g.next() >> 11) * 0x1.0p-53;
+    G[k] = std::sqrt(-2.0 * std::log(u1)) * std::cos(two_pi * u2);
+  }
+  // columns of G: col c has entries G[r * d + c]
+  Pi.assign((size_t)d * d, 0.0);
+  std::vector<double> v(d);
+  for (int c = 0; c < d; ++c) {
+    for (int r = 0; r < d; ++r) v[r] = G[(size_t)r * d + c];
+    for (int pass = 0; pass < 2; ++pass) {
+      for (int k = 0; k < c; ++k) {
+        double dot = 0.0;
+        for (int r = 0; r < d; ++r) dot += Pi[(size_t)r * d + k] * v[r];
+        for (int r = 0; r < d; ++r) v[r] -= dot * Pi[(size_t)r * d + k];
+      }
+    }
+    double nrm = 0.0;
+    for (int r = 0; r < d; ++r) nrm += v[r] * v[r];
+    nrm = std::sqrt(nrm);
+    for (int r = 0; r < d; ++r) Pi[(size_t)r * d + c] = v[r] / nrm;
+  }
+}
+
 // ----------------------------------------------------------------- Lloyd-Max
 // Gauss-Legendre rule on [-1, 1] by Newton's method on the Legendre recurrence.
 struct GaussLegendre {
@@ -229,6 +266,10 @@ static tq_status check_spec(const tq_spec* s) {
     return tq_fail(TQ_ERR_INVALID_ARG, "m = %d: need 0 or a multiple of 32 up to %d", s->m, TQ_MAX_M);
   if (s->residual != TQ_RESIDUAL_QJL && s->residual != TQ_RESIDUAL_SIGN)
     return tq_fail(TQ_ERR_INVALID_ARG, "residual = %d: need TQ_RESIDUAL_QJL or TQ_RESIDUAL_SIGN", s->residual);
+  if (s->rotation != TQ_ROTATION_RHT && s->rotation != TQ_ROTATION_HAAR)
+    return tq_fail(TQ_ERR_INVALID_ARG, "rotation = %d: need TQ_ROTATION_RHT or TQ_ROTATION_HAAR", s->rotation);
+  if (s->rotation == TQ_ROTATION_HAAR && d > 256)
+    return tq_fail(TQ_ERR_UNSUPPORTED, "TQ_ROTATION_HAAR: d = %d above 256", d);
   if (s->residual == TQ_RESIDUAL_SIGN && (s->nseg != 1 || s->m != d))
     return tq_fail(TQ_ERR_INVALID_ARG, "TQ_RESIDUAL_SIGN needs one segment and m = d (got nseg %d, m %d)", s->nseg,
                    s->m);
@@ -338,6 +379,12 @@ extern "C" tq_status tq_codec_create(const tq_spec* spec, int device, tq_codec**
     }
   }
   draw_signs(spec->seed, d, c->dbits_host);
+  if (spec->rotation == TQ_ROTATION_HAAR) {
+    // the dense Haar rotation replaces H D / sqrt(d): D = I
+    std::fill(c->dbits_host.begin(), c->dbits_host.end(), 0u);
+    draw_haar(spec->seed, d, c->haar);
+    p.haar = 1;
+  }
   if (spec->residual == TQ_RESIDUAL_SIGN) {
     // per-element residual sign: S = I (m = d), every row's stored residual
     // scale is the constant mu sqrt(2d/pi), so that the estimator's
@@ -404,7 +451,8 @@ extern "C" tq_status tq_codec_create(const tq_spec* spec, int device, tq_codec**
     const size_t o1n = align256(oM + sizeof(uint32_t) * d);
     const size_t o2n = align256(o1n + sizeof(float) * m);
     const size_t oE = align256(o2n + sizeof(float) * m);
-    const size_t total = align256(oE + 16);
+    const size_t oH = align256(oE + 16);  // Haar: Pi^T [d][d] fp32 (element (i, j) = Pi_ji)
+    const size_t total = align256(oH + (p.haar ? sizeof(float) * (size_t)d * d : 0));
     e = cudaMalloc(&c->dev_block, total);
     if (e != cudaSuccess) {
       delete c;
@@ -425,11 +473,18 @@ extern "C" tq_status tq_codec_create(const tq_spec* spec, int device, tq_codec**
       if (e == cudaSuccess) e = cudaMemcpy(base + o1n, l1n.data(), sizeof(float) * m, cudaMemcpyHostToDevice);
       if (e == cudaSuccess) e = cudaMemcpy(base + o2n, l2n.data(), sizeof(float) * m, cudaMemcpyHostToDevice);
     }
+    if (e == cudaSuccess && p.haar) {
+      std::vector<float> PiT((size_t)d * d);
+      for (int j = 0; j < d; ++j)
+        for (int i = 0; i < d; ++i) PiT[(size_t)i * d + j] = (float)c->haar[(size_t)j * d + i];
+      e = cudaMemcpy(base + oH, PiT.data(), sizeof(float) * PiT.size(), cudaMemcpyHostToDevice);
+    }
     if (e != cudaSuccess) {
       cudaFree(c->dev_block);
       delete c;
       return cuda_fail(e, "codec upload");
     }
+    if (p.haar) p.piT = (const float*)(base + oH);
     p.S = (const float*)(base + oS);
     p.St = (const float*)(base + oSt);
     p.s_l1 = (const float*)(base + o1);
@@ -469,6 +524,29 @@ extern "C" tq_status tq_codec_export(const tq_codec* c, float* S, uint32_t* dsig
     if (cen) cen = std::copy(c->cen_host[s].begin(), c->cen_host[s].end(), cen);
     if (bnd) bnd = std::copy(c->bnd_host[s].begin(), c->bnd_host[s].end(), bnd);
   }
+  return TQ_OK;
+}
+
+extern "C" tq_status tq_codec_rotation(const tq_codec* c, float* Pi) {
+  if (!c || !Pi) return tq_fail(TQ_ERR_INVALID_ARG, "tq_codec_rotation: null argument");
+  const int d = c->p.d;
+  if (c->p.haar) {
+    for (size_t k = 0; k < (size_t)d * d; ++k) Pi[k] = (float)c->haar[k];
+    return TQ_OK;
+  }
+  // randomized Hadamard: Pi_ji = H_p[j % p][i % p] D_i / sqrt(p) inside the blocks
+  const int hp = c->p.hblock;
+  const double sc = 1.0 / std::sqrt((double)hp);
+  for (int j = 0; j < d; ++j)
+    for (int i = 0; i < d; ++i) {
+      double v = 0.0;
+      if (j / hp == i / hp) {
+        const int par = __builtin_popcount((unsigned)((j % hp) & (i % hp))) & 1;
+        const bool neg = (c->dbits_host[i / 32] >> (i % 32)) & 1u;
+        v = ((par != 0) != neg ? -1.0 : 1.0) * sc;
+      }
+      Pi[(size_t)j * d + i] = (float)v;
+    }
   return TQ_OK;
 }
 

@@ -52,6 +52,11 @@ struct tq_params {
   const int32_t* rope_pos;
   int rope_max_pos;
   int rope_pos_fixed;
+  // dense Haar rotation (TQ_ROTATION_HAAR): Pi^T [d][d] fp32, element (i, j)
+  // = Pi_ji, so that lanes reading consecutive j at fixed i are coalesced; the
+  // codec's D signs are all +1
+  int haar;
+  const float* piT;
   // per-element residual sign (TQ_RESIDUAL_SIGN): rnorms hold this constant
   // instead of ||r|| (0 with the QJL sketch)
   float rnorm_const;
@@ -84,6 +89,7 @@ struct tq_codec {
   std::vector<float> cen_host[2];
   std::vector<float> bnd_host[2];
   double mu = 0.0;  // TQ_RESIDUAL_SIGN: mean residual magnitude (z units)
+  std::vector<double> haar;  // TQ_ROTATION_HAAR: Pi [d][d] row-major, fp64
   // device allocations (one block)
   void* dev_block = nullptr;
 };

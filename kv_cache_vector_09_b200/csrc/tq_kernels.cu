@@ -80,13 +80,27 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
       const float v = xv[k] * inv;
       z[k] = tq_dneg(p.dbits, k, lane) ? -v : v;
     }
-    tq_fwht_warp<VPL>(z, lane);
-    if (p.zscale != 1.0f) {
-#pragma unroll
-      for (int k = 0; k < VPL; ++k) z[k] *= p.zscale;
-    }
     const float l1u = l1 * inv * 1.001f;  // >= ||u||_1 despite fp32 rounding of the sum
-    const float ez0 = kUlp * (float)(p.log2_hblock + 2) * l1u * p.zscale;
+    // rotation error bound of z in units of u = 2^-24: the FWHT sums every
+    // input once per stage, so each stage adds at most ||u||_1 (L stages);
+    // the dense Haar product is a d-term FMA chain per output, at most
+    // (d + 2) u sum_i |Pi_ji u_i| <= (d + 2) u ||u||_2, times sqrt(d) for z
+    float rot_term;
+    if (p.haar) {
+      tq_dense_rotate_warp<VPL>(z, lane, p.piT, rbuf_f);
+      const float sd = sqrtf((float)d);
+#pragma unroll
+      for (int k = 0; k < VPL; ++k) z[k] *= sd;
+      rot_term = (float)(d + 2) * sd * 1.001f;
+    } else {
+      tq_fwht_warp<VPL>(z, lane);
+      if (p.zscale != 1.0f) {
+#pragma unroll
+        for (int k = 0; k < VPL; ++k) z[k] *= p.zscale;
+      }
+      rot_term = (float)(p.log2_hblock + 2) * l1u * p.zscale;
+    }
+    const float ez0 = kUlp * rot_term;
     int code[VPL];
     bool flag = false;
     float zmax = 0.f;
@@ -121,8 +135,7 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
 #pragma unroll
       for (int k = 0; k < VPL; ++k) rbuf_f[lane + 32 * k] = r[k];
       __syncwarp();
-      const float er =
-          1.01f * kUlp * ((float)(p.log2_hblock + 2) * l1u * p.zscale + 4.f * zmax + 2.f * p.cmax) * p.inv_sqrt_d;
+      const float er = 1.01f * kUlp * (rot_term + 4.f * zmax + 2.f * p.cmax) * p.inv_sqrt_d;
       for (int q = 0; q < Q; ++q) {
         const int col = lane * Q + q;
         const float* sc = p.St + col;
@@ -145,11 +158,18 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
         const double v = (double)xv[k] * invd;
         zd[k] = tq_dneg(p.dbits, k, lane) ? -v : v;
       }
-      tq_fwht_warp<VPL>(zd, lane);
-      if (p.hblock != d) {
-        const double zs = sqrt((double)d / (double)p.hblock);
+      if (p.haar) {
+        tq_dense_rotate_warp<VPL>(zd, lane, p.piT, rbuf);
+        const double sd = sqrt((double)d);
 #pragma unroll
-        for (int k = 0; k < VPL; ++k) zd[k] *= zs;
+        for (int k = 0; k < VPL; ++k) zd[k] *= sd;
+      } else {
+        tq_fwht_warp<VPL>(zd, lane);
+        if (p.hblock != d) {
+          const double zs = sqrt((double)d / (double)p.hblock);
+#pragma unroll
+          for (int k = 0; k < VPL; ++k) zd[k] *= zs;
+        }
       }
       const double isd = 1.0 / sqrt((double)d);
       double g2d = 0.0;
@@ -228,10 +248,15 @@ __global__ void __launch_bounds__(256)
       const float a = tq_to_f32(q[(size_t)row * d + lane + 32 * k]);
       v[k] = tq_dneg(p.dbits, k, lane) ? -a : a;
     }
-    tq_fwht_warp<VPL>(v, lane);
+    if (p.haar) {
+      tq_dense_rotate_warp<VPL>(v, lane, p.piT, buf);
+    } else {
+      tq_fwht_warp<VPL>(v, lane);
+#pragma unroll
+      for (int k = 0; k < VPL; ++k) v[k] *= p.inv_sqrt_p;
+    }
 #pragma unroll
     for (int k = 0; k < VPL; ++k) {
-      v[k] *= p.inv_sqrt_p;
       o[lane + 32 * k] = v[k];
       buf[lane + 32 * k] = v[k];
     }
@@ -528,6 +553,23 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
       for (int k = 0; k < VPL; ++k) acc[k] = fmaf(__ldg(Sj + lane + 32 * k), aj, acc[k]);
     }
+  }
+  if (vp.haar) {
+    // out_i = sum_j Pi_ji acc_j, acc_j broadcast from its lane
+    float o[VPL];
+#pragma unroll
+    for (int k = 0; k < VPL; ++k) o[k] = 0.f;
+    for (int j = 0; j < d; ++j) {
+      float aj = 0.f;
+#pragma unroll
+      for (int k = 0; k < VPL; ++k)
+        if (k == (j >> 5)) aj = __shfl_sync(TQ_FULL_MASK, acc[k], j & 31);
+#pragma unroll
+      for (int k = 0; k < VPL; ++k) o[k] = fmaf(__ldg(vp.piT + (size_t)(lane + 32 * k) * d + j), aj, o[k]);
+    }
+#pragma unroll
+    for (int k = 0; k < VPL; ++k) out[(size_t)bh * d + lane + 32 * k] = o[k];
+    return;
   }
   tq_fwht_warp<VPL>(acc, lane);
 #pragma unroll

@@ -67,11 +67,12 @@ __all__ = [
     "fd_density", "fd_normaliser", "gaussian_density", "lloyd_max", "published_codebook",
     "Compressed", "quantize", "quantize_with", "pack_codes", "unpack_codes", "pack_bits", "unpack_bits",
     "estimate_scores", "attend", "dequantize", "search_topk", "exact_topk", "topk_rows", "hadamard_block",
-    "rope_rotate_half", "residual_mean_magnitude",
+    "rope_rotate_half", "residual_mean_magnitude", "haar_rotation", "HAAR_SEED_XOR",
 ]
 
 MASK64 = (1 << 64) - 1
 S_SEED_XOR = 0x5851F42D4C957F2D
+HAAR_SEED_XOR = 0x2545F4914F6CDD1D
 HADAMARD_BLOCK = 512          # largest Hadamard block; longer vectors use blocks
 
 
@@ -129,6 +130,23 @@ def hadamard_block(d: int) -> int:
     if d % HADAMARD_BLOCK == 0:
         return HADAMARD_BLOCK
     raise ValueError(f"unsupported dimension {d}")
+
+
+def haar_rotation(seed: int, d: int) -> np.ndarray:
+    """Dense Haar-distributed orthogonal Pi (FibQuant page, section 1: a shared
+    random orthogonal rotation, Haar): G is d x d iid N(0, 1), drawn like S
+    (Box-Muller cosine branch on output pairs of splitmix64 from
+    seed ^ HAAR_SEED_XOR, row-major, in double), and Pi is the Q of G = QR with
+    the signs fixed so that diag(R) > 0 (the unique such Q, Haar-distributed
+    when G is Gaussian)."""
+    outs = splitmix64(seed ^ HAAR_SEED_XOR, 2 * d * d)
+    g = np.empty(d * d)
+    for k in range(d * d):
+        u1 = ((outs[2 * k] >> 11) + 1) * 2.0 ** -53
+        u2 = (outs[2 * k + 1] >> 11) * 2.0 ** -53
+        g[k] = math.sqrt(-2.0 * math.log(u1)) * math.cos(2.0 * math.pi * u2)
+    Q, R = np.linalg.qr(g.reshape(d, d))
+    return Q * np.sign(np.diag(R))[None, :]
 
 
 def rotation_matrix(D: np.ndarray) -> np.ndarray:
@@ -261,6 +279,9 @@ class Codec:
     # per coordinate and the constant mean magnitude mu; then S = I, m = d)
     residual: str = "qjl"
     mu: float = 0.0
+    # rotation: "rht" (randomized Hadamard from D) or "haar" (dense, D = 1)
+    rotation: str = "rht"
+    haar: Optional[np.ndarray] = None
 
     @property
     def nseg(self) -> int:
@@ -281,7 +302,7 @@ class Codec:
 
     @functools.cached_property
     def Pi(self) -> np.ndarray:
-        return rotation_matrix(self.D)
+        return self.haar if self.rotation == "haar" else rotation_matrix(self.D)
 
     def coord_cen(self, codes: np.ndarray) -> np.ndarray:
         """Centroid (z units) of every coordinate's code; codes (..., d)."""
@@ -293,12 +314,18 @@ class Codec:
 
 
 def make_codec(d: int, seg_bits: Sequence[int], m: int, seed: int,
-               D: Optional[np.ndarray] = None, S: Optional[np.ndarray] = None, residual: str = "qjl") -> Codec:
+               D: Optional[np.ndarray] = None, S: Optional[np.ndarray] = None, residual: str = "qjl",
+               rotation: str = "rht") -> Codec:
     """Codec from the seed (or from explicit D and S, for Monte-Carlo tests).
     residual="sign" is TurboESM's per-element residual sign: one segment,
-    m = d, S = I, and mu from the codebook."""
+    m = d, S = I, and mu from the codebook.  rotation="haar" takes the dense
+    Haar rotation of the seed (D = 1)."""
     seg_bits = tuple(int(b) for b in seg_bits)
-    if D is None:
+    haar = None
+    if rotation == "haar":
+        D = np.ones(d)
+        haar = haar_rotation(seed, d)
+    elif D is None:
         D = rademacher_signs(seed, d)
     cen, bnd = [], []
     for b in seg_bits:
@@ -313,7 +340,8 @@ def make_codec(d: int, seg_bits: Sequence[int], m: int, seed: int,
         mu = residual_mean_magnitude(cen[0], bnd[0], d)
     elif S is None:
         S = gaussian_sketch(seed, m, d) if m > 0 else np.zeros((0, d), dtype=np.float32)
-    return Codec(d, seg_bits, m, seed, np.asarray(D, dtype=np.float64), np.asarray(S), cen, bnd, residual, mu)
+    return Codec(d, seg_bits, m, seed, np.asarray(D, dtype=np.float64), np.asarray(S), cen, bnd, residual, mu,
+                 rotation, haar)
 
 
 # ---------------------------------------------------------------------- bit packing

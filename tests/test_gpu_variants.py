@@ -85,3 +85,52 @@ def test_sign_residual_values_in_attend():
     oo = O.attend(q.to(torch.float64).numpy(), Ko, Vo, okc, ovc, B, Hq, Hkv, T)
     err = attend_errors(out.cpu().numpy().astype(np.float64), oo)
     assert err.max() <= ATTEND_RTOL, err.max()
+
+
+# ------------------------------------------------------------ Haar rotation
+# FibQuant page, section 1, step 2: a shared random orthogonal rotation,
+# Haar.  The library applies the fp32 rounding of the dense Pi; the oracle its
+# fp64 Pi from numpy's QR, so z differs by at most sqrt(d) 2^-24: only codes
+# and signs within 1e-6 of a decision (ties, counted) may differ.
+HAAR = 1
+
+
+@pytest.mark.parametrize("d,bits,m", [(128, 3, 128), (64, 2, 64)])
+def test_haar_quantize_scores_attend(d, bits, m):
+    B, Hq, Hkv, T = 1, 8, 2, 1200
+    kc = tq.Codec(d, (bits,), m, 9, rotation=HAAR)
+    vc = tq.Codec(d, (4,), 0, 10, rotation=HAAR)
+    okc = O.make_codec(d, (bits,), m, 9, rotation="haar")
+    ovc = O.make_codec(d, (4,), 0, 10, rotation="haar")
+    k = synth.heavy_rows(61, B * Hkv * T, d, n_out=2)
+    v = synth.heavy_rows(62, B * Hkv * T, d, n_out=2)
+    q = synth.gaussian_rows(63, B * Hq, d, dtype=torch.bfloat16).reshape(B, Hq, d) * 2.0
+    K, V = tq.Compressed.empty(kc, B * Hkv * T), tq.Compressed.empty(vc, B * Hkv * T)
+    tq.tq_quantize(kc, k.to(DEV), K)
+    tq.tq_quantize(vc, v.to(DEV), V)
+    torch.cuda.synchronize()
+    assert tq.tq_codec_device_error(kc) == 0 and tq.tq_codec_device_error(vc) == 0
+    Ko = O.quantize(k.to(torch.float64).numpy(), okc)
+    Vo = O.quantize(v.to(torch.float64).numpy(), ovc)
+    print("haar K", compare_compressed(K, Ko, okc), "V", compare_compressed(V, Vo, ovc))
+    qg = q.to(DEV).contiguous()
+    # scores on the oracle's compressed keys
+    ws = tq.workspace(tq.tq_scores_workspace_size(kc, B, Hq, Hkv), DEV)
+    logits = torch.empty((B, Hq, T), device=DEV)
+    tq.tq_scores(kc, qg, B, Hq, Hkv, T, _up(Ko, m), logits, ws)
+    torch.cuda.synchronize()
+    lo = O.estimate_scores(q.to(torch.float64).numpy(), Ko, okc, B, Hq, Hkv, T)
+    nu = Ko.nu64.reshape(B, Hkv, 1, T).repeat(Hq // Hkv, axis=2).reshape(B, Hq, T)
+    qn = np.linalg.norm(q.to(torch.float64).numpy(), axis=-1)[:, :, None]
+    err = logit_errors(logits.cpu().numpy().astype(np.float64), lo, nu, qn, d)
+    assert err.max() <= LOGIT_RTOL, err.max()
+    # attention (inverse rotation of the output by Pi^T)
+    out = torch.empty((B, Hq, d), device=DEV)
+    wsa = tq.workspace(tq.tq_attend_workspace_size(kc, vc, B, Hq, Hkv, T), DEV)
+    g = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int32)).to(DEV)
+    Vg = tq.Compressed(g(Vo.codes), None, torch.from_numpy(Vo.norms).to(DEV), None)
+    tq.tq_attend(kc, vc, qg, B, Hq, Hkv, T, _up(Ko, m), Vg, out, wsa)
+    torch.cuda.synchronize()
+    oo = O.attend(q.to(torch.float64).numpy(), Ko, Vo, okc, ovc, B, Hq, Hkv, T)
+    err = attend_errors(out.cpu().numpy().astype(np.float64), oo)
+    assert err.max() <= ATTEND_RTOL, err.max()

@@ -165,3 +165,17 @@ def test_sign_residual_codec_checks_and_tables():
     c = tq.Codec(128, (3,), 128, 0, device=-1, residual=tq.TQ_RESIDUAL_SIGN)
     S, _, _, _ = c.export()
     assert np.array_equal(S, np.eye(128, dtype=np.float32))
+
+
+def test_haar_rotation_matches_the_oracle():
+    # independent draws and factorisations (fp64 Gram-Schmidt in the library,
+    # numpy QR in the oracle) of the same Haar rotation
+    for d, seed in ((64, 5), (128, 1)):
+        c = tq.Codec(d, (3,), 0, seed, device=-1, rotation=tq.TQ_ROTATION_HAAR)
+        Pi = c.rotation_matrix().astype(np.float64)
+        assert np.abs(Pi - O.haar_rotation(seed, d)).max() < 1e-6
+    # the Hadamard codec's dense form equals the oracle's
+    c = tq.Codec(128, (3,), 0, 7, device=-1)
+    assert np.abs(c.rotation_matrix() - O.rotation_matrix(O.rademacher_signs(7, 128))).max() < 1e-7
+    with pytest.raises(tq.TQError):
+        tq.Codec(512, (3,), 0, 0, device=-1, rotation=tq.TQ_ROTATION_HAAR)

@@ -619,6 +619,48 @@ def test_sign_residual_estimator_and_format():
     assert np.mean(err ** 2) < np.mean(err0 ** 2)
 
 
+def test_haar_rotation_is_orthogonal_and_haar():
+    # orthogonal to rounding; and Haar: for Pi uniform on O(d) the first column
+    # is uniform on the sphere, so sqrt(d) Pi_00 follows f_d (KS over seeds),
+    # and distinct entries are uncorrelated
+    d = 16
+    Pi = O.haar_rotation(3, 64)
+    assert np.abs(Pi @ Pi.T - np.eye(64)).max() < 1e-12
+    vals, prods = [], []
+    for sd in range(300):
+        P = O.haar_rotation(sd, d)
+        vals.append(math.sqrt(d) * P[0, 0])
+        prods.append(P[0, 0] * P[1, 1])
+    f, edge = O.fd_density(d)
+    from scipy import integrate
+    cdf = lambda z: integrate.quad(f, -edge, z)[0]
+    ks = stats.kstest(vals, np.vectorize(cdf))
+    assert ks.pvalue > 1e-3, ks
+    assert abs(np.mean(prods)) < 4 * np.std(prods) / math.sqrt(len(prods))
+    # the QR convention: the codec's Pi maps G to an upper-triangular R with
+    # a positive diagonal, i.e. Pi^T G = R
+    outs = O.splitmix64(3 ^ O.HAAR_SEED_XOR, 2 * 64 * 64)
+    G = np.array([math.sqrt(-2 * math.log(((outs[2 * k] >> 11) + 1) * 2.0 ** -53))
+                  * math.cos(2 * math.pi * (outs[2 * k + 1] >> 11) * 2.0 ** -53) for k in range(64 * 64)]).reshape(64, 64)
+    R = Pi.T @ G
+    assert np.abs(np.tril(R, -1)).max() < 1e-10 and np.all(np.diag(R) > 0)
+
+
+def test_haar_codec_quantizes_in_its_rotation():
+    # with a Haar codec, the codes are those of z = sqrt(d) Pi x / ||x|| and
+    # the estimator keeps inner products (QJL Monte Carlo at one S draw is in
+    # the generic tests; here: exact reconstruction of an on-grid vector)
+    d = 64
+    c = O.make_codec(d, (3,), 0, 5, rotation="haar")
+    rng = np.random.default_rng(2)
+    codes = np.searchsorted(c.bnd[0], rng.standard_normal(d), side="right")
+    chat = c.cen[0].astype(np.float64)[codes]
+    x = 1.5 * (chat / np.linalg.norm(chat)) @ c.haar          # Pi^T y as a row
+    comp = O.quantize(x[None], c)
+    assert np.array_equal(comp.code_idx[0], codes)
+    assert np.allclose(O.dequantize(comp, c)[0], 1.5 * (chat / math.sqrt(d)) @ c.haar, atol=1e-12)
+
+
 # ----------------------------------------------------------------------- top-k
 def test_topk_order_and_ties():
     sc = np.array([[0.5, 2.0, 2.0, -1.0, 2.0, 0.7]])
