@@ -26,6 +26,16 @@ source pages):
   ``rope_rotate_half`` is that RoPE (rotate-half pairs (i, i + d/2), angle
   pos * theta^(-2i/d)); the encoder of RoPE'd keys is ``quantize`` of its
   output.
+* "FibQuant ...", section 2.2 (codebook) and 2.3 (encoder): with k = 2 the
+  rotated unit vector is cut into d/2 blocks of two consecutive coordinates and
+  every block takes the nearest of N = 2^vq_bits shared codewords (vq_bits / 2
+  bits per coordinate).  The codebook (``fibquant_codebook``) starts from a
+  planar Fibonacci spiral with Bennett-Gersho radii and is refined by Lloyd's
+  algorithm with several restarts.  Readings: codewords live in z units (the
+  page's unit-ball source scaled by sqrt(d)); the expectation Lloyd needs is
+  taken over a deterministic quasi-Monte-Carlo point set of the block law
+  (``fibquant_source_points``); 40 iterations, 3 restarts turned by a fraction
+  of the golden angle, the least-distortion restart kept; codewords in fp32.
 * The estimator of <q, x> that the library evaluates is
   nu * ( <Pi q, c_hat> / sqrt(d) + ||r|| * sqrt(pi/2) / m * <S Pi q, sign(S r)> ).
 
@@ -68,6 +78,7 @@ __all__ = [
     "Compressed", "quantize", "quantize_with", "pack_codes", "unpack_codes", "pack_bits", "unpack_bits",
     "estimate_scores", "attend", "dequantize", "search_topk", "exact_topk", "topk_rows", "hadamard_block",
     "rope_rotate_half", "residual_mean_magnitude", "haar_rotation", "HAAR_SEED_XOR",
+    "fibquant_init", "fibquant_source_points", "fibquant_codebook", "fibquant_distortion",
 ]
 
 MASK64 = (1 << 64) - 1
@@ -250,6 +261,75 @@ def published_codebook(bits: int, d: int) -> Tuple[np.ndarray, np.ndarray]:
     return cen.astype(np.float32), bnd
 
 
+# ------------------------------------------------------------ FibQuant, k = 2
+GOLDEN_ANGLE = math.pi * (3.0 - math.sqrt(5.0))   # 2 pi (1 - 1/phi)
+
+
+def fibquant_init(N: int, d: int, offset: float = 0.0) -> np.ndarray:
+    """Initial k = 2 codebook of the FibQuant page (section 2.2), in z units
+    (z = sqrt(d) times the rotated unit vector): N points on a planar Fibonacci
+    spiral, point n at angle n * golden_angle + offset and at the radius whose
+    Bennett-Gersho point density (proportional to f^(k/(k+2)) = f^(1/2) of the
+    source density f_{d,2}(z) ~ (1 - |z|^2/d)^((d-4)/2)) leaves a fraction
+    (n + 1/2)/N of the points inside: Lambda(r) = 1 - (1 - r^2/d)^(d/4), so
+        r_n^2 = d (1 - (1 - (n + 1/2)/N)^(4/d))."""
+    n = np.arange(N, dtype=np.float64)
+    r = np.sqrt(d * (1.0 - np.power(1.0 - (n + 0.5) / N, 4.0 / d)))
+    a = n * GOLDEN_ANGLE + offset
+    return np.stack([r * np.cos(a), r * np.sin(a)], axis=1)
+
+
+def fibquant_source_points(d: int, M: int) -> np.ndarray:
+    """A deterministic quasi-Monte-Carlo stand-in for the source f_{d,2}: M
+    equally weighted points, point i at the radius whose radial CDF is
+    (i + 1/2)/M (for u uniform on S^{d-1}, u_1^2 + u_2^2 ~ Beta(1, (d-2)/2),
+    CDF 1 - (1 - t)^((d-2)/2), so |z|^2 = d (1 - (1 - (i + 1/2)/M)^(2/(d-2))))
+    and at angle i * golden_angle."""
+    i = np.arange(M, dtype=np.float64)
+    r = np.sqrt(d * (1.0 - np.power(1.0 - (i + 0.5) / M, 2.0 / (d - 2))))
+    a = i * GOLDEN_ANGLE
+    return np.stack([r * np.cos(a), r * np.sin(a)], axis=1)
+
+
+def _nearest(points: np.ndarray, cb: np.ndarray) -> np.ndarray:
+    d2 = ((points[:, None, :] - cb[None, :, :]) ** 2).sum(axis=2)
+    return np.argmin(d2, axis=1)                     # ties -> lower index
+
+
+def fibquant_distortion(points: np.ndarray, cb: np.ndarray) -> float:
+    """Mean squared error per 2-block of the nearest-codeword quantiser."""
+    idx = _nearest(points, cb)
+    return float(np.mean(((points - cb[idx]) ** 2).sum(axis=1)))
+
+
+@functools.lru_cache(maxsize=None)
+def fibquant_codebook(vq_bits: int, d: int, M: int = 16384, iters: int = 40, restarts: int = 3) -> np.ndarray:
+    """FibQuant k = 2 codebook (page section 2.2): the Fibonacci-spiral
+    initialisation refined by Lloyd's algorithm (nearest-codeword cells, then
+    every codeword moved to the mean of its cell) on the quasi-Monte-Carlo
+    source points, from `restarts` initial spirals turned by r * golden_angle /
+    restarts; the restart with the least distortion is kept (ties: the
+    first).  Returned in fp32, [N][2], z units."""
+    pts = fibquant_source_points(d, M)
+    N = 1 << vq_bits
+    best, best_d = None, math.inf
+    for rs in range(restarts):
+        cb = fibquant_init(N, d, rs * GOLDEN_ANGLE / restarts)
+        for _ in range(iters):
+            idx = _nearest(pts, cb)
+            cnt = np.bincount(idx, minlength=N)
+            sx = np.bincount(idx, weights=pts[:, 0], minlength=N)
+            sy = np.bincount(idx, weights=pts[:, 1], minlength=N)
+            keep = cnt > 0
+            cb = cb.copy()
+            cb[keep, 0] = sx[keep] / cnt[keep]
+            cb[keep, 1] = sy[keep] / cnt[keep]
+        dist = fibquant_distortion(pts, cb)
+        if dist < best_d:
+            best, best_d = cb, dist
+    return best.astype(np.float32)
+
+
 # -------------------------------------------------------------------------- codec
 def residual_mean_magnitude(cen: np.ndarray, bnd: np.ndarray, d: int) -> float:
     """mu = E|z - cen[code(z)]| for z with density f_d and the published
@@ -282,6 +362,10 @@ class Codec:
     # rotation: "rht" (randomized Hadamard from D) or "haar" (dense, D = 1)
     rotation: str = "rht"
     haar: Optional[np.ndarray] = None
+    # FibQuant k = 2 (vq_bits > 0): blocks (z_2j, z_2j+1) take the nearest of
+    # the 2^vq_bits codewords of vq_cb [N][2] (fp32, z units); seg_bits unused
+    vq_bits: int = 0
+    vq_cb: Optional[np.ndarray] = None
 
     @property
     def nseg(self) -> int:
@@ -298,6 +382,8 @@ class Codec:
 
     @property
     def words(self) -> int:
+        if self.vq_bits:
+            return self.vq_bits * ((self.d // 2 + 31) // 32)
         return sum(b * self.plane_words for b in self.seg_bits)
 
     @functools.cached_property
@@ -305,7 +391,12 @@ class Codec:
         return self.haar if self.rotation == "haar" else rotation_matrix(self.D)
 
     def coord_cen(self, codes: np.ndarray) -> np.ndarray:
-        """Centroid (z units) of every coordinate's code; codes (..., d)."""
+        """Centroid (z units) of every coordinate's code; codes (..., d).  With
+        FibQuant the code of coordinate i is its block's codeword index and the
+        centroid is that codeword's component i % 2."""
+        if self.vq_bits:
+            cb = self.vq_cb.astype(np.float64)
+            return cb[codes, np.arange(self.d) % 2]
         out = np.empty(codes.shape)
         L = self.seg_len
         for s in range(self.nseg):
@@ -315,7 +406,7 @@ class Codec:
 
 def make_codec(d: int, seg_bits: Sequence[int], m: int, seed: int,
                D: Optional[np.ndarray] = None, S: Optional[np.ndarray] = None, residual: str = "qjl",
-               rotation: str = "rht") -> Codec:
+               rotation: str = "rht", vq_bits: int = 0) -> Codec:
     """Codec from the seed (or from explicit D and S, for Monte-Carlo tests).
     residual="sign" is TurboESM's per-element residual sign: one segment,
     m = d, S = I, and mu from the codebook.  rotation="haar" takes the dense
@@ -340,16 +431,46 @@ def make_codec(d: int, seg_bits: Sequence[int], m: int, seed: int,
         mu = residual_mean_magnitude(cen[0], bnd[0], d)
     elif S is None:
         S = gaussian_sketch(seed, m, d) if m > 0 else np.zeros((0, d), dtype=np.float32)
+    vq_cb = fibquant_codebook(vq_bits, d) if vq_bits else None
     return Codec(d, seg_bits, m, seed, np.asarray(D, dtype=np.float64), np.asarray(S), cen, bnd, residual, mu,
-                 rotation, haar)
+                 rotation, haar, vq_bits, vq_cb)
 
 
 # ---------------------------------------------------------------------- bit packing
+def _pack_vq(codes: np.ndarray, codec: Codec) -> np.ndarray:
+    """FibQuant codes: plane p (p = 0..vq_bits-1), word w holds bit p of the
+    codes of blocks 32w..32w+31, block 32w+t at bit t; codes holds each
+    block's index on both of its coordinates."""
+    n, nb = codes.shape[0], codec.d // 2
+    pw = (nb + 31) // 32
+    blk = codes[:, 0::2].astype(np.uint64)
+    out = np.zeros((n, codec.vq_bits * pw), dtype=np.uint64)
+    for p in range(codec.vq_bits):
+        for w in range(pw):
+            for t in range(min(32, nb - 32 * w)):
+                out[:, p * pw + w] |= ((blk[:, 32 * w + t] >> np.uint64(p)) & np.uint64(1)) << np.uint64(t)
+    return out.astype(np.uint32)
+
+
+def _unpack_vq(words: np.ndarray, codec: Codec) -> np.ndarray:
+    n, nb = words.shape[0], codec.d // 2
+    pw = (nb + 31) // 32
+    w64 = words.astype(np.uint64)
+    blk = np.zeros((n, nb), dtype=np.int64)
+    for p in range(codec.vq_bits):
+        for w in range(pw):
+            for t in range(min(32, nb - 32 * w)):
+                blk[:, 32 * w + t] |= ((w64[:, p * pw + w] >> np.uint64(t)) & np.uint64(1)).astype(np.int64) << p
+    return np.repeat(blk, 2, axis=1)
+
+
 def pack_codes(codes: np.ndarray, codec: Codec) -> np.ndarray:
     """Planar packing: segments in order; inside a segment of b bits, plane p
     (p = 0..b-1) holds bit p of each code; word w of a plane holds the codes of
     coordinates 32w..32w+31 of the segment, coordinate 32w+t at bit t (bits
     past the end of a segment shorter than a whole word are zero)."""
+    if codec.vq_bits:
+        return _pack_vq(codes, codec)
     n = codes.shape[0]
     L = codec.seg_len
     out = np.zeros((n, codec.words), dtype=np.uint64)
@@ -367,6 +488,8 @@ def pack_codes(codes: np.ndarray, codec: Codec) -> np.ndarray:
 
 
 def unpack_codes(words: np.ndarray, codec: Codec) -> np.ndarray:
+    if codec.vq_bits:
+        return _unpack_vq(words, codec)
     n = words.shape[0]
     L = codec.seg_len
     w64 = words.astype(np.uint64)
@@ -430,7 +553,24 @@ def quantize_with(z: np.ndarray, y: np.ndarray, nu: np.ndarray, codec: Codec) ->
     L = codec.seg_len
     codes = np.empty(z.shape, dtype=np.int64)
     margin = np.empty(z.shape)
-    for s in range(codec.nseg):
+    if codec.vq_bits:
+        # FibQuant section 2.3: each block (z_2j, z_2j+1) takes its nearest
+        # codeword (ties: the lower index); the margin is the block's distance
+        # to its Voronoi cell's boundary, the least over the other codewords c_j
+        # of the distance to the bisector of c_i1 and c_j,
+        # (|z - c_j|^2 - |z - c_i1|^2) / (2 |c_j - c_i1|)
+        cb = codec.vq_cb.astype(np.float64)
+        blocks = z.reshape(z.shape[0], d // 2, 2)
+        d2 = ((blocks[:, :, None, :] - cb[None, None, :, :]) ** 2).sum(axis=3)
+        i1 = np.argmin(d2, axis=2)
+        d1 = np.take_along_axis(d2, i1[:, :, None], 2)
+        sep = np.sqrt(((cb[:, None, :] - cb[None, :, :]) ** 2).sum(axis=2))[i1]
+        with np.errstate(divide="ignore", invalid="ignore"):
+            bis = np.where(sep > 0, (d2 - d1) / (2.0 * sep), np.inf)
+        bis[np.arange(bis.shape[2])[None, None, :] == i1[:, :, None]] = np.inf
+        codes[:] = np.repeat(i1, 2, axis=1)
+        margin[:] = np.repeat(np.min(bis, axis=2), 2, axis=1)
+    for s in range(codec.nseg if not codec.vq_bits else 0):
         zs = z[:, s * L:(s + 1) * L]
         bnd = codec.bnd[s].astype(np.float64)
         codes[:, s * L:(s + 1) * L] = np.sum(zs[:, :, None] >= bnd[None, None, :], axis=2)

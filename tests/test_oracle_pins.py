@@ -726,3 +726,176 @@ def test_search_scores_are_the_estimator(m):
     # a smaller k is the prefix of the full order
     idx3, score3 = O.search_topk(q, comp, codec, 3)
     assert np.array_equal(idx3, idx[:, :3] - 5) and np.array_equal(score3, score[:, :3])
+
+
+# ------------------------------------------------------------- FibQuant, k = 2
+def _block_radius_cdf(d):
+    """CDF of |(z_1, z_2)|^2 for z = sqrt(d) u, u uniform on S^{d-1}, by
+    quadrature of the 2-D marginal (1 - rho^2/d)^((d-4)/2) times the ring
+    length 2 pi rho (normalised numerically, not by a closed form)."""
+    from scipy import integrate
+    g = lambda rho: rho * (1.0 - rho * rho / d) ** ((d - 4) / 2.0)
+    tot = integrate.quad(g, 0.0, math.sqrt(d), epsrel=1e-12)[0]
+    return lambda s: integrate.quad(g, 0.0, math.sqrt(min(max(s, 0.0), d)), epsrel=1e-12)[0] / tot
+
+
+@pytest.mark.parametrize("d", [16, 128])
+def test_fibquant_source_points_follow_the_block_law(d):
+    # the quasi-Monte-Carlo stand-in for the block source: its squared radii
+    # match sampled blocks of uniform unit vectors (two-sample KS) and the
+    # quadrature CDF of the 2-D marginal, and its moments are E|z|^2 = 2 and
+    # E|z|^4 = 8d / (d + 2) (z_1^2 + z_2^2 = d Beta(1, (d-2)/2))
+    pts = O.fibquant_source_points(d, 16384)
+    r2 = (pts ** 2).sum(axis=1)
+    assert abs(r2.mean() - 2.0) < 1e-3
+    assert abs((r2 ** 2).mean() - 8.0 * d / (d + 2)) < 2e-3 * 8
+    rng = np.random.default_rng(d)
+    g = rng.standard_normal((20000, d))
+    u = g / np.linalg.norm(g, axis=1, keepdims=True)
+    mc = d * (u[:, 0] ** 2 + u[:, 1] ** 2)
+    assert stats.ks_2samp(r2, mc).pvalue > 1e-3
+    cdf = _block_radius_cdf(d)
+    for qv in (0.1, 0.5, 0.9, 0.99):
+        s = float(np.quantile(r2, qv))
+        assert abs(cdf(s) - qv) < 2e-4, (qv, cdf(s))
+    # the angles advance by the golden angle 2 pi (1 - 1/phi)
+    ang = np.arctan2(pts[:, 1], pts[:, 0])
+    step = np.mod(np.diff(ang), 2 * math.pi)
+    phi = (1 + math.sqrt(5)) / 2
+    assert np.allclose(step, 2 * math.pi * (1 - 1 / phi), atol=1e-9)
+
+
+@pytest.mark.parametrize("d,N", [(64, 16), (128, 32)])
+def test_fibquant_spiral_radii_are_bennett_gersho(d, N):
+    # section 2.2: the point density of the initial spiral follows f^(k/(k+2))
+    # = f^(1/2) of the block law; the fraction of the N points inside radius
+    # r_n must be the quadrature of that density, (n + 1/2) / N
+    from scipy import integrate
+    lam = lambda rho: rho * (1.0 - rho * rho / d) ** ((d - 4) / 4.0)
+    tot = integrate.quad(lam, 0.0, math.sqrt(d), epsrel=1e-12)[0]
+    cb = O.fibquant_init(N, d)
+    r = np.linalg.norm(cb, axis=1)
+    assert np.all(np.diff(r) > 0)
+    for n in range(N):
+        frac = integrate.quad(lam, 0.0, r[n], epsrel=1e-12)[0] / tot
+        assert abs(frac - (n + 0.5) / N) < 1e-9, (n, frac)
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_fibquant_two_codewords_are_antipodal_scalar_centroids(d):
+    # N = 2 on a rotationally symmetric source: the optimum splits the plane by
+    # a line through 0 and puts each codeword at its half-plane's mean, i.e.
+    # at distance E[z_1 | z_1 > 0] = the 1-bit Lloyd-Max centroid (closed form)
+    cb = O.fibquant_codebook(1, d).astype(np.float64)
+    want = math.sqrt(d) * math.exp(math.lgamma(d / 2) - math.lgamma((d + 1) / 2)) / math.sqrt(math.pi)
+    assert np.allclose(np.linalg.norm(cb, axis=1), want, rtol=3e-3), (np.linalg.norm(cb, axis=1), want)
+    assert np.linalg.norm(cb[0] + cb[1]) < 3e-3
+
+
+def test_fibquant_lloyd_descends_to_a_fixed_point():
+    # Lloyd never increases the distortion, and the result is (nearly) the
+    # mean of its own cells over the source points
+    d, vb = 64, 4
+    pts = O.fibquant_source_points(d, 16384)
+    seq = [O.fibquant_distortion(pts, O.fibquant_codebook.__wrapped__(vb, d, iters=it, restarts=1).astype(np.float64))
+           for it in (0, 1, 2, 5, 10, 40)]
+    assert all(b <= a * (1 + 1e-6) for a, b in zip(seq, seq[1:])), seq
+    assert seq[-1] < 0.97 * seq[0]
+    cb = O.fibquant_codebook(vb, d).astype(np.float64)
+    d2 = ((pts[:, None, :] - cb[None, :, :]) ** 2).sum(axis=2)
+    own = d2.argmin(axis=1)
+    for n in range(len(cb)):
+        cell = pts[own == n]
+        assert len(cell) > 0
+        assert np.linalg.norm(cell.mean(axis=0) - cb[n]) < 0.02, n
+
+
+@pytest.mark.parametrize("b", [2, 3])
+def test_fibquant_beats_scalar_lloyd_max_at_integer_rates(b):
+    # section 3.2 / 4: at matched rate the k = 2 code has strictly lower MSE
+    # than the scalar Lloyd-Max table (integrated exactly under f_d)
+    d = 128
+    f, edge = O.fd_density(d)
+    cen, bnd, _ = O.lloyd_max(b, O.fd_density(d))
+    scalar = _mse(cen, bnd, f, edge)
+    pts = O.fibquant_source_points(d, 16384)
+    vq = O.fibquant_distortion(pts, O.fibquant_codebook(2 * b, d).astype(np.float64)) / 2
+    assert vq < 0.97 * scalar, (vq, scalar)
+    # and the fractional rate b + 1/2 lies between the neighbouring integer rates
+    half = O.fibquant_distortion(pts, O.fibquant_codebook(2 * b + 1, d).astype(np.float64)) / 2
+    assert vq * 0.4 < half < vq * 0.75
+
+
+def test_fibquant_packing_positions():
+    # block 32w + t's code bit p sits at bit t of word p * pw + w
+    d = 64
+    c = O.make_codec(d, (1,), 0, 0, vq_bits=3)
+    blk = np.arange(32) % 8
+    codes = np.repeat(blk, 2)[None]
+    w = O.pack_codes(codes, c)
+    assert w.shape == (1, 3) and c.words == 3
+    assert [int(v) for v in w[0]] == [0xAAAAAAAA, 0xCCCCCCCC, 0xF0F0F0F0]
+    assert np.array_equal(O.unpack_codes(w, c), codes)
+
+
+def test_fibquant_encoder_is_the_nearest_codeword():
+    # brute force on small rows: every block's code is its nearest codeword;
+    # moving the block by 0.999 of its margin in any direction keeps the code,
+    # moving it just past the margin towards the nearest bisector changes it
+    d = 16
+    c = O.make_codec(d, (1,), 0, 0, vq_bits=4)
+    cb = c.vq_cb.astype(np.float64)
+    x = np.random.default_rng(3).standard_t(3, size=(20, d))
+    comp = O.quantize(x, c)
+    rng = np.random.default_rng(4)
+    for i in range(x.shape[0]):
+        for j in range(d // 2):
+            zb = comp.z[i, 2 * j:2 * j + 2]
+            dist = [float(np.sum((zb - cw) ** 2)) for cw in cb]
+            n = comp.code_idx[i, 2 * j]
+            assert comp.code_idx[i, 2 * j + 1] == n and dist[n] == min(dist)
+            mg = comp.code_margin[i, 2 * j]
+            for _ in range(16):
+                a = rng.uniform(0, 2 * math.pi)
+                zp = zb + 0.999 * mg * np.array([math.cos(a), math.sin(a)])
+                assert int(np.argmin(((zp - cb) ** 2).sum(axis=1))) == n
+            # the nearest bisector: step towards each other codeword's cell
+            moved = False
+            for k in range(len(cb)):
+                if k == n:
+                    continue
+                e = (cb[k] - cb[n]) / np.linalg.norm(cb[k] - cb[n])
+                zp = zb + 1.001 * mg * e
+                moved |= int(np.argmin(((zp - cb) ** 2).sum(axis=1))) != n
+            assert moved
+
+
+def test_fibquant_decoder_error_matches_design_distortion():
+    # E ||x - x_hat||^2 / ||x||^2 = (per-block distortion) / 2 per coordinate
+    d = 64
+    c = O.make_codec(d, (1,), 0, 0, vq_bits=5)
+    x = np.random.default_rng(9).standard_t(3, size=(3000, d))
+    comp = O.quantize(x, c)
+    rel = np.sum((x - O.dequantize(comp, c)) ** 2, axis=1) / np.sum(x * x, axis=1)
+    want = O.fibquant_distortion(O.fibquant_source_points(d, 16384), c.vq_cb.astype(np.float64)) / 2
+    assert abs(rel.mean() - want) < 0.05 * want, (rel.mean(), want)
+
+
+def test_fibquant_qjl_estimator_is_unbiased_monte_carlo():
+    # the QJL stage corrects whatever the first stage leaves: over S, the
+    # estimator's mean is <q, x> with the vector codes too
+    d, m, N = 16, 32, 6000
+    rng = np.random.default_rng(31)
+    x = rng.standard_t(3, size=(1, d))
+    q = rng.standard_normal((1, 1, d))
+    c0 = O.make_codec(d, (1,), m, 0, S=np.zeros((m, d)), vq_bits=3)
+    exact = float(q[0, 0] @ x[0])
+    est = np.empty(N)
+    for k in range(N):
+        c = O.make_codec(d, (1,), m, 0, D=c0.D, S=rng.standard_normal((m, d)), vq_bits=3)
+        est[k] = O.estimate_scores(q, O.quantize(x, c), c, 1, 1, 1, 1)[0, 0, 0]
+    se = est.std() / math.sqrt(N)
+    assert abs(est.mean() - exact) < 4 * se + 1e-6 * abs(exact), (est.mean(), exact, se)
+    comp0 = O.quantize(x, c0)
+    mse_only = np.linalg.norm(x) * float((q[0, 0] @ c0.Pi.T) @ c0.coord_cen(comp0.code_idx)[0]) / math.sqrt(d)
+    assert abs(mse_only - exact) > 10 * se
