@@ -88,7 +88,22 @@ typedef enum { TQ_F32 = 0, TQ_BF16 = 1, TQ_F16 = 2 } tq_dtype;
  *              (splitmix64 from seed ^ 0x5851F42D4C957F2D, Box-Muller cosine
  *              branch on output pairs, double, rounded to fp32, row-major m x d)
  *   residual : TQ_RESIDUAL_QJL (0) or TQ_RESIDUAL_SIGN (1), see tq_residual
- *   rotation : TQ_ROTATION_RHT (0) or TQ_ROTATION_HAAR (1), see tq_rotation  */
+ *   rotation : TQ_ROTATION_RHT (0) or TQ_ROTATION_HAAR (1), see tq_rotation
+ *   vq_bits  : 0 = scalar Lloyd-Max codes (seg_bits); 1..8 = FibQuant k = 2
+ *              vector codes (FibQuant page, sections 2.2-2.3): the rotated
+ *              coordinates are cut into d/2 blocks (z_2j, z_2j+1), each block
+ *              stores the index of its nearest codeword among N = 2^vq_bits,
+ *              i.e. vq_bits / 2 bits per coordinate (0.5 .. 4, half steps);
+ *              needs nseg = 1 (seg_bits is then ignored) and TQ_RESIDUAL_QJL.
+ *              The codebook (in z units, fp32, see tq_codec_vq_codebook) is a
+ *              planar Fibonacci spiral, point n at angle n * 2 pi (1 - 1/phi)
+ *              and radius r_n = sqrt(d (1 - (1 - (n + 1/2)/N)^(4/d))) (the
+ *              Bennett-Gersho density f^(1/2) of the block law), refined by
+ *              40 Lloyd iterations over the 16384 quasi-Monte-Carlo points
+ *              i = 0.. of that law (radius sqrt(d (1 - (1 - (i + 1/2)/16384)
+ *              ^(2/(d-2)))), angle i * 2 pi (1 - 1/phi)); three restarts turn
+ *              the spiral by r/3 of the golden angle, the least-distortion one
+ *              is kept.  Code = the nearest codeword (ties: lower index).    */
 typedef struct {
   int32_t d;
   int32_t nseg;
@@ -97,6 +112,7 @@ typedef struct {
   uint64_t seed;
   int32_t residual;   /* tq_residual: form of the 1-bit residual stage */
   int32_t rotation;   /* tq_rotation: the shared random rotation Pi */
+  int32_t vq_bits;    /* 0: scalar codes; 1..8: FibQuant k = 2 block codes */
 } tq_spec;
 
 /* Rotation (tq_spec.rotation).
@@ -134,6 +150,9 @@ typedef enum { TQ_RESIDUAL_QJL = 0, TQ_RESIDUAL_SIGN = 1 } tq_residual;
  *          Planar layout: segments in order; inside segment s, bit planes
  *          p = 0..seg_bits[s]-1; inside a plane, word w holds bit p of the codes
  *          of the segment's coordinates 32w..32w+31, coordinate 32w+t at bit t.
+ *          FibQuant codes (vq_bits > 0): W = vq_bits * d / 64, planes
+ *          p = 0..vq_bits-1 of d/64 words; word w of plane p holds bit p of
+ *          the codeword indices of blocks 32w..32w+31, block 32w+t at bit t.
  *   signs  [n][m/32] uint32, bit j%32 of word j/32 = bit_j; NULL iff m == 0
  *   norms  [n] fp32, nu
  *   rnorms [n] fp32, gamma; NULL iff m == 0                                   */
@@ -178,6 +197,11 @@ TQ_API tq_status tq_codec_destroy(tq_codec *codec);
  *   bnd    [sum_s 2^seg_bits[s] - 1]  per-segment boundaries, concatenated    */
 TQ_API tq_status tq_codec_export(const tq_codec *codec, float *S, uint32_t *dsigns,
                           float *cen, float *bnd);
+
+/* FibQuant codebook of a codec with vq_bits > 0: cb [2^vq_bits][2] fp32, in
+ * z units (codeword n = (cb[n][0], cb[n][1]) reconstructs the block
+ * (z_2j, z_2j+1)).  TQ_ERR_INVALID_ARG for a scalar codec.                  */
+TQ_API tq_status tq_codec_vq_codebook(const tq_codec *codec, float *cb);
 
 /* The codec's rotation as a dense matrix: Pi [d][d] fp32 row-major, y = Pi u
  * (host copy, for checking; the Hadamard rotation is expanded).            */
@@ -232,8 +256,8 @@ TQ_API tq_status tq_rope_cache(double theta, int d, int max_pos, float *cos_sin,
 /* tq_quantize of the RoPE'd rows: row i is rotated by RoPE at position
  * rope->positions[i] before normalisation.  A position outside [0, max_pos)
  * is replaced by 0 and recorded as code 3 in the codec's device error word
- * (tq_codec_device_error).  Requires d = 64 or 128, TQ_BF16 or TQ_F32 rows
- * and m <= 256 (else TQ_ERR_UNSUPPORTED).                                    */
+ * (tq_codec_device_error).  Requires d = 64 or 128, TQ_BF16 or TQ_F32 rows,
+ * m <= 256, scalar codes and the Hadamard rotation (else TQ_ERR_UNSUPPORTED). */
 TQ_API tq_status tq_quantize_rope(const tq_codec *codec, const void *x, tq_dtype dtype,
                                   int64_t n, int64_t ld, const tq_rope *rope,
                                   const tq_compressed *out, void *stream);
@@ -265,7 +289,8 @@ TQ_API tq_status tq_scores_workspace_size(const tq_codec *kc, int B, int Hq,
  *           (b*Hkv + h_kv)*T + t
  *   logits  [B][Hq][T] fp32 out; query head h uses KV head h / (Hq / Hkv)
  *   workspace, ws_bytes  >= tq_scores_workspace_size(kc, B, Hq, Hkv)
- * Hq must be a multiple of Hkv, Hq / Hkv <= 32.  T = 0 is a no-op.          */
+ * Hq must be a multiple of Hkv, Hq / Hkv <= 32.  T = 0 is a no-op.  With
+ * FibQuant codes the first term reads <q'_2j, q'_2j+1> . cb[code_j] per block. */
 TQ_API tq_status tq_scores(const tq_codec *kc, const void *q, tq_dtype dtype, int B,
                     int Hq, int Hkv, int64_t T, const tq_compressed *K,
                     float *logits, void *workspace, size_t ws_bytes,
@@ -307,7 +332,8 @@ TQ_API tq_status tq_attend_workspace_size(const tq_codec *kc, const tq_codec *vc
  * the QJL residual estimate, makes every v~_t unbiased for its value (the
  * TurboQuant pages' unbiasing stage applied to values); with m_v = 0 it is
  * absent.  Shapes as tq_scores; out [B][Hq][d] fp32.  kc and vc must have the
- * same d.  T >= 1.                                                         */
+ * same d.  T >= 1.  FibQuant codes (vq_bits > 0) on either side run on the
+ * CUDA-core kernel, which needs m_v = 0 (else TQ_ERR_UNSUPPORTED).          */
 TQ_API tq_status tq_attend(const tq_codec *kc, const tq_codec *vc, const void *q,
                     tq_dtype dtype, int B, int Hq, int Hkv, int64_t T,
                     float scale, const tq_compressed *K,
@@ -328,7 +354,7 @@ TQ_API tq_status tq_search_workspace_size(const tq_codec *codec, int nq, int k,
  * and idx[i][0..k) / score[i][0..k) (device, int32 / fp32, row-major) receive
  * the k best rows in descending score, ties to the lower row index.  The
  * scores are never stored in full: tensor-core tiles of 128 rows x 256
- * queries feed per-query top-k lists.  Requires one segment (nseg = 1),
+ * queries feed per-query top-k lists.  Requires scalar codes of one segment,
  * d a multiple of 32 with 64 <= d <= 2048, m <= 512, k <= 32, 1 <= k <= n,
  * n < 2^31.  The workspace (device, 256-byte aligned) is sized by
  * tq_search_workspace_size.                                                 */

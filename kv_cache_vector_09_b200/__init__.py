@@ -38,7 +38,7 @@ TQ_ROTATION_RHT, TQ_ROTATION_HAAR = 0, 1
 class tq_spec(ctypes.Structure):
     _fields_ = [("d", ctypes.c_int32), ("nseg", ctypes.c_int32), ("seg_bits", ctypes.c_int32 * 2),
                 ("m", ctypes.c_int32), ("seed", ctypes.c_uint64), ("residual", ctypes.c_int32),
-                ("rotation", ctypes.c_int32)]
+                ("rotation", ctypes.c_int32), ("vq_bits", ctypes.c_int32)]
 
 
 class tq_compressed(ctypes.Structure):
@@ -62,6 +62,7 @@ def _load() -> ctypes.CDLL:
         "tq_codec_export": [P, P, P, P, P],
         "tq_codec_layout": [P, ctypes.POINTER(I), ctypes.POINTER(I)],
         "tq_codec_rotation": [P, P],
+        "tq_codec_vq_codebook": [P, P],
         "tq_quantize": [P, P, I, I64, I64, P, P],
         "tq_rope_cache": [ctypes.c_double, I, I, P, P],
         "tq_quantize_rope": [P, P, I, I64, I64, P, P, P],
@@ -129,12 +130,12 @@ class Codec:
     """A tq_codec handle (freed with the object)."""
 
     def __init__(self, d: int, seg_bits: Sequence[int], m: int, seed: int = 0, device: int = 0,
-                 residual: int = TQ_RESIDUAL_QJL, rotation: int = TQ_ROTATION_RHT):
+                 residual: int = TQ_RESIDUAL_QJL, rotation: int = TQ_ROTATION_RHT, vq_bits: int = 0):
         seg_bits = tuple(int(b) for b in seg_bits)
         self.d, self.seg_bits, self.m, self.seed, self.device = d, seg_bits, m, seed, device
-        self.residual, self.rotation = residual, rotation
+        self.residual, self.rotation, self.vq_bits = residual, rotation, vq_bits
         spec = tq_spec(d, len(seg_bits), (ctypes.c_int32 * 2)(*(seg_bits + (0,) * (2 - len(seg_bits)))), m, seed,
-                       residual, rotation)
+                       residual, rotation, vq_bits)
         h = ctypes.c_void_p()
         _check(_lib.tq_codec_create(ctypes.byref(spec), device, ctypes.byref(h)), "tq_codec_create")
         self._h = h
@@ -162,6 +163,12 @@ class Codec:
             oc += 1 << b
             ob += (1 << b) - 1
         return S, ds, cl, bl
+
+    def vq_codebook(self) -> np.ndarray:
+        """FibQuant codewords [2^vq_bits, 2] fp32 (z units), host copy."""
+        cb = np.zeros((1 << self.vq_bits, 2), dtype=np.float32)
+        _check(_lib.tq_codec_vq_codebook(self._h, cb.ctypes.data), "tq_codec_vq_codebook")
+        return cb
 
     def rotation_matrix(self) -> np.ndarray:
         """The codec's rotation Pi [d, d] (y = Pi u), host copy."""

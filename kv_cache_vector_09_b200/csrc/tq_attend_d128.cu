@@ -10,6 +10,7 @@ cudaError_t tq_launch_attend_fused(const tq_params& kp, const tq_params& vp, con
                                    int Hkv, int64_t T, float scale, const tq_compressed& K, const tq_compressed& V,
                                    float* partials, int nchunk, cudaStream_t st) {
   if (kp.d != vp.d || kp.m % 32 != 0 || kp.m > 256) return cudaErrorNotSupported;
+  if (kp.vq_bits || vp.vq_bits) return cudaErrorNotSupported;  // FibQuant codes: CUDA-core kernel
   // row starts of 16-byte vector loads
   if ((uintptr_t)K.codes % 16 != 0 || (kp.MS > 0 && (uintptr_t)K.signs % 16 != 0)) return cudaErrorNotSupported;
   switch (kp.d) {

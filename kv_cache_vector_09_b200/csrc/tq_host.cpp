@@ -9,6 +9,8 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <map>
+#include <mutex>
 #include <new>
 #include <string>
 #include <vector>
@@ -273,7 +275,123 @@ static tq_status check_spec(const tq_spec* s) {
   if (s->residual == TQ_RESIDUAL_SIGN && (s->nseg != 1 || s->m != d))
     return tq_fail(TQ_ERR_INVALID_ARG, "TQ_RESIDUAL_SIGN needs one segment and m = d (got nseg %d, m %d)", s->nseg,
                    s->m);
+  if (s->vq_bits < 0 || s->vq_bits > TQ_MAX_VQ_BITS)
+    return tq_fail(TQ_ERR_INVALID_ARG, "vq_bits = %d not in 0..%d", s->vq_bits, TQ_MAX_VQ_BITS);
+  if (s->vq_bits > 0 && (s->nseg != 1 || s->residual != TQ_RESIDUAL_QJL))
+    return tq_fail(TQ_ERR_UNSUPPORTED, "FibQuant codes (vq_bits %d) need nseg = 1 and TQ_RESIDUAL_QJL", s->vq_bits);
   return TQ_OK;
+}
+
+// ------------------------------------------------------- FibQuant, k = 2
+// The codebook of the FibQuant page, sections 2.2 (construction) and 2.1 (the
+// source): the block (z_2j, z_2j+1) of z = sqrt(d) u, u uniform on S^{d-1},
+// has density proportional to (1 - |z|^2 / d)^((d - 4) / 2) on the disc of
+// radius sqrt(d).
+//  - initial codewords: a planar Fibonacci spiral, codeword n at angle
+//    n * g + offset (g the golden angle 2 pi (1 - 1/phi)) and at the radius
+//    where the Bennett-Gersho point density, proportional to the square root of
+//    the block density, has put a fraction (n + 1/2) / N of the codewords:
+//    r_n^2 = d (1 - (1 - (n + 1/2) / N)^(4 / d));
+//  - Lloyd refinement: the expectation over the source is taken on M points
+//    i = 0..M-1 at angle i * g and at the (i + 1/2) / M quantile of the radius
+//    (|z|^2 / d ~ Beta(1, (d - 2) / 2): |z|^2 = d (1 - (1 - (i + 1/2) / M)^(2 / (d - 2))));
+//    every iteration assigns each point to its nearest codeword (ties: lower
+//    index) and moves every codeword with a nonempty cell to the cell's mean;
+//  - restarts r = 0..R-1 turn the spiral by r g / R; the restart with the
+//    least mean distortion is kept (ties: the first).
+// Sums run in point order in double, so the result does not depend on
+// threading; the cache holds one codebook per (vq_bits, d).
+constexpr int kVqPoints = 16384;
+constexpr int kVqIters = 40;
+constexpr int kVqRestarts = 3;
+
+static void fibquant_lloyd(int N, int d, double offset, const std::vector<double>& px, const std::vector<double>& py,
+                           std::vector<double>& cx, std::vector<double>& cy, double* distortion) {
+  const double pi = 3.14159265358979323846;
+  const double g = pi * (3.0 - std::sqrt(5.0));
+  cx.resize(N);
+  cy.resize(N);
+  for (int n = 0; n < N; ++n) {
+    const double r = std::sqrt(d * (1.0 - std::pow(1.0 - (n + 0.5) / N, 4.0 / d)));
+    const double a = n * g + offset;
+    cx[n] = r * std::cos(a);
+    cy[n] = r * std::sin(a);
+  }
+  const size_t M = px.size();
+  std::vector<int> own(M);
+  std::vector<double> sx(N), sy(N);
+  std::vector<long> cnt(N);
+  auto assign = [&]() {
+    for (size_t i = 0; i < M; ++i) {
+      int best = 0;
+      double bd = INFINITY;
+      for (int n = 0; n < N; ++n) {
+        const double dx = px[i] - cx[n], dy = py[i] - cy[n];
+        const double e = dx * dx + dy * dy;
+        if (e < bd) {
+          bd = e;
+          best = n;
+        }
+      }
+      own[i] = best;
+    }
+  };
+  for (int it = 0; it < kVqIters; ++it) {
+    assign();
+    std::fill(sx.begin(), sx.end(), 0.0);
+    std::fill(sy.begin(), sy.end(), 0.0);
+    std::fill(cnt.begin(), cnt.end(), 0L);
+    for (size_t i = 0; i < M; ++i) {
+      sx[own[i]] += px[i];
+      sy[own[i]] += py[i];
+      ++cnt[own[i]];
+    }
+    for (int n = 0; n < N; ++n)
+      if (cnt[n] > 0) {
+        cx[n] = sx[n] / (double)cnt[n];
+        cy[n] = sy[n] / (double)cnt[n];
+      }
+  }
+  assign();
+  double tot = 0.0;
+  for (size_t i = 0; i < M; ++i) {
+    const double dx = px[i] - cx[own[i]], dy = py[i] - cy[own[i]];
+    tot += dx * dx + dy * dy;
+  }
+  *distortion = tot / (double)M;
+}
+
+static const std::vector<float>& fibquant_codebook(int vq_bits, int d) {
+  static std::mutex mu;
+  static std::map<std::pair<int, int>, std::vector<float>> cache;
+  std::lock_guard<std::mutex> lock(mu);
+  std::vector<float>& out = cache[{vq_bits, d}];
+  if (!out.empty()) return out;
+  const double pi = 3.14159265358979323846;
+  const double g = pi * (3.0 - std::sqrt(5.0));
+  std::vector<double> px(kVqPoints), py(kVqPoints);
+  for (int i = 0; i < kVqPoints; ++i) {
+    const double r = std::sqrt(d * (1.0 - std::pow(1.0 - (i + 0.5) / kVqPoints, 2.0 / (d - 2))));
+    const double a = i * g;
+    px[i] = r * std::cos(a);
+    py[i] = r * std::sin(a);
+  }
+  const int N = 1 << vq_bits;
+  double best = INFINITY;
+  std::vector<double> cx, cy;
+  for (int rs = 0; rs < kVqRestarts; ++rs) {
+    double dist = 0.0;
+    fibquant_lloyd(N, d, rs * g / kVqRestarts, px, py, cx, cy, &dist);
+    if (dist < best) {
+      best = dist;
+      out.resize(2 * (size_t)N);
+      for (int n = 0; n < N; ++n) {
+        out[2 * n] = (float)cx[n];
+        out[2 * n + 1] = (float)cy[n];
+      }
+    }
+  }
+  return out;
 }
 
 // Mean residual magnitude mu = E|z - cen[code(z)]| under f_d for a published
@@ -326,7 +444,7 @@ extern "C" tq_status tq_codec_create(const tq_spec* spec, int device, tq_codec**
   p.inv_sqrt_p = (float)(1.0 / std::sqrt((double)p.hblock));
   p.qjl_coef = m > 0 ? (float)(std::sqrt(3.14159265358979323846 / 2.0) / m) : 0.0f;
   int W = 0;
-  for (int s = 0; s < spec->nseg; ++s) {
+  for (int s = 0; s < (spec->vq_bits ? 0 : spec->nseg); ++s) {
     const int bits = spec->seg_bits[s];
     p.bits[s] = bits;
     p.segbase[s] = W;
@@ -351,10 +469,21 @@ extern "C" tq_status tq_codec_create(const tq_spec* spec, int device, tq_codec**
       p.bnd[s][k] = c->bnd_host[s][k];
     }
   }
+  if (spec->vq_bits) {
+    // FibQuant block codes: no scalar tables (bits 0, every boundary +inf)
+    c->spec.seg_bits[0] = 0;
+    p.bits[0] = 0;
+    for (int k = 0; k < TQ_MAX_LEVELS; ++k) p.bnd[0][k] = p.bnd[1][k] = INFINITY;
+    p.vq_bits = spec->vq_bits;
+    p.vq_pw = d / 64;
+    W = p.vq_bits * p.vq_pw;
+    c->vq_host = fibquant_codebook(spec->vq_bits, d);
+    for (float v : c->vq_host) p.cmax = std::max(p.cmax, std::fabs(v));
+  }
   p.W = W;
   // plane-identity coefficients: alpha_t = 2^-b sum_c cen[c] prod_{k in t} s_k(c)
-  p.plane_ok = 1;
-  for (int s = 0; s < spec->nseg; ++s) {
+  p.plane_ok = spec->vq_bits ? 0 : 1;
+  for (int s = 0; s < (spec->vq_bits ? 0 : spec->nseg); ++s) {
     const int bits = spec->seg_bits[s], L = 1 << bits;
     p.nterms[s] = tq_term_count[bits];
     for (int t = 0; t < p.nterms[s]; ++t) {
@@ -452,7 +581,8 @@ extern "C" tq_status tq_codec_create(const tq_spec* spec, int device, tq_codec**
     const size_t o2n = align256(o1n + sizeof(float) * m);
     const size_t oE = align256(o2n + sizeof(float) * m);
     const size_t oH = align256(oE + 16);  // Haar: Pi^T [d][d] fp32 (element (i, j) = Pi_ji)
-    const size_t total = align256(oH + (p.haar ? sizeof(float) * (size_t)d * d : 0));
+    const size_t oV = align256(oH + (p.haar ? sizeof(float) * (size_t)d * d : 0));  // FibQuant codebook
+    const size_t total = align256(oV + sizeof(float) * c->vq_host.size());
     e = cudaMalloc(&c->dev_block, total);
     if (e != cudaSuccess) {
       delete c;
@@ -479,12 +609,15 @@ extern "C" tq_status tq_codec_create(const tq_spec* spec, int device, tq_codec**
         for (int i = 0; i < d; ++i) PiT[(size_t)i * d + j] = (float)c->haar[(size_t)j * d + i];
       e = cudaMemcpy(base + oH, PiT.data(), sizeof(float) * PiT.size(), cudaMemcpyHostToDevice);
     }
+    if (e == cudaSuccess && p.vq_bits)
+      e = cudaMemcpy(base + oV, c->vq_host.data(), sizeof(float) * c->vq_host.size(), cudaMemcpyHostToDevice);
     if (e != cudaSuccess) {
       cudaFree(c->dev_block);
       delete c;
       return cuda_fail(e, "codec upload");
     }
     if (p.haar) p.piT = (const float*)(base + oH);
+    if (p.vq_bits) p.vq_cb = (const float*)(base + oV);
     p.S = (const float*)(base + oS);
     p.St = (const float*)(base + oSt);
     p.s_l1 = (const float*)(base + o1);
@@ -524,6 +657,13 @@ extern "C" tq_status tq_codec_export(const tq_codec* c, float* S, uint32_t* dsig
     if (cen) cen = std::copy(c->cen_host[s].begin(), c->cen_host[s].end(), cen);
     if (bnd) bnd = std::copy(c->bnd_host[s].begin(), c->bnd_host[s].end(), bnd);
   }
+  return TQ_OK;
+}
+
+extern "C" tq_status tq_codec_vq_codebook(const tq_codec* c, float* cb) {
+  if (!c || !cb) return tq_fail(TQ_ERR_INVALID_ARG, "tq_codec_vq_codebook: null argument");
+  if (!c->p.vq_bits) return tq_fail(TQ_ERR_INVALID_ARG, "tq_codec_vq_codebook: the codec has scalar codes");
+  std::copy(c->vq_host.begin(), c->vq_host.end(), cb);
   return TQ_OK;
 }
 
@@ -830,6 +970,7 @@ extern "C" tq_status tq_attend(const tq_codec* kc, const tq_codec* vc, const voi
 // ---------------------------------------------------------------- search
 static tq_status check_search_codec(const tq_codec* c, const char* name) {
   if (c->p.nseg != 1) return tq_fail(TQ_ERR_UNSUPPORTED, "%s: needs one segment (nseg = %d)", name, c->p.nseg);
+  if (c->p.vq_bits) return tq_fail(TQ_ERR_UNSUPPORTED, "%s: needs scalar codes (the codec has FibQuant codes)", name);
   if (c->p.d % 32 != 0 || c->p.d < 64 || c->p.d > 2048)
     return tq_fail(TQ_ERR_UNSUPPORTED, "%s: d = %d (needs a multiple of 32 in [64, 2048])", name, c->p.d);
   if (c->p.m > 512) return tq_fail(TQ_ERR_UNSUPPORTED, "%s: m = %d above 512", name, c->p.m);

@@ -10,6 +10,7 @@
 #include "../../include/tq.h"
 
 #define TQ_MAX_LEVELS 16
+#define TQ_MAX_VQ_BITS 8  // FibQuant k = 2: at most 256 codewords
 #define TQ_MAX_M 1024
 #define TQ_HBLOCK_MAX 512  // longest Hadamard block; longer vectors use blocks
 
@@ -57,6 +58,11 @@ struct tq_params {
   // codec's D signs are all +1
   int haar;
   const float* piT;
+  // FibQuant k = 2 block codes (vq_bits > 0; bits/nseg/cen/bnd unused):
+  // vq_pw words per plane (d / 64), vq_cb [2^vq_bits][2] fp32 in z units
+  int vq_bits;
+  int vq_pw;
+  const float* vq_cb;
   // per-element residual sign (TQ_RESIDUAL_SIGN): rnorms hold this constant
   // instead of ||r|| (0 with the QJL sketch)
   float rnorm_const;
@@ -90,6 +96,7 @@ struct tq_codec {
   std::vector<float> bnd_host[2];
   double mu = 0.0;  // TQ_RESIDUAL_SIGN: mean residual magnitude (z units)
   std::vector<double> haar;  // TQ_ROTATION_HAAR: Pi [d][d] row-major, fp64
+  std::vector<float> vq_host;  // FibQuant codebook [2^vq_bits][2] (z units)
   // device allocations (one block)
   void* dev_block = nullptr;
 };

@@ -11,10 +11,12 @@ namespace {
 constexpr int kQuantWarps = 8;
 constexpr float kUlp = 5.9604644775390625e-08f;  // 2^-24, unit roundoff of fp32
 
-// Copies of the per-segment codebooks in shared memory (indexed per lane).
+// Copies of the per-segment codebooks in shared memory (indexed per lane),
+// and of the FibQuant codewords when the codec has block codes.
 struct SmemBook {
   float cen[2][TQ_MAX_LEVELS];
   float bnd[2][TQ_MAX_LEVELS];
+  float2 vq[1 << TQ_MAX_VQ_BITS];
 };
 
 __device__ __forceinline__ void load_book(const tq_params& p, SmemBook& sb) {
@@ -22,6 +24,42 @@ __device__ __forceinline__ void load_book(const tq_params& p, SmemBook& sb) {
     sb.cen[i / TQ_MAX_LEVELS][i % TQ_MAX_LEVELS] = p.cen[i / TQ_MAX_LEVELS][i % TQ_MAX_LEVELS];
     sb.bnd[i / TQ_MAX_LEVELS][i % TQ_MAX_LEVELS] = p.bnd[i / TQ_MAX_LEVELS][i % TQ_MAX_LEVELS];
   }
+  if (p.vq_bits)
+    for (int i = threadIdx.x; i < (1 << p.vq_bits); i += blockDim.x)
+      sb.vq[i] = make_float2(__ldg(p.vq_cb + 2 * i), __ldg(p.vq_cb + 2 * i + 1));
+}
+
+// FibQuant block codes.  Block j = (z_2j, z_2j+1) sits in lanes 2t and 2t+1
+// at register k (j = 16 k + t); both lanes search the codebook for the block
+// (same operands, same order, hence the same answer).  Returns the nearest
+// codeword (ties: the lower index) and the squared distances to the nearest
+// and second-nearest ones.
+template <typename F>
+__device__ __forceinline__ int vq_nearest(const SmemBook& sb, int N, F za, F zb, F& e1, F& e2) {
+  int best = 0;
+  e1 = F(INFINITY);
+  e2 = F(INFINITY);
+  for (int n = 0; n < N; ++n) {
+    const F dx = za - (F)sb.vq[n].x, dy = zb - (F)sb.vq[n].y;
+    const F e = dx * dx + dy * dy;
+    if (e < e1) {
+      e2 = e1;
+      e1 = e;
+      best = n;
+    } else if (e < e2) {
+      e2 = e;
+    }
+  }
+  return best;
+}
+
+// bits 0, 2, .., 30 of v moved to bits 0..15 (the even lanes of a ballot)
+__device__ __forceinline__ uint32_t even_bits(uint32_t v) {
+  v &= 0x55555555u;
+  v = (v | (v >> 1)) & 0x33333333u;
+  v = (v | (v >> 2)) & 0x0f0f0f0fu;
+  v = (v | (v >> 4)) & 0x00ff00ffu;
+  return (v | (v >> 8)) & 0x0000ffffu;
 }
 
 // =============================================================== quantise
@@ -102,10 +140,33 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
     }
     const float ez0 = kUlp * rot_term;
     int code[VPL];
+    float cval[VPL];  // centroid value of each coordinate (z units)
     bool flag = false;
     float zmax = 0.f;
+    if (p.vq_bits) {
+      // nearest codeword per block; the code is certified when the distances
+      // from the fp32 block to its nearest and second-nearest codewords differ
+      // by more than twice the block's error radius delta (every distance moves
+      // by at most delta between the fp32 and the exact block) plus the fp32
+      // evaluation error of the two distances (below 4.5 u (D1 + D2))
+      const int N = 1 << p.vq_bits;
 #pragma unroll
-    for (int k = 0; k < VPL; ++k) {
+      for (int k = 0; k < VPL; ++k) {
+        const float za = __shfl_sync(TQ_FULL_MASK, z[k], lane & ~1);
+        const float zb = __shfl_sync(TQ_FULL_MASK, z[k], lane | 1);
+        float e1, e2;
+        const int c = vq_nearest<float>(sb, N, za, zb, e1, e2);
+        code[k] = c;
+        cval[k] = (lane & 1) ? sb.vq[c].y : sb.vq[c].x;
+        const float ea = ez0 + 2.f * kUlp * fabsf(za), eb = ez0 + 2.f * kUlp * fabsf(zb);
+        const float delta = 1.01f * sqrtf(ea * ea + eb * eb);
+        const float D1 = sqrtf(e1), D2 = sqrtf(e2);
+        flag |= (D2 - D1) <= 2.f * delta + 8.f * kUlp * (D1 + D2);
+        zmax = fmaxf(zmax, fabsf(z[k]));
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < (p.vq_bits ? 0 : VPL); ++k) {
       const int s = (p.nseg == 2 && k >= VPL / 2) ? 1 : 0;
       const int nb = (1 << p.bits[s]) - 1;
       int c = 0;
@@ -116,6 +177,7 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
         mg = fminf(mg, fabsf(z[k] - bv));
       }
       code[k] = c;
+      cval[k] = sb.cen[s][c];
       flag |= mg <= 1.01f * (ez0 + 2.f * kUlp * fabsf(z[k]));
       zmax = fmaxf(zmax, fabsf(z[k]));
     }
@@ -123,8 +185,7 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
     float g2 = 0.f;
 #pragma unroll
     for (int k = 0; k < VPL; ++k) {
-      const int s = (p.nseg == 2 && k >= VPL / 2) ? 1 : 0;
-      r[k] = (z[k] - sb.cen[s][code[k]]) * p.inv_sqrt_d;
+      r[k] = (z[k] - cval[k]) * p.inv_sqrt_d;
       g2 = fmaf(r[k], r[k], g2);
     }
     g2 = tq_warp_sum(g2);
@@ -175,12 +236,23 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
       double g2d = 0.0;
 #pragma unroll
       for (int k = 0; k < VPL; ++k) {
-        const int s = (p.nseg == 2 && k >= VPL / 2) ? 1 : 0;
-        const int nb = (1 << p.bits[s]) - 1;
-        int c = 0;
-        for (int b = 0; b < nb; ++b) c += (zd[k] >= (double)sb.bnd[s][b]) ? 1 : 0;
-        code[k] = c;
-        const double rv = (zd[k] - (double)sb.cen[s][c]) * isd;
+        double cv;
+        if (p.vq_bits) {
+          const double za = __shfl_sync(TQ_FULL_MASK, zd[k], lane & ~1);
+          const double zb = __shfl_sync(TQ_FULL_MASK, zd[k], lane | 1);
+          double e1, e2;
+          const int c = vq_nearest<double>(sb, 1 << p.vq_bits, za, zb, e1, e2);
+          code[k] = c;
+          cv = (lane & 1) ? (double)sb.vq[c].y : (double)sb.vq[c].x;
+        } else {
+          const int s = (p.nseg == 2 && k >= VPL / 2) ? 1 : 0;
+          const int nb = (1 << p.bits[s]) - 1;
+          int c = 0;
+          for (int b = 0; b < nb; ++b) c += (zd[k] >= (double)sb.bnd[s][b]) ? 1 : 0;
+          code[k] = c;
+          cv = (double)sb.cen[s][c];
+        }
+        const double rv = (zd[k] - cv) * isd;
         rbuf[lane + 32 * k] = rv;
         g2d = fma(rv, rv, g2d);
       }
@@ -201,8 +273,20 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
     uint32_t cw[SLOTS];
 #pragma unroll
     for (int sl = 0; sl < SLOTS; ++sl) cw[sl] = 0;
+    if (p.vq_bits) {
+      // plane pl, word k / 2: blocks 16 k + t (t < 16) at bits 16 (k % 2) + t
 #pragma unroll
-    for (int k = 0; k < VPL; ++k) {
+      for (int k = 0; k < VPL; ++k)
+        for (int pl = 0; pl < p.vq_bits; ++pl) {
+          const uint32_t half = even_bits(__ballot_sync(TQ_FULL_MASK, (code[k] >> pl) & 1));
+          const int widx = pl * p.vq_pw + (k >> 1);
+#pragma unroll
+          for (int sl = 0; sl < SLOTS; ++sl)
+            if (sl == (widx >> 5) && lane == (widx & 31)) cw[sl] |= half << (16 * (k & 1));
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < (p.vq_bits ? 0 : VPL); ++k) {
       const int s = (p.nseg == 2 && k >= VPL / 2) ? 1 : 0;
       const int kk = s ? k - VPL / 2 : k;
       for (int pl = 0; pl < p.bits[s]; ++pl) {
@@ -287,6 +371,28 @@ __global__ void __launch_bounds__(256)
 template <int NG>
 __device__ __forceinline__ void mse_dot(const tq_params& p, const uint32_t* __restrict__ cw, const float* qp,
                                         const SmemBook& sb, float (&acc)[NG]) {
+  if (p.vq_bits) {
+    // FibQuant: block 32w + t's codeword times (q'_2j, q'_2j+1), j = 32w + t
+    for (int w = 0; w < p.vq_pw; ++w) {
+      uint32_t pl[TQ_MAX_VQ_BITS];
+#pragma unroll
+      for (int b = 0; b < TQ_MAX_VQ_BITS; ++b) pl[b] = b < p.vq_bits ? __ldg(cw + b * p.vq_pw + w) : 0u;
+      const float* qrow = qp + (size_t)(64 * w) * NG;
+#pragma unroll 4
+      for (int t = 0; t < 32; ++t) {
+        int c = 0;
+#pragma unroll
+        for (int b = 0; b < TQ_MAX_VQ_BITS; ++b) c |= ((pl[b] >> t) & 1) << b;
+        const float2 v = sb.vq[c];
+#pragma unroll
+        for (int g = 0; g < NG; ++g) {
+          acc[g] = fmaf(v.x, qrow[(2 * t) * NG + g], acc[g]);
+          acc[g] = fmaf(v.y, qrow[(2 * t + 1) * NG + g], acc[g]);
+        }
+      }
+    }
+    return;
+  }
   for (int s = 0; s < p.nseg; ++s) {
     const int bits = p.bits[s];
     for (int w = 0; w < p.pw; ++w) {
@@ -475,16 +581,20 @@ __global__ void __launch_bounds__(kAttThreads)
 #pragma unroll
   for (int g = 0; g < NG; ++g) acc[g] = 0.f;
   if (grp < groups) {
-    const int s = (vp.nseg == 2 && i >= vp.seg_len) ? 1 : 0;
-    const int il = i - s * vp.seg_len;
+    // scalar codes: coordinate i's own code; FibQuant: block i / 2's code,
+    // component i % 2 of its codeword
+    const bool vq = vp.vq_bits != 0;
+    const int s = (!vq && vp.nseg == 2 && i >= vp.seg_len) ? 1 : 0;
+    const int il = vq ? (i >> 1) : i - s * vp.seg_len;
     const int w = il >> 5, bit = il & 31;
-    const int bits = vp.bits[s];
-    const int wbase = vp.segbase[s] + w;
+    const int bits = vq ? vp.vq_bits : vp.bits[s];
+    const int pstride = vq ? vp.vq_pw : vp.pw;
+    const int wbase = (vq ? 0 : vp.segbase[s]) + w;
     for (int64_t t = t0 + grp; t < t1; t += groups) {
       const uint32_t* cw = V.codes + (rowbase + t) * vp.W + wbase;
       int c = 0;
-      for (int pb = 0; pb < bits; ++pb) c |= ((__ldg(cw + pb * vp.pw) >> bit) & 1) << pb;
-      const float v = sbv.cen[s][c];
+      for (int pb = 0; pb < bits; ++pb) c |= ((__ldg(cw + pb * pstride) >> bit) & 1) << pb;
+      const float v = vq ? ((i & 1) ? sbv.vq[c].y : sbv.vq[c].x) : sbv.cen[s][c];
       const float* lr = L + (t - t0) * NG;
 #pragma unroll
       for (int g = 0; g < NG; ++g) acc[g] = fmaf(lr[g], v, acc[g]);

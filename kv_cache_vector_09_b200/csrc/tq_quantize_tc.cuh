@@ -902,6 +902,7 @@ cudaError_t launch_quantize_tc(const tq_params& p, const void* x, tq_dtype dt, i
   if (p.m > 256 || (p.m > 0 && p.m % 32 != 0)) return cudaErrorNotSupported;
   if (dt != TQ_BF16 && dt != TQ_F32) return cudaErrorNotSupported;
   if (p.haar) return cudaErrorNotSupported;  // the dense Haar rotation runs on the CUDA-core encoder
+  if (p.vq_bits) return cudaErrorNotSupported;  // FibQuant block codes: CUDA-core encoder
   if (p.d == 128) {
     return dt == TQ_BF16 ? dispatch_bits<128, __nv_bfloat16, ROPE>(p, x, n, ld, out, st)
                          : dispatch_bits<128, float, ROPE>(p, x, n, ld, out, st);

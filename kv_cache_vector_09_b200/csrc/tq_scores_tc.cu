@@ -793,7 +793,7 @@ size_t tq_scores_tc_bytes(const tq_params& p, int B, int Hq, int Hkv) {
 }
 
 bool tq_scores_tc_supported(const tq_params& p, int Hq, int Hkv) {
-  return Hkv > 0 && Hq % Hkv == 0 && supported(p, Hq / Hkv, nullptr);
+  return Hkv > 0 && Hq % Hkv == 0 && !p.vq_bits && supported(p, Hq / Hkv, nullptr);
 }
 
 cudaError_t tq_launch_scores_tc(const tq_params& p, const float* qprep, int B, int Hq, int Hkv, int64_t T,

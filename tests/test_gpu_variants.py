@@ -1,4 +1,5 @@
-"""Codec variants against the oracle: TurboESM's per-element residual sign.
+"""Codec variants against the oracle: TurboESM's per-element residual sign,
+the dense Haar rotation and FibQuant's k = 2 vector codes.
 
 TurboESM page, "Resumo tecnico" section 2, "Correcao de Residuo QJL de 1
 Bit": one sign bit per element of the quantisation residual, and a
@@ -134,3 +135,84 @@ def test_haar_quantize_scores_attend(d, bits, m):
     oo = O.attend(q.to(torch.float64).numpy(), Ko, Vo, okc, ovc, B, Hq, Hkv, T)
     err = attend_errors(out.cpu().numpy().astype(np.float64), oo)
     assert err.max() <= ATTEND_RTOL, err.max()
+
+
+# ------------------------------------------------------------ FibQuant, k = 2
+# FibQuant page, sections 2.2-2.3: blocks of two rotated coordinates take the
+# nearest of 2^vq_bits shared codewords.  The library's codebook is checked
+# against the oracle's on the host; here the encoder (fp32 with a certified
+# nearest-codeword decision, fp64 for the uncertain rows), the CUDA-core
+# scorer and the attention kernel against the oracle.
+@pytest.mark.parametrize("d,vq_bits,m,dtype", [(128, 5, 128, torch.bfloat16), (64, 4, 64, torch.float32),
+                                               (128, 3, 0, torch.bfloat16), (256, 6, 0, torch.float32)])
+def test_fibquant_quantize_scores_attend(d, vq_bits, m, dtype):
+    B, Hq, Hkv, T = 1, 8, 2, 1100
+    kc = tq.Codec(d, (1,), m, 11, vq_bits=vq_bits)
+    vc = tq.Codec(d, (1,), 0, 12, vq_bits=vq_bits)
+    okc = O.make_codec(d, (1,), m, 11, vq_bits=vq_bits)
+    ovc = O.make_codec(d, (1,), 0, 12, vq_bits=vq_bits)
+    k = synth.heavy_rows(71, B * Hkv * T, d, n_out=2).to(dtype)
+    k[3] = 0
+    v = synth.heavy_rows(72, B * Hkv * T, d, n_out=2).to(dtype)
+    q = synth.gaussian_rows(73, B * Hq, d, dtype=torch.bfloat16).reshape(B, Hq, d) * 2.0
+    K, V = tq.Compressed.empty(kc, B * Hkv * T), tq.Compressed.empty(vc, B * Hkv * T)
+    tq.tq_quantize(kc, k.to(DEV), K)
+    tq.tq_quantize(vc, v.to(DEV), V)
+    torch.cuda.synchronize()
+    assert tq.tq_codec_device_error(kc) == 0 and tq.tq_codec_device_error(vc) == 0
+    Ko = O.quantize(k.to(torch.float64).numpy(), okc)
+    Vo = O.quantize(v.to(torch.float64).numpy(), ovc)
+    print("fibquant K", compare_compressed(K, Ko, okc), "V", compare_compressed(V, Vo, ovc))
+    qg = q.to(DEV).contiguous()
+    ws = tq.workspace(tq.tq_scores_workspace_size(kc, B, Hq, Hkv), DEV)
+    lo = O.estimate_scores(q.to(torch.float64).numpy(), Ko, okc, B, Hq, Hkv, T)
+    nu = Ko.nu64.reshape(B, Hkv, 1, T).repeat(Hq // Hkv, axis=2).reshape(B, Hq, T)
+    qn = np.linalg.norm(q.to(torch.float64).numpy(), axis=-1)[:, :, None]
+    logits = torch.empty((B, Hq, T), device=DEV)
+    tq.tq_scores(kc, qg, B, Hq, Hkv, T, _up(Ko, m), logits, ws)
+    torch.cuda.synchronize()
+    err = logit_errors(logits.cpu().numpy().astype(np.float64), lo, nu, qn, d)
+    assert err.max() <= LOGIT_RTOL, err.max()
+    # attention: FibQuant keys and values, and FibQuant values under scalar keys
+    g = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int32)).to(DEV)
+    Vg = tq.Compressed(g(Vo.codes), None, torch.from_numpy(Vo.norms).to(DEV), None)
+    oo = O.attend(q.to(torch.float64).numpy(), Ko, Vo, okc, ovc, B, Hq, Hkv, T)
+    out = torch.empty((B, Hq, d), device=DEV)
+    tq.tq_attend(kc, vc, qg, B, Hq, Hkv, T, _up(Ko, m), Vg, out,
+                 tq.workspace(tq.tq_attend_workspace_size(kc, vc, B, Hq, Hkv, T), DEV))
+    torch.cuda.synchronize()
+    assert attend_errors(out.cpu().numpy().astype(np.float64), oo).max() <= ATTEND_RTOL
+    sc, osc = tq.Codec(d, (3,), 64, 13), O.make_codec(d, (3,), 64, 13)
+    So = O.quantize(k.to(torch.float64).numpy(), osc)
+    tq.tq_attend(sc, vc, qg, B, Hq, Hkv, T, _up(So, 64), Vg, out,
+                 tq.workspace(tq.tq_attend_workspace_size(sc, vc, B, Hq, Hkv, T), DEV))
+    torch.cuda.synchronize()
+    oo = O.attend(q.to(torch.float64).numpy(), So, Vo, osc, ovc, B, Hq, Hkv, T)
+    assert attend_errors(out.cpu().numpy().astype(np.float64), oo).max() <= ATTEND_RTOL
+
+
+def test_fibquant_unsupported_paths_are_refused():
+    # the top-k search and the fused RoPE encoder take scalar codes only, and
+    # FibQuant values with a sketch have no attention kernel
+    d = 128
+    c = tq.Codec(d, (1,), 64, 0, vq_bits=4)
+    x = synth.gaussian_rows(1, 64, d, dtype=torch.bfloat16).to(DEV)
+    X = tq.Compressed.empty(c, 64)
+    tq.tq_quantize(c, x, X)
+    ws = tq.workspace(1 << 20, DEV)
+    idx = torch.empty((4, 4), dtype=torch.int32, device=DEV)
+    sc = torch.empty((4, 4), dtype=torch.float32, device=DEV)
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_search_topk(c, x[:4].contiguous(), X, 64, 4, idx, sc, ws)
+    assert e.value.status == 2
+    cs = tq.tq_rope_cache(10000.0, d, 16)
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_quantize_rope(c, x, cs, torch.zeros(64, dtype=torch.int32, device=DEV), X)
+    assert e.value.status == 2
+    q = x[:4].reshape(1, 4, d).contiguous()
+    out = torch.empty((1, 4, d), device=DEV)
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_attend(c, c, q, 1, 4, 1, 64, X, X, out, tq.workspace(tq.tq_attend_workspace_size(c, c, 1, 4, 1, 64), DEV))
+    assert e.value.status == 2
+    torch.cuda.synchronize()
+    assert tq.tq_codec_device_error(c) == 0

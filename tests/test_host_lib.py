@@ -179,3 +179,35 @@ def test_haar_rotation_matches_the_oracle():
     assert np.abs(c.rotation_matrix() - O.rotation_matrix(O.rademacher_signs(7, 128))).max() < 1e-7
     with pytest.raises(tq.TQError):
         tq.Codec(512, (3,), 0, 0, device=-1, rotation=tq.TQ_ROTATION_HAAR)
+
+
+@pytest.mark.parametrize("vq_bits,d", [(1, 64), (3, 128), (5, 128), (4, 256), (6, 64)])
+def test_fibquant_codebook_matches_the_oracle(vq_bits, d):
+    # the library's FibQuant construction (C++) against the oracle's (numpy):
+    # both run the same fp64 spiral + Lloyd steps in the same order, so the
+    # fp32 codewords agree to within one rounding
+    c = tq.Codec(d, (1,), 64, 0, device=-1, vq_bits=vq_bits)
+    cb = c.vq_codebook()
+    ob = O.fibquant_codebook(vq_bits, d)
+    assert cb.shape == ob.shape == (1 << vq_bits, 2)
+    assert np.all(np.abs(cb - ob) <= np.spacing(np.abs(ob))), np.abs(cb - ob).max()
+    assert c.code_words == vq_bits * d // 64
+
+
+def test_fibquant_codec_checks():
+    for kw in (dict(vq_bits=9), dict(vq_bits=-1)):
+        with pytest.raises(tq.TQError) as e:
+            tq.Codec(128, (1,), 0, 0, device=-1, **kw)
+        assert e.value.status == 1  # TQ_ERR_INVALID_ARG
+    with pytest.raises(tq.TQError) as e:
+        tq.Codec(128, (2, 3), 0, 0, device=-1, vq_bits=4)
+    assert e.value.status == 2  # TQ_ERR_UNSUPPORTED
+    with pytest.raises(tq.TQError) as e:
+        tq.Codec(128, (1,), 128, 0, device=-1, vq_bits=4, residual=tq.TQ_RESIDUAL_SIGN)
+    assert e.value.status == 2  # TQ_ERR_UNSUPPORTED
+    # a scalar codec has no vector codebook; the search takes scalar codes only
+    with pytest.raises(tq.TQError):
+        tq.Codec(128, (3,), 0, 0, device=-1).vq_codebook()
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_search_workspace_size(tq.Codec(128, (1,), 0, 0, device=-1, vq_bits=4), 8, 4)
+    assert e.value.status == 2  # TQ_ERR_UNSUPPORTED
