@@ -415,6 +415,51 @@ def config_esm_prefill(tq, dev, stream, flush, iters, hbm, peak_src):
             "roofline_rope_fused": hbm_roof(bytes_kv_fused, t_fused, hbm, peak_src)}
 
 
+def config_variants(tq, layer, dev, stream, flush, iters, hbm, peak_src):
+    """The codec variants on one batch element of the Llama-8B layer (8 KV
+    heads x 32768 keys, 32 query heads): tq_quantize of the keys and
+    tq_scores over them, L2 flushed before every call.  Variants: the layer's
+    own key codec (3 bits + QJL m = 128, randomized Hadamard), TurboESM's
+    per-element residual sign (3 bits, S = I), the dense Haar rotation (3 bits
+    + QJL), and FibQuant k = 2 at 2.5 bits per coordinate (32 codewords per
+    2-coordinate block) + QJL."""
+    w = layer.w
+    d, n, Hq, Hkv = w.d, w.Hkv * w.T, w.Hq, w.Hkv
+    k = layer.k[:n]                      # rows (0 * Hkv + h) * T + t: batch element 0
+    q = layer.q[:1].contiguous()
+    logits = torch.empty((1, Hq, w.T), device=dev)
+    specs = {
+        "rht_3bit_qjl128": dict(seg_bits=(3,), m=128),
+        "sign_residual_3bit": dict(seg_bits=(3,), m=d, residual=tq.TQ_RESIDUAL_SIGN),
+        "haar_3bit_qjl128": dict(seg_bits=(3,), m=128, rotation=tq.TQ_ROTATION_HAAR),
+        "fibquant_2p5bit_qjl128": dict(seg_bits=(1,), m=128, vq_bits=5),
+    }
+    out = {"workload": "llama8b_decode, batch element 0", "keys": n, "Hq": Hq, "Hkv": Hkv, "T": w.T,
+           "input_dtype": "bf16", "l2": "256 MB written before every call (outside the timing)"}
+    for name, sp in specs.items():
+        kc = tq.Codec(d, sp["seg_bits"], sp["m"], w.codec_seed, device=dev.index,
+                      residual=sp.get("residual", tq.TQ_RESIDUAL_QJL), rotation=sp.get("rotation", tq.TQ_ROTATION_RHT),
+                      vq_bits=sp.get("vq_bits", 0))
+        K = tq.Compressed.empty(kc, n, dev)
+        ws = tq.workspace(tq.tq_scores_workspace_size(kc, 1, Hq, Hkv), dev)
+        fq = lambda: tq.tq_quantize(kc, k, K)
+        fs = lambda: tq.tq_scores(kc, q, 1, Hq, Hkv, w.T, K, logits, ws)
+        for _ in range(3):
+            fq()
+            fs()
+        mq = statistics.median(timed_calls(fq, iters, stream, flush))
+        ms = statistics.median(timed_calls(fs, iters, stream, flush))
+        if tq.tq_codec_device_error(kc) != 0:
+            raise RuntimeError(f"device error in the {name} variant")
+        krow = 4 * kc.code_words + 4 * kc.sign_words + 8
+        out[name] = {"quantize_ms": round(mq, 5), "scores_ms": round(ms, 5), "key_row_bytes": krow,
+                     "keys_quantised_per_s": n / (mq * 1e-3), "keys_scored_per_s": n / (ms * 1e-3),
+                     "roofline_quantize": hbm_roof(n * (2 * d + krow), mq, hbm, peak_src),
+                     "roofline_scores": hbm_roof(n * (krow + 4 * (Hq // Hkv)), ms, hbm, peak_src)}
+        del K, ws, kc
+    return out
+
+
 def config_vsearch(tq, dev, stream, iters):
     """Vector search over the 1M x 1536 compressed index, top-10 per query,
     with recall@10 against exact fp32 inner products computed on the GPU."""
@@ -504,6 +549,7 @@ def run_configs(tq, layer, dev, stream, iters: int):
     out = {"decode_append_attend": decode_append_step(tq, layer, dev, stream, iters, hbm, peak_src)}
     out["longctx"] = config_longctx(tq, dev, stream, flush, iters, hbm, peak_src)
     out["esm_prefill"] = config_esm_prefill(tq, dev, stream, flush, iters, hbm, peak_src)
+    out["variants"] = config_variants(tq, layer, dev, stream, flush, max(3, iters // 4), hbm, peak_src)
     del flush
     torch.cuda.empty_cache()
     out["vsearch"] = config_vsearch(tq, dev, stream, max(3, iters // 4))

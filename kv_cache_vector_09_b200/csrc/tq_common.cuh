@@ -66,21 +66,32 @@ __device__ __forceinline__ bool tq_dneg(const uint32_t* dbits, int k, int lane) 
 // j = lane + 32 k, k < VPL, d = 32 VPL): v_j <- sum_i Pi_ji v_i with piT
 // [d][d] holding Pi_ji at (i, j), so the lanes' loads at fixed i are
 // coalesced.  buf: d elements of this warp's scratch (shared memory).
+// Each output is four FMA chains over i = c mod 4 (d/4 terms each) added
+// pairwise, (c0 + c1) + (c2 + c3): every product meets at most d/4 + 2
+// roundings, so |error| <= (d/4 + 2) u sum_i |Pi_ji v_i| to first order.
+// Defined for d <= 256 (VPL <= 8), the dense rotations the codecs allow; the
+// longer instantiations are empty and never reached.
 template <int VPL, typename F>
 __device__ __forceinline__ void tq_dense_rotate_warp(F (&v)[VPL], int lane, const float* __restrict__ piT, F* buf) {
+  if constexpr (VPL > 8) return;
   constexpr int d = 32 * VPL;
 #pragma unroll
   for (int k = 0; k < VPL; ++k) buf[lane + 32 * k] = v[k];
   __syncwarp();
-  F acc[VPL];
+  F acc[4][VPL];
 #pragma unroll
-  for (int k = 0; k < VPL; ++k) acc[k] = F(0);
-  for (int i = 0; i < d; ++i) {
-    const F bi = buf[i];
+  for (int c = 0; c < 4; ++c)
 #pragma unroll
-    for (int k = 0; k < VPL; ++k) acc[k] = fma((F)__ldg(piT + (size_t)i * d + lane + 32 * k), bi, acc[k]);
+    for (int k = 0; k < VPL; ++k) acc[c][k] = F(0);
+  for (int i = 0; i < d; i += 4) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const F bi = buf[i + c];
+#pragma unroll
+      for (int k = 0; k < VPL; ++k) acc[c][k] = fma((F)__ldg(piT + (size_t)(i + c) * d + lane + 32 * k), bi, acc[c][k]);
+    }
   }
   __syncwarp();
 #pragma unroll
-  for (int k = 0; k < VPL; ++k) v[k] = acc[k];
+  for (int k = 0; k < VPL; ++k) v[k] = (acc[0][k] + acc[1][k]) + (acc[2][k] + acc[3][k]);
 }

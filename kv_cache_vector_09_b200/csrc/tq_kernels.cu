@@ -30,16 +30,17 @@ __device__ __forceinline__ void load_book(const tq_params& p, SmemBook& sb) {
 }
 
 // FibQuant block codes.  Block j = (z_2j, z_2j+1) sits in lanes 2t and 2t+1
-// at register k (j = 16 k + t); both lanes search the codebook for the block
-// (same operands, same order, hence the same answer).  Returns the nearest
-// codeword (ties: the lower index) and the squared distances to the nearest
-// and second-nearest ones.
+// at register k (j = 16 k + t).  vq_nearest scans codewords [n0, n1) and
+// returns the nearest (ties: the lower index) with the squared distances to
+// the nearest and second-nearest ones; vq_pair_nearest gives each lane of a
+// pair one half of the codebook and merges the halves, so both lanes end with
+// the whole codebook's answer.
 template <typename F>
-__device__ __forceinline__ int vq_nearest(const SmemBook& sb, int N, F za, F zb, F& e1, F& e2) {
-  int best = 0;
+__device__ __forceinline__ int vq_nearest(const SmemBook& sb, int n0, int n1, F za, F zb, F& e1, F& e2) {
+  int best = n0;
   e1 = F(INFINITY);
   e2 = F(INFINITY);
-  for (int n = 0; n < N; ++n) {
+  for (int n = n0; n < n1; ++n) {
     const F dx = za - (F)sb.vq[n].x, dy = zb - (F)sb.vq[n].y;
     const F e = dx * dx + dy * dy;
     if (e < e1) {
@@ -51,6 +52,26 @@ __device__ __forceinline__ int vq_nearest(const SmemBook& sb, int N, F za, F zb,
     }
   }
   return best;
+}
+
+template <typename F>
+__device__ __forceinline__ int vq_pair_nearest(const SmemBook& sb, int N, int lane, F za, F zb, F& e1, F& e2) {
+  const int odd = lane & 1;
+  F a1, a2;
+  const int ia = vq_nearest<F>(sb, odd ? N / 2 : 0, odd ? N : N / 2, za, zb, a1, a2);
+  const F b1 = __shfl_xor_sync(TQ_FULL_MASK, a1, 1), b2 = __shfl_xor_sync(TQ_FULL_MASK, a2, 1);
+  const int ib = __shfl_xor_sync(TQ_FULL_MASK, ia, 1);
+  // (lo1, lo2, ilo): the lower half's results, (hi1, hi2, ihi): the upper's
+  const F lo1 = odd ? b1 : a1, lo2 = odd ? b2 : a2, hi1 = odd ? a1 : b1, hi2 = odd ? a2 : b2;
+  const int ilo = odd ? ib : ia, ihi = odd ? ia : ib;
+  if (lo1 <= hi1) {  // equal distances: the lower index wins
+    e1 = lo1;
+    e2 = lo2 < hi1 ? lo2 : hi1;
+    return ilo;
+  }
+  e1 = hi1;
+  e2 = hi2 < lo1 ? hi2 : lo1;
+  return ihi;
 }
 
 // bits 0, 2, .., 30 of v moved to bits 0..15 (the even lanes of a ballot)
@@ -121,15 +142,17 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
     const float l1u = l1 * inv * 1.001f;  // >= ||u||_1 despite fp32 rounding of the sum
     // rotation error bound of z in units of u = 2^-24: the FWHT sums every
     // input once per stage, so each stage adds at most ||u||_1 (L stages);
-    // the dense Haar product is a d-term FMA chain per output, at most
-    // (d + 2) u sum_i |Pi_ji u_i| <= (d + 2) u ||u||_2, times sqrt(d) for z
+    // the dense Haar product takes at most d/4 + 2 roundings per product
+    // (four chains added pairwise), plus 2 for the scaling by 1/nu, so at
+    // most (d/4 + 4) u sum_i |Pi_ji u_i| <= (d/4 + 4) u ||u||_2, times
+    // sqrt(d) for z
     float rot_term;
     if (p.haar) {
       tq_dense_rotate_warp<VPL>(z, lane, p.piT, rbuf_f);
       const float sd = sqrtf((float)d);
 #pragma unroll
       for (int k = 0; k < VPL; ++k) z[k] *= sd;
-      rot_term = (float)(d + 2) * sd * 1.001f;
+      rot_term = (float)(d / 4 + 4) * sd * 1.001f;
     } else {
       tq_fwht_warp<VPL>(z, lane);
       if (p.zscale != 1.0f) {
@@ -155,7 +178,7 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
         const float za = __shfl_sync(TQ_FULL_MASK, z[k], lane & ~1);
         const float zb = __shfl_sync(TQ_FULL_MASK, z[k], lane | 1);
         float e1, e2;
-        const int c = vq_nearest<float>(sb, N, za, zb, e1, e2);
+        const int c = vq_pair_nearest<float>(sb, N, lane, za, zb, e1, e2);
         code[k] = c;
         cval[k] = (lane & 1) ? sb.vq[c].y : sb.vq[c].x;
         const float ea = ez0 + 2.f * kUlp * fabsf(za), eb = ez0 + 2.f * kUlp * fabsf(zb);
@@ -197,15 +220,51 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
       for (int k = 0; k < VPL; ++k) rbuf_f[lane + 32 * k] = r[k];
       __syncwarp();
       const float er = 1.01f * kUlp * (rot_term + 4.f * zmax + 2.f * p.cmax) * p.inv_sqrt_d;
-      for (int q = 0; q < Q; ++q) {
-        const int col = lane * Q + q;
-        const float* sc = p.St + col;
-        float t = 0.f;
-        for (int i = 0; i < d; ++i) t = fmaf(__ldg(sc + (size_t)i * p.m), rbuf_f[i], t);
-        const float et = 1.01f * (__ldg(p.s_l1 + col) * er + (float)(d + 2) * kUlp * __ldg(p.s_l2 + col) * gamma * 1.01f);
-        flag |= fabsf(t) <= et;
-        const uint32_t wv = __ballot_sync(TQ_FULL_MASK, t >= 0.f);
-        if (lane == q) signword = wv;
+      // sketch rows lane * Q + q: up to eight chains side by side (each one
+      // the same sequential FMA chain over i as alone), then one at a time
+      constexpr int QB = 8;
+      for (int q0 = 0; q0 < Q; q0 += QB) {
+        float t[QB];
+#pragma unroll
+        for (int qq = 0; qq < QB; ++qq) t[qq] = 0.f;
+        const float* sc = p.St + lane * Q + q0;
+        if ((Q & 3) == 0) {
+          // this lane's columns are 16-byte aligned runs (Q, q0 and m are
+          // multiples of 4): one 128-bit load per four chains
+          for (int i = 0; i < d; ++i) {
+            const float ri = rbuf_f[i];
+            const float4* s4 = reinterpret_cast<const float4*>(sc + (size_t)i * p.m);
+#pragma unroll
+            for (int qv = 0; qv < QB / 4; ++qv) {
+              if (q0 + 4 * qv < Q) {
+                const float4 a = __ldg(s4 + qv);
+                t[4 * qv] = fmaf(a.x, ri, t[4 * qv]);
+                t[4 * qv + 1] = fmaf(a.y, ri, t[4 * qv + 1]);
+                t[4 * qv + 2] = fmaf(a.z, ri, t[4 * qv + 2]);
+                t[4 * qv + 3] = fmaf(a.w, ri, t[4 * qv + 3]);
+              }
+            }
+          }
+        } else {
+          for (int i = 0; i < d; ++i) {
+            const float ri = rbuf_f[i];
+#pragma unroll
+            for (int qq = 0; qq < QB; ++qq)
+              if (q0 + qq < Q) t[qq] = fmaf(__ldg(sc + (size_t)i * p.m + qq), ri, t[qq]);
+          }
+        }
+#pragma unroll
+        for (int qq = 0; qq < QB; ++qq) {
+          const int q = q0 + qq;
+          if (q < Q) {
+            const int col = lane * Q + q;
+            const float et =
+                1.01f * (__ldg(p.s_l1 + col) * er + (float)(d + 2) * kUlp * __ldg(p.s_l2 + col) * gamma * 1.01f);
+            flag |= fabsf(t[qq]) <= et;
+            const uint32_t wv = __ballot_sync(TQ_FULL_MASK, t[qq] >= 0.f);
+            if (lane == q) signword = wv;
+          }
+        }
       }
       __syncwarp();
     }
@@ -241,7 +300,7 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
           const double za = __shfl_sync(TQ_FULL_MASK, zd[k], lane & ~1);
           const double zb = __shfl_sync(TQ_FULL_MASK, zd[k], lane | 1);
           double e1, e2;
-          const int c = vq_nearest<double>(sb, 1 << p.vq_bits, za, zb, e1, e2);
+          const int c = vq_pair_nearest<double>(sb, 1 << p.vq_bits, lane, za, zb, e1, e2);
           code[k] = c;
           cv = (lane & 1) ? (double)sb.vq[c].y : (double)sb.vq[c].x;
         } else {
