@@ -55,10 +55,10 @@ STAGE_SOURCES = {
     "tq_attend": ("tq_attend.cuh", "tq_attend_d128.cu", "tq_attend_d64.cu"),
 }
 TRAFFIC = {  # stage: (bytes per launch, sources digest)
-    "tq_quantize_K": (548_016_384 + 136_585_984, "26ada5d12091b490aedbca72de0379a59c1d43f8d2302d4423ebd3492e99b32b"),
-    "tq_quantize_V": (539_167_744 + 124_734_208, "26ada5d12091b490aedbca72de0379a59c1d43f8d2302d4423ebd3492e99b32b"),
-    "tq_scores": (152_448_768 + 20_797_440, "efc9132fa0b5f4277ea303f22773632b626ddac9682ed89271d989a890dca52c"),
-    "tq_attend": (293_933_056 + 6_545_152, "853a0d84650adc29ff6221ba2b913f6880341e9e3376bae69430231e8357d47e"),
+    "tq_quantize_K": (548_033_280 + 136_723_200, "8f8b01cbdec3b6f75605a2f016cbe431c5dc3d414b1361d4eef856f736e3f7b4"),
+    "tq_quantize_V": (539_169_536 + 124_970_752, "8f8b01cbdec3b6f75605a2f016cbe431c5dc3d414b1361d4eef856f736e3f7b4"),
+    "tq_scores": (152_425_216 + 16_209_152, "45348e3cd27d5aa45c98ac4162fe5c1da2a6626e9d4b11afdfe474179f8499e2"),
+    "tq_attend": (294_011_648 + 1_265_408, "6f14879f48fe4937f67c34bdc801060ae9d7e9b9ef2b97183262a81c333d1867"),
 }
 
 
