@@ -216,3 +216,55 @@ def test_fibquant_unsupported_paths_are_refused():
     assert e.value.status == 2
     torch.cuda.synchronize()
     assert tq.tq_codec_device_error(c) == 0
+
+
+@pytest.mark.parametrize("d,vq_bits,m,dtype,n", [(64, 1, 0, torch.float16, 777), (512, 8, 32, torch.bfloat16, 300)])
+def test_fibquant_smallest_and_largest_codebooks(d, vq_bits, m, dtype, n):
+    # N = 2 (0.5 bits per coordinate, two antipodal codewords) with fp16 rows,
+    # and N = 256 (4 bits per coordinate) at d = 512 (eight words per plane,
+    # one sign word per row)
+    c = tq.Codec(d, (1,), m, 21, vq_bits=vq_bits)
+    oc = O.make_codec(d, (1,), m, 21, vq_bits=vq_bits)
+    assert np.array_equal(c.vq_codebook(), oc.vq_cb)
+    x = synth.heavy_rows(81, n, d, n_out=2).to(dtype)
+    x[5] = 0
+    X = tq.Compressed.empty(c, n)
+    tq.tq_quantize(c, x.to(DEV), X)
+    torch.cuda.synchronize()
+    assert tq.tq_codec_device_error(c) == 0
+    Xo = O.quantize(x.to(torch.float64).numpy(), oc)
+    print("fibquant N =", 1 << vq_bits, compare_compressed(X, Xo, oc))
+    B, Hq, Hkv = 1, 4, 1
+    q = synth.gaussian_rows(82, Hq, d, dtype=torch.bfloat16).reshape(B, Hq, d)
+    logits = torch.empty((B, Hq, n), device=DEV)
+    tq.tq_scores(c, q.to(DEV).contiguous(), B, Hq, Hkv, n, _up(Xo, m), logits,
+                 tq.workspace(tq.tq_scores_workspace_size(c, B, Hq, Hkv), DEV))
+    torch.cuda.synchronize()
+    lo = O.estimate_scores(q.to(torch.float64).numpy(), Xo, oc, B, Hq, Hkv, n)
+    qn = np.linalg.norm(q.to(torch.float64).numpy(), axis=-1)[:, :, None]
+    err = logit_errors(logits.cpu().numpy().astype(np.float64), lo, Xo.nu64[None, None, :], qn, d)
+    assert err.max() <= LOGIT_RTOL, err.max()
+
+
+def test_fibquant_append_writes_its_slots():
+    # single-token append of FibQuant keys into slot t of every (b, h) row
+    # block: the slots equal the oracle's codes of those rows, every other
+    # cache row is untouched
+    d, vq_bits, m, rows, T, t = 128, 5, 64, 6, 50, 37
+    c = tq.Codec(d, (1,), m, 5, vq_bits=vq_bits)
+    oc = O.make_codec(d, (1,), m, 5, vq_bits=vq_bits)
+    x = synth.heavy_rows(91, rows, d, n_out=2).to(torch.bfloat16)
+    cache = tq.Compressed.empty(c, rows * T)
+    for a in (cache.codes, cache.signs):
+        a.fill_(-1)
+    cache.norms.fill_(-1.0)
+    cache.rnorms.fill_(-1.0)
+    tq.tq_append(c, x.to(DEV), t, T, cache)
+    torch.cuda.synchronize()
+    assert tq.tq_codec_device_error(c) == 0
+    slots = [r * T + t for r in range(rows)]
+    Xo = O.quantize(x.to(torch.float64).numpy(), oc)
+    print("fibquant append", compare_compressed(cache, Xo, oc, rows=slots))
+    others = np.setdiff1d(np.arange(rows * T), slots)
+    assert np.all(cache.codes.cpu().numpy()[others] == -1)
+    assert np.all(cache.norms.cpu().numpy()[others] == -1.0)
