@@ -639,7 +639,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               __syncwarp();
             }
           }
-          // this round's staging tile is read before the next round writes it
+          // this pass's staging tile is read before the next pass writes it
           if (!(alive = epi_sync())) break;
         }
       }
