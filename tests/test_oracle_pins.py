@@ -899,3 +899,20 @@ def test_fibquant_qjl_estimator_is_unbiased_monte_carlo():
     comp0 = O.quantize(x, c0)
     mse_only = np.linalg.norm(x) * float((q[0, 0] @ c0.Pi.T) @ c0.coord_cen(comp0.code_idx)[0]) / math.sqrt(d)
     assert abs(mse_only - exact) > 10 * se
+
+
+def test_fibquant_d4_block_law_is_uniform_on_the_disc():
+    # at d = 4 the density of (z_1, z_2) is constant on the disc |z| < 2
+    # (exponent (d - 4)/2 = 0): the quasi-Monte-Carlo radii are the uniform
+    # disc's quantiles |z|^2 = 4 (i + 1/2)/M, and the Bennett-Gersho spiral
+    # (density f^(1/2), also uniform) puts codeword n at |z|^2 = 4 (n + 1/2)/N
+    M, N = 1000, 16
+    pts = O.fibquant_source_points(4, M)
+    assert np.allclose((pts ** 2).sum(axis=1), 4.0 * (np.arange(M) + 0.5) / M, rtol=0, atol=1e-12)
+    cb = O.fibquant_init(N, 4)
+    assert np.allclose((cb ** 2).sum(axis=1), 4.0 * (np.arange(N) + 0.5) / N, rtol=0, atol=1e-12)
+    # N = 1 would sit at the mean 0; with N = 2 on a uniform disc Lloyd's
+    # optimum is two antipodal points at 4 rho / (3 pi) (half-disc centroid)
+    cb2 = O.fibquant_codebook.__wrapped__(1, 4, M=16384, iters=40, restarts=3).astype(np.float64)
+    want = 4.0 * 2.0 / (3.0 * math.pi)
+    assert np.allclose(np.linalg.norm(cb2, axis=1), want, rtol=3e-3), (np.linalg.norm(cb2, axis=1), want)
