@@ -11,12 +11,10 @@ namespace {
 constexpr int kQuantWarps = 8;
 constexpr float kUlp = 5.9604644775390625e-08f;  // 2^-24, unit roundoff of fp32
 
-// Copies of the per-segment codebooks in shared memory (indexed per lane),
-// and of the FibQuant codewords when the codec has block codes.
+// Copies of the per-segment codebooks in shared memory (indexed per lane).
 struct SmemBook {
   float cen[2][TQ_MAX_LEVELS];
   float bnd[2][TQ_MAX_LEVELS];
-  float2 vq[1 << TQ_MAX_VQ_BITS];
 };
 
 __device__ __forceinline__ void load_book(const tq_params& p, SmemBook& sb) {
@@ -24,9 +22,19 @@ __device__ __forceinline__ void load_book(const tq_params& p, SmemBook& sb) {
     sb.cen[i / TQ_MAX_LEVELS][i % TQ_MAX_LEVELS] = p.cen[i / TQ_MAX_LEVELS][i % TQ_MAX_LEVELS];
     sb.bnd[i / TQ_MAX_LEVELS][i % TQ_MAX_LEVELS] = p.bnd[i / TQ_MAX_LEVELS][i % TQ_MAX_LEVELS];
   }
+}
+
+// The FibQuant codewords live at the end of a kernel's dynamic shared memory
+// (2^vq_bits float2, sized by the launcher only for codecs with block codes),
+// so that scalar codecs keep their shared-memory budget.
+__host__ __device__ inline size_t vq_table_bytes(const tq_params& p) {
+  return p.vq_bits ? sizeof(float2) * ((size_t)1 << p.vq_bits) : 0;
+}
+
+__device__ __forceinline__ void load_vq(const tq_params& p, float2* vq) {
   if (p.vq_bits)
     for (int i = threadIdx.x; i < (1 << p.vq_bits); i += blockDim.x)
-      sb.vq[i] = make_float2(__ldg(p.vq_cb + 2 * i), __ldg(p.vq_cb + 2 * i + 1));
+      vq[i] = make_float2(__ldg(p.vq_cb + 2 * i), __ldg(p.vq_cb + 2 * i + 1));
 }
 
 // FibQuant block codes.  Block j = (z_2j, z_2j+1) sits in lanes 2t and 2t+1
@@ -36,12 +44,12 @@ __device__ __forceinline__ void load_book(const tq_params& p, SmemBook& sb) {
 // pair one half of the codebook and merges the halves, so both lanes end with
 // the whole codebook's answer.
 template <typename F>
-__device__ __forceinline__ int vq_nearest(const SmemBook& sb, int n0, int n1, F za, F zb, F& e1, F& e2) {
+__device__ __forceinline__ int vq_nearest(const float2* vq, int n0, int n1, F za, F zb, F& e1, F& e2) {
   int best = n0;
   e1 = F(INFINITY);
   e2 = F(INFINITY);
   for (int n = n0; n < n1; ++n) {
-    const F dx = za - (F)sb.vq[n].x, dy = zb - (F)sb.vq[n].y;
+    const F dx = za - (F)vq[n].x, dy = zb - (F)vq[n].y;
     const F e = dx * dx + dy * dy;
     if (e < e1) {
       e2 = e1;
@@ -55,10 +63,10 @@ __device__ __forceinline__ int vq_nearest(const SmemBook& sb, int n0, int n1, F 
 }
 
 template <typename F>
-__device__ __forceinline__ int vq_pair_nearest(const SmemBook& sb, int N, int lane, F za, F zb, F& e1, F& e2) {
+__device__ __forceinline__ int vq_pair_nearest(const float2* vq, int N, int lane, F za, F zb, F& e1, F& e2) {
   const int odd = lane & 1;
   F a1, a2;
-  const int ia = vq_nearest<F>(sb, odd ? N / 2 : 0, odd ? N : N / 2, za, zb, a1, a2);
+  const int ia = vq_nearest<F>(vq, odd ? N / 2 : 0, odd ? N : N / 2, za, zb, a1, a2);
   const F b1 = __shfl_xor_sync(TQ_FULL_MASK, a1, 1), b2 = __shfl_xor_sync(TQ_FULL_MASK, a2, 1);
   const int ib = __shfl_xor_sync(TQ_FULL_MASK, ia, 1);
   // (lo1, lo2, ilo): the lower half's results, (hi1, hi2, ihi): the upper's
@@ -106,7 +114,9 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
                        const tq_compressed out) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   __shared__ SmemBook sb;
+  float2* vqs = reinterpret_cast<float2*>(smem_raw + sizeof(double) * (size_t)kQuantWarps * p.d);
   load_book(p, sb);
+  load_vq(p, vqs);
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int d = p.d;
@@ -178,9 +188,9 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
         const float za = __shfl_sync(TQ_FULL_MASK, z[k], lane & ~1);
         const float zb = __shfl_sync(TQ_FULL_MASK, z[k], lane | 1);
         float e1, e2;
-        const int c = vq_pair_nearest<float>(sb, N, lane, za, zb, e1, e2);
+        const int c = vq_pair_nearest<float>(vqs, N, lane, za, zb, e1, e2);
         code[k] = c;
-        cval[k] = (lane & 1) ? sb.vq[c].y : sb.vq[c].x;
+        cval[k] = (lane & 1) ? vqs[c].y : vqs[c].x;
         const float ea = ez0 + 2.f * kUlp * fabsf(za), eb = ez0 + 2.f * kUlp * fabsf(zb);
         const float delta = 1.01f * sqrtf(ea * ea + eb * eb);
         const float D1 = sqrtf(e1), D2 = sqrtf(e2);
@@ -300,9 +310,9 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
           const double za = __shfl_sync(TQ_FULL_MASK, zd[k], lane & ~1);
           const double zb = __shfl_sync(TQ_FULL_MASK, zd[k], lane | 1);
           double e1, e2;
-          const int c = vq_pair_nearest<double>(sb, 1 << p.vq_bits, lane, za, zb, e1, e2);
+          const int c = vq_pair_nearest<double>(vqs, 1 << p.vq_bits, lane, za, zb, e1, e2);
           code[k] = c;
-          cv = (lane & 1) ? (double)sb.vq[c].y : (double)sb.vq[c].x;
+          cv = (lane & 1) ? (double)vqs[c].y : (double)vqs[c].x;
         } else {
           const int s = (p.nseg == 2 && k >= VPL / 2) ? 1 : 0;
           const int nb = (1 << p.bits[s]) - 1;
@@ -429,7 +439,7 @@ __global__ void __launch_bounds__(256)
 // qp is [d][NG] in shared memory.
 template <int NG>
 __device__ __forceinline__ void mse_dot(const tq_params& p, const uint32_t* __restrict__ cw, const float* qp,
-                                        const SmemBook& sb, float (&acc)[NG]) {
+                                        const SmemBook& sb, const float2* vq, float (&acc)[NG]) {
   if (p.vq_bits) {
     // FibQuant: block 32w + t's codeword times (q'_2j, q'_2j+1), j = 32w + t
     for (int w = 0; w < p.vq_pw; ++w) {
@@ -442,7 +452,7 @@ __device__ __forceinline__ void mse_dot(const tq_params& p, const uint32_t* __re
         int c = 0;
 #pragma unroll
         for (int b = 0; b < TQ_MAX_VQ_BITS; ++b) c |= ((pl[b] >> t) & 1) << b;
-        const float2 v = sb.vq[c];
+        const float2 v = vq[c];
 #pragma unroll
         for (int g = 0; g < NG; ++g) {
           acc[g] = fmaf(v.x, qrow[(2 * t) * NG + g], acc[g]);
@@ -513,8 +523,10 @@ __global__ void __launch_bounds__(kScoreThreads)
   __shared__ SmemBook sb;
   float* qp = reinterpret_cast<float*>(smem_raw);
   float* wq = qp + (size_t)NG * p.d;
+  float2* vqs = reinterpret_cast<float2*>(wq + (size_t)NG * p.m);
   const int b = blockIdx.z, hk = blockIdx.y, G = Hq / Hkv;
   load_book(p, sb);
+  load_vq(p, vqs);
   load_queries<NG>(p, qprep, b, Hq, hk, G, qp, wq);
   __syncthreads();
   const int64_t t0 = (int64_t)blockIdx.x * kScoreTile;
@@ -524,7 +536,7 @@ __global__ void __launch_bounds__(kScoreThreads)
     float acc[NG], acc2[NG];
 #pragma unroll
     for (int g = 0; g < NG; ++g) acc[g] = acc2[g] = 0.f;
-    mse_dot<NG>(p, K.codes + row * p.W, qp, sb, acc);
+    mse_dot<NG>(p, K.codes + row * p.W, qp, sb, vqs, acc);
     float gam = 0.f;
     if (p.m > 0) {
       qjl_dot<NG>(p, K.signs + row * p.MS, wq, acc2);
@@ -561,10 +573,16 @@ __global__ void __launch_bounds__(kAttThreads)
   float* wq = qp + (size_t)NG * d;
   float* L = wq + (size_t)NG * kp.m;                  // [chunk_len][NG]
   float* accbuf = L + (size_t)chunk_len * NG;         // [groups][d][NG]
+  // FibQuant codewords of the keys, then of the values, 8-byte aligned
+  const size_t vq_off = ((size_t)(accbuf - qp) + (size_t)(kAttThreads / d) * d * NG + 1) & ~(size_t)1;
+  float2* vqk = reinterpret_cast<float2*>(qp + vq_off);
+  float2* vqv = vqk + (kp.vq_bits ? (1 << kp.vq_bits) : 0);
   const int b = blockIdx.z, hk = blockIdx.y, G = Hq / Hkv, chunk = blockIdx.x;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   load_book(kp, sbk);
   load_book(vp, sbv);
+  load_vq(kp, vqk);
+  load_vq(vp, vqv);
   load_queries<NG>(kp, qprep, b, Hq, hk, G, qp, wq);
   __syncthreads();
   const int64_t t0 = (int64_t)chunk * chunk_len;
@@ -580,7 +598,7 @@ __global__ void __launch_bounds__(kAttThreads)
     float acc[NG], acc2[NG];
 #pragma unroll
     for (int g = 0; g < NG; ++g) acc[g] = acc2[g] = 0.f;
-    mse_dot<NG>(kp, K.codes + row * kp.W, qp, sbk, acc);
+    mse_dot<NG>(kp, K.codes + row * kp.W, qp, sbk, vqk, acc);
     float gam = 0.f;
     if (kp.m > 0) {
       qjl_dot<NG>(kp, K.signs + row * kp.MS, wq, acc2);
@@ -653,7 +671,7 @@ __global__ void __launch_bounds__(kAttThreads)
       const uint32_t* cw = V.codes + (rowbase + t) * vp.W + wbase;
       int c = 0;
       for (int pb = 0; pb < bits; ++pb) c |= ((__ldg(cw + pb * pstride) >> bit) & 1) << pb;
-      const float v = vq ? ((i & 1) ? sbv.vq[c].y : sbv.vq[c].x) : sbv.cen[s][c];
+      const float v = vq ? ((i & 1) ? vqv[c].y : vqv[c].x) : sbv.cen[s][c];
       const float* lr = L + (t - t0) * NG;
 #pragma unroll
       for (int g = 0; g < NG; ++g) acc[g] = fmaf(lr[g], v, acc[g]);
@@ -769,7 +787,7 @@ cudaError_t set_smem(Fn* fn, size_t bytes) {
 template <int VPL, typename TIn>
 cudaError_t launch_quantize_t(const tq_params& p, const void* x, int64_t n, int64_t ld, const tq_compressed& out,
                               cudaStream_t st) {
-  const size_t smem = sizeof(double) * (size_t)kQuantWarps * p.d;
+  const size_t smem = sizeof(double) * (size_t)kQuantWarps * p.d + vq_table_bytes(p);
   auto fn = tq_quantize_kernel<VPL, TIn>;
   cudaError_t e = set_smem(fn, smem);
   if (e != cudaSuccess) return e;
@@ -819,7 +837,7 @@ int padded_groups(int G) {
 template <int NG>
 cudaError_t launch_scores_g(const tq_params& p, const float* qprep, int B, int Hq, int Hkv, int64_t T,
                             const tq_compressed& K, float* logits, cudaStream_t st) {
-  const size_t smem = sizeof(float) * (size_t)NG * (p.d + p.m);
+  const size_t smem = sizeof(float) * (size_t)NG * (p.d + p.m) + vq_table_bytes(p);
   auto fn = tq_scores_kernel<NG>;
   cudaError_t e = set_smem(fn, smem);
   if (e != cudaSuccess) return e;
@@ -836,7 +854,8 @@ cudaError_t launch_attend_g(const tq_params& kp, const tq_params& vp, const floa
                             int nchunk, cudaStream_t st) {
   const int chunk_len = attend_chunk_len(B, Hkv, T, nchunk);
   const int groups = kAttThreads / kp.d;
-  const size_t smem = sizeof(float) * ((size_t)NG * (kp.d + kp.m) + (size_t)chunk_len * NG + (size_t)groups * kp.d * NG);
+  const size_t floats = (size_t)NG * (kp.d + kp.m) + (size_t)chunk_len * NG + (size_t)groups * kp.d * NG;
+  const size_t smem = sizeof(float) * ((floats + 1) & ~(size_t)1) + vq_table_bytes(kp) + vq_table_bytes(vp);
   auto fn = tq_attend_kernel<NG>;
   cudaError_t e = set_smem(fn, smem);
   if (e != cudaSuccess) return e;
