@@ -268,3 +268,41 @@ def test_fibquant_append_writes_its_slots():
     others = np.setdiff1d(np.arange(rows * T), slots)
     assert np.all(cache.codes.cpu().numpy()[others] == -1)
     assert np.all(cache.norms.cpu().numpy()[others] == -1.0)
+
+
+def test_haar_with_fibquant_codes():
+    # the FibQuant page's own pipeline: norm, shared Haar rotation, k = 2
+    # vector codes (plus the QJL stage here); values Haar + FibQuant, m = 0
+    d, vq_bits, m = 128, 4, 64
+    B, Hq, Hkv, T = 1, 4, 1, 900
+    kc = tq.Codec(d, (1,), m, 31, rotation=HAAR, vq_bits=vq_bits)
+    vc = tq.Codec(d, (1,), 0, 32, rotation=HAAR, vq_bits=vq_bits)
+    okc = O.make_codec(d, (1,), m, 31, rotation="haar", vq_bits=vq_bits)
+    ovc = O.make_codec(d, (1,), 0, 32, rotation="haar", vq_bits=vq_bits)
+    k = synth.heavy_rows(101, T, d, n_out=2).to(torch.bfloat16)
+    v = synth.heavy_rows(102, T, d, n_out=2).to(torch.bfloat16)
+    q = synth.gaussian_rows(103, Hq, d, dtype=torch.bfloat16).reshape(B, Hq, d) * 2.0
+    K, V = tq.Compressed.empty(kc, T), tq.Compressed.empty(vc, T)
+    tq.tq_quantize(kc, k.to(DEV), K)
+    tq.tq_quantize(vc, v.to(DEV), V)
+    torch.cuda.synchronize()
+    assert tq.tq_codec_device_error(kc) == 0 and tq.tq_codec_device_error(vc) == 0
+    Ko = O.quantize(k.to(torch.float64).numpy(), okc)
+    Vo = O.quantize(v.to(torch.float64).numpy(), ovc)
+    print("haar + fibquant K", compare_compressed(K, Ko, okc), "V", compare_compressed(V, Vo, ovc))
+    qg = q.to(DEV).contiguous()
+    logits = torch.empty((B, Hq, T), device=DEV)
+    tq.tq_scores(kc, qg, B, Hq, Hkv, T, _up(Ko, m), logits, tq.workspace(tq.tq_scores_workspace_size(kc, B, Hq, Hkv), DEV))
+    torch.cuda.synchronize()
+    lo = O.estimate_scores(q.to(torch.float64).numpy(), Ko, okc, B, Hq, Hkv, T)
+    qn = np.linalg.norm(q.to(torch.float64).numpy(), axis=-1)[:, :, None]
+    err = logit_errors(logits.cpu().numpy().astype(np.float64), lo, Ko.nu64[None, None, :], qn, d)
+    assert err.max() <= LOGIT_RTOL, err.max()
+    g = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int32)).to(DEV)
+    Vg = tq.Compressed(g(Vo.codes), None, torch.from_numpy(Vo.norms).to(DEV), None)
+    out = torch.empty((B, Hq, d), device=DEV)
+    tq.tq_attend(kc, vc, qg, B, Hq, Hkv, T, _up(Ko, m), Vg, out,
+                 tq.workspace(tq.tq_attend_workspace_size(kc, vc, B, Hq, Hkv, T), DEV))
+    torch.cuda.synchronize()
+    oo = O.attend(q.to(torch.float64).numpy(), Ko, Vo, okc, ovc, B, Hq, Hkv, T)
+    assert attend_errors(out.cpu().numpy().astype(np.float64), oo).max() <= ATTEND_RTOL
